@@ -1,0 +1,138 @@
+"""CPU oracle for the ROSA retrieval step -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA path
+(``suffix_automaton_retrieval_b200``) and never imports it.
+
+The arithmetic lives in ``rosa_oracle.c`` (plain C, compiled here with gcc);
+this module only marshals numpy arrays.  Citations are to "ROSA-Tuning:
+Enhancing Windowed Attention with Global Recall" (arXiv 2602.02499):
+
+* ``discretize`` -- section 3.2, Eqs. (10)-(15); section 4.1 (R = C / M).
+* ``match_brute`` -- the definition of the retrieval destination, section 3.3
+  Eq. (16) and appendix B.3, written out as an O(T^2) longest-common-suffix
+  recurrence.
+* ``match_sam`` -- the online suffix automaton of section 2.2 run in lockstep
+  with the query stream (appendix B.3: tau = endpos + 1).
+* ``gather`` -- appendix C.4 read-out at tau with the Eq. (17) mask.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rosa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``rosa_oracle.c`` into ``liboracle.so`` (gcc, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        c_int = ctypes.c_int
+        lib.oracle_discretize.argtypes = [u16p, c_int, c_int, c_int, c_int, u8p]
+        lib.oracle_match_brute.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p]
+        lib.oracle_match_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
+        lib.oracle_gather.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, i32p,
+                                      c_int, c_int, c_int, c_int, u16p]
+        for f in (lib.oracle_discretize, lib.oracle_match_brute, lib.oracle_match_sam, lib.oracle_gather):
+            f.restype = c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def discretize(x_bits: np.ndarray, M: int) -> np.ndarray:
+    """bf16 bit patterns ``[B, T, C]`` (uint16) -> uint8 symbols ``[B, C//M, T]``."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    B, T, C = x_bits.shape
+    if M < 1 or M > 8 or C % M:
+        raise ValueError("need 1 <= M <= 8 and C % M == 0")
+    out = np.empty((B, C // M, T), dtype=np.uint8)
+    _check(_load().oracle_discretize(_ptr(x_bits, ctypes.c_uint16), B, T, C, M,
+                                     _ptr(out, ctypes.c_uint8)), "discretize")
+    return out
+
+
+def _match(fn: str, q, k, v, g, threads=None):
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    k = np.ascontiguousarray(k, dtype=np.uint8)
+    if q.ndim == 1:
+        q, k = q[None], k[None]
+        if v is not None:
+            v = np.asarray(v)[None]
+    S, T = q.shape
+    if k.shape != (S, T):
+        raise ValueError("q and k must have the same shape [S, T]")
+    v = k if v is None else np.ascontiguousarray(v, dtype=np.uint8)
+    if v.shape != (S, T):
+        raise ValueError("v must have shape [S, T]")
+    end = np.empty((S, T), np.int32)
+    ln = np.empty((S, T), np.int32)
+    sym = np.empty((S, T), np.int32)
+    lib = _load()
+    args = [_ptr(q, ctypes.c_uint8), _ptr(k, ctypes.c_uint8), _ptr(v, ctypes.c_uint8), S, T, g,
+            _ptr(end, ctypes.c_int32), _ptr(ln, ctypes.c_int32), _ptr(sym, ctypes.c_int32)]
+    if fn == "sam":
+        args.append(threads if threads else (os.cpu_count() or 1))
+        _check(lib.oracle_match_sam(*args), "match_sam")
+    else:
+        _check(lib.oracle_match_brute(*args), "match_brute")
+    return end, ln, sym
+
+
+def match_brute(q, k, v=None, g: int = 2):
+    """Definition-level matcher, O(T^2) per stream.  Returns (end_idx, len, sym)."""
+    return _match("brute", q, k, v, g)
+
+
+def match_sam(q, k, v=None, g: int = 2, threads: int | None = None):
+    """Online suffix-automaton matcher over host threads.  Returns (end_idx, len, sym)."""
+    return _match("sam", q, k, v, g, threads)
+
+
+def gather(V_bits: np.ndarray, end_idx: np.ndarray, R: int, d: int, rho: int) -> np.ndarray:
+    """Row read-out at tau = end_idx + 1.
+
+    ``V_bits``: ``[B, T, Cv]`` uint16 (bf16 bits); route r reads columns
+    ``r*rho .. r*rho + d``.  ``end_idx``: ``[B*R, T]`` int32.
+    Returns ``[B, T, R*d]`` uint16, zero rows where end_idx = -1.
+    """
+    V_bits = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    end_idx = np.ascontiguousarray(end_idx, dtype=np.int32)
+    B, T, Cv = V_bits.shape
+    if end_idx.shape != (B * R, T):
+        raise ValueError("end_idx must be [B*R, T]")
+    if (R - 1) * rho + d > Cv:
+        raise ValueError("route slice exceeds the V row")
+    out = np.empty((B, T, R * d), np.uint16)
+    _check(_load().oracle_gather(_ptr(V_bits, ctypes.c_uint16), Cv, rho, _ptr(end_idx, ctypes.c_int32),
+                                 B, R, T, d, _ptr(out, ctypes.c_uint16)), "gather")
+    return out

@@ -1,0 +1,387 @@
+/*
+ * CPU oracle for the ROSA retrieval step -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * may load this file's library.  It shares no code, header, table or helper
+ * with the CUDA path and is deliberately plain and slow.
+ *
+ * Source: "ROSA-Tuning: Enhancing Windowed Attention with Global Recall"
+ * (arXiv 2602.02499), the pages cited below by section / equation:
+ *
+ *   section 3.2, Eqs. (10)-(15)   binary discretisation q_bit = I[q_vec > 0]
+ *                                  and multi-route packing a = sum_j bit_(r,j) 2^j
+ *   section 4.1                    routes of M consecutive channels, R = C / M
+ *   section 3.3, Eq. (16)          retrieval destination tau in {-1, 0, .., t-1}
+ *                                  from k_{1:t} and q_{1:t}, read strictly from
+ *                                  the past
+ *   section 2.2                    suffix automaton: <= 2n-1 states, amortised
+ *                                  O(1) transitions and suffix-link jumps
+ *   appendix B.3                   tau_t = endpos(s_t) + 1 when it exists, else -1
+ *   appendix C.4, Eq. (17)         read-out of the value at tau, mask I[tau >= 0]
+ *
+ * Readings taken where the pages are garbled or silent (Eq. 16 itself is lost
+ * in the page text):
+ *   - causal lag g >= 1: a key end i is admissible at query time t iff
+ *     i <= t - g; the default g = 2 gives tau = i + 1 <= t - 1, the range the
+ *     section 3.3 text keeps; the restriction applies before maximising.
+ *   - among admissible ends with the maximal match length, the most recent
+ *     (largest) i is taken.
+ *   - a match of length 0 never counts: tau = -1, len = 0, sym = -1.
+ *   - the recalled symbol is v[i + 1] (v defaults to the key stream k).
+ *
+ * Two matchers are given.  oracle_match_brute is the definition written out
+ * (O(T^2) per stream).  oracle_match_sam is the method the pages name: an
+ * online suffix automaton over the key stream, advanced in lockstep with the
+ * query stream.  The two share nothing but the output convention.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <pthread.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_NOMEM 2
+
+/* ------------------------------------------------------------------------ */
+/* Discretisation: section 3.2, Eqs. (10)-(15); section 4.1 route layout.    */
+/* ------------------------------------------------------------------------ */
+
+static float bf16_bits_to_float(uint16_t h)
+{
+    uint32_t w = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return f;
+}
+
+/*
+ * x: bf16 bit patterns, shape [B, T, C] row-major.
+ * sym: uint8 output, shape [B, R, T] with R = C / M.
+ * Channel c = r * M + j carries bit j (weight 2^j) of route r's symbol.
+ */
+int oracle_discretize(const uint16_t *x, int B, int T, int C, int M, uint8_t *sym)
+{
+    if (B < 0 || T < 0 || C < 1 || M < 1 || M > 8 || C % M != 0)
+        return ORACLE_ERR_ARG;
+    int R = C / M;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int r = 0; r < R; ++r) {
+                unsigned a = 0;
+                for (int j = 0; j < M; ++j) {
+                    float xv = bf16_bits_to_float(x[((size_t)b * T + t) * C + (size_t)r * M + j]);
+                    unsigned bit = (xv > 0.0f) ? 1u : 0u;   /* I[x > 0] */
+                    a += bit << j;                            /* bit * 2^j */
+                }
+                sym[((size_t)b * R + r) * T + t] = (uint8_t)a;
+            }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Matching by the definition (brute force).                                 */
+/*                                                                           */
+/* D(t, i) = q[t] == k[i] ? 1 + D(t-1, i-1) : 0   (D = 0 off the grid) is    */
+/* the length of the longest common suffix of q[0..t] and k[0..i].           */
+/* L_t = max over 0 <= i <= t-g of D(t, i); i*_t = largest such i with       */
+/* D(t, i) = L_t when L_t > 0.                                               */
+/* ------------------------------------------------------------------------ */
+
+static int brute_stream(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                        int T, int g, int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    int32_t *prev = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));
+    int32_t *cur = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));
+    if (!prev || !cur) { free(prev); free(cur); return ORACLE_ERR_NOMEM; }
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < T; ++i) {
+            if (q[t] == k[i])
+                cur[i] = 1 + ((t > 0 && i > 0) ? prev[i - 1] : 0);
+            else
+                cur[i] = 0;
+        }
+        int best = 0, best_i = -1;
+        for (int i = 0; i <= t - g; ++i) {
+            if (cur[i] > 0 && cur[i] >= best) {   /* ">=": later i wins ties */
+                best = cur[i];
+                best_i = i;
+            }
+        }
+        end_idx[t] = best_i;
+        len[t] = best;
+        sym[t] = (best_i >= 0) ? (int32_t)v[best_i + 1] : -1;
+        int32_t *tmp = prev; prev = cur; cur = tmp;
+    }
+    free(prev);
+    free(cur);
+    return ORACLE_OK;
+}
+
+int oracle_match_brute(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                       int S, int T, int g,
+                       int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    if (S < 0 || T < 0 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    if (!v) v = k;
+    for (int s = 0; s < S; ++s) {
+        size_t o = (size_t)s * T;
+        int rc = brute_stream(q + o, k + o, v + o, T, g, end_idx + o, len + o, sym + o);
+        if (rc) return rc;
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Matching with an online suffix automaton (section 2.2; appendix B.3).      */
+/*                                                                           */
+/* State fields: len (longest string of the state), link (suffix link),      */
+/* last_end (largest end position, among the keys inserted so far, of the     */
+/* strings of the state), and a singly linked list of outgoing transitions.  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t *len, *link, *last_end, *edge_head;   /* per state */
+    int32_t *edge_next, *edge_to;                 /* per edge */
+    uint8_t *edge_sym;
+    int n_states, n_edges, cap_states, cap_edges;
+    int last;                                     /* state of the whole key prefix */
+} sam_t;
+
+static int sam_init(sam_t *a, int T)
+{
+    a->cap_states = 2 * T + 2;      /* <= 2n - 1 states, plus the root */
+    a->cap_edges = 3 * T + 4;       /* <= 3n - 4 transitions for n >= 3 */
+    a->len = (int32_t *)malloc(sizeof(int32_t) * a->cap_states);
+    a->link = (int32_t *)malloc(sizeof(int32_t) * a->cap_states);
+    a->last_end = (int32_t *)malloc(sizeof(int32_t) * a->cap_states);
+    a->edge_head = (int32_t *)malloc(sizeof(int32_t) * a->cap_states);
+    a->edge_next = (int32_t *)malloc(sizeof(int32_t) * a->cap_edges);
+    a->edge_to = (int32_t *)malloc(sizeof(int32_t) * a->cap_edges);
+    a->edge_sym = (uint8_t *)malloc(a->cap_edges);
+    if (!a->len || !a->link || !a->last_end || !a->edge_head ||
+        !a->edge_next || !a->edge_to || !a->edge_sym)
+        return ORACLE_ERR_NOMEM;
+    a->n_states = 1;
+    a->n_edges = 0;
+    a->len[0] = 0;
+    a->link[0] = -1;
+    a->last_end[0] = -1;
+    a->edge_head[0] = -1;
+    a->last = 0;
+    return ORACLE_OK;
+}
+
+static void sam_free(sam_t *a)
+{
+    free(a->len); free(a->link); free(a->last_end); free(a->edge_head);
+    free(a->edge_next); free(a->edge_to); free(a->edge_sym);
+}
+
+/* Target of the transition (s, c), or -1. */
+static int sam_get(const sam_t *a, int s, uint8_t c)
+{
+    for (int e = a->edge_head[s]; e >= 0; e = a->edge_next[e])
+        if (a->edge_sym[e] == c) return a->edge_to[e];
+    return -1;
+}
+
+/* Set (s, c) -> to, adding the edge if missing. */
+static int sam_set(sam_t *a, int s, uint8_t c, int to)
+{
+    for (int e = a->edge_head[s]; e >= 0; e = a->edge_next[e])
+        if (a->edge_sym[e] == c) { a->edge_to[e] = to; return ORACLE_OK; }
+    if (a->n_edges >= a->cap_edges) return ORACLE_ERR_NOMEM;
+    int e = a->n_edges++;
+    a->edge_sym[e] = c;
+    a->edge_to[e] = to;
+    a->edge_next[e] = a->edge_head[s];
+    a->edge_head[s] = e;
+    return ORACLE_OK;
+}
+
+/*
+ * Append key symbol c, which sits at key position p (Blumer et al.'s online
+ * construction), then record p as the most recent end of every state whose
+ * strings are suffixes of k[0..p]: those are the states on the suffix-link
+ * path from the new state up to (not including) the root.
+ */
+static int sam_extend(sam_t *a, uint8_t c, int p)
+{
+    if (a->n_states + 2 > a->cap_states) return ORACLE_ERR_NOMEM;
+    int cur = a->n_states++;
+    a->len[cur] = a->len[a->last] + 1;
+    a->link[cur] = 0;
+    a->last_end[cur] = p;
+    a->edge_head[cur] = -1;
+    int x = a->last;
+    while (x != -1 && sam_get(a, x, c) < 0) {
+        if (sam_set(a, x, c, cur)) return ORACLE_ERR_NOMEM;
+        x = a->link[x];
+    }
+    if (x != -1) {
+        int y = sam_get(a, x, c);
+        if (a->len[x] + 1 == a->len[y]) {
+            a->link[cur] = y;
+        } else {
+            int cl = a->n_states++;
+            a->len[cl] = a->len[x] + 1;
+            a->link[cl] = a->link[y];
+            a->last_end[cl] = a->last_end[y];
+            a->edge_head[cl] = -1;
+            for (int e = a->edge_head[y]; e >= 0; e = a->edge_next[e])
+                if (sam_set(a, cl, a->edge_sym[e], a->edge_to[e])) return ORACLE_ERR_NOMEM;
+            while (x != -1 && sam_get(a, x, c) == y) {
+                if (sam_set(a, x, c, cl)) return ORACLE_ERR_NOMEM;
+                x = a->link[x];
+            }
+            a->link[y] = cl;
+            a->link[cur] = cl;
+        }
+    }
+    a->last = cur;
+    for (int s = cur; s > 0; s = a->link[s])
+        a->last_end[s] = p;
+    return ORACLE_OK;
+}
+
+/*
+ * One stream, in lockstep over t = 0..T-1:
+ *   1. if t - g >= 0, insert key symbol k[t-g] (the automaton then holds
+ *      exactly the admissible keys k[0..t-g]);
+ *   2. advance the matching state (state, L) with query symbol q[t]: follow
+ *      suffix links until a transition on q[t] exists (or the root is left
+ *      without one), then take it;
+ *   3. emit (last_end(state), L) when L > 0.
+ *
+ * A clone made by step 1 may take over the shorter strings of the state the
+ * matcher stands in.  Until the next insertion the clone has exactly the
+ * transitions of that state and is its suffix link, so step 2 reaches the
+ * same result from either: a missing transition leads through the clone to
+ * the same suffix-link chain, a present one to the same target.
+ */
+static int sam_stream(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                      int T, int g, int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    sam_t a;
+    int rc = sam_init(&a, T);
+    if (rc) { sam_free(&a); return rc; }
+    int st = 0, L = 0;
+    for (int t = 0; t < T; ++t) {
+        int p = t - g;
+        if (p >= 0) {
+            rc = sam_extend(&a, k[p], p);
+            if (rc) { sam_free(&a); return rc; }
+        }
+        uint8_t c = q[t];
+        while (st != 0 && sam_get(&a, st, c) < 0) {
+            st = a.link[st];
+            L = a.len[st];
+        }
+        int nx = sam_get(&a, st, c);
+        if (nx >= 0) {
+            st = nx;
+            L += 1;
+        } else {
+            st = 0;
+            L = 0;
+        }
+        if (L > 0) {
+            int i = a.last_end[st];
+            end_idx[t] = i;
+            len[t] = L;
+            sym[t] = (int32_t)v[i + 1];
+        } else {
+            end_idx[t] = -1;
+            len[t] = 0;
+            sym[t] = -1;
+        }
+    }
+    sam_free(&a);
+    return ORACLE_OK;
+}
+
+typedef struct {
+    const uint8_t *q, *k, *v;
+    int S, T, g, nthreads, tid;
+    int32_t *end_idx, *len, *sym;
+    int rc;
+} sam_job_t;
+
+static void *sam_worker(void *arg)
+{
+    sam_job_t *j = (sam_job_t *)arg;
+    j->rc = ORACLE_OK;
+    for (int s = j->tid; s < j->S; s += j->nthreads) {
+        size_t o = (size_t)s * j->T;
+        int rc = sam_stream(j->q + o, j->k + o, j->v + o, j->T, j->g,
+                            j->end_idx + o, j->len + o, j->sym + o);
+        if (rc) { j->rc = rc; break; }
+    }
+    return NULL;
+}
+
+/* All S streams ([S, T] row-major), streams spread over nthreads threads. */
+int oracle_match_sam(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                     int S, int T, int g,
+                     int32_t *end_idx, int32_t *len, int32_t *sym, int nthreads)
+{
+    if (S < 0 || T < 0 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    if (!v) v = k;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > S) nthreads = S > 0 ? S : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    sam_job_t *jobs = (sam_job_t *)malloc(sizeof(sam_job_t) * nthreads);
+    if (!th || !jobs) { free(th); free(jobs); return ORACLE_ERR_NOMEM; }
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        sam_job_t jb = {q, k, v, S, T, g, nthreads, i, end_idx, len, sym, 0};
+        jobs[i] = jb;
+        if (i == 0) continue;
+        if (pthread_create(&th[i], NULL, sam_worker, &jobs[i]) != 0) break;
+        started = i;
+    }
+    sam_worker(&jobs[0]);
+    int rc = jobs[0].rc;
+    for (int i = 1; i <= started; ++i) {
+        pthread_join(th[i], NULL);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    /* streams of threads that failed to start are done here */
+    for (int i = started + 1; i < nthreads; ++i) {
+        sam_worker(&jobs[i]);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    free(th);
+    free(jobs);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Read-out of the value rows at tau (appendix C.4; mask of Eq. 17).         */
+/*                                                                           */
+/* out[b, t, r*d + m] = V[b, tau, r*rho + m] for m < d when tau >= 0, and 0  */
+/* (all-zero bits) when tau = -1, where tau = end_idx[b*R + r, t] + 1.       */
+/* V: [B, T, Cv] bf16 bits with row stride Cv; out: [B, T, R*d].             */
+/* ------------------------------------------------------------------------ */
+
+int oracle_gather(const uint16_t *V, int64_t v_row_stride, int64_t rho,
+                  const int32_t *end_idx, int B, int R, int T, int d, uint16_t *out)
+{
+    if (B < 0 || R < 0 || T < 0 || d < 0 || rho < 0) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int r = 0; r < R; ++r) {
+                int32_t e = end_idx[((size_t)b * R + r) * T + t];
+                int64_t tau = (int64_t)e + 1;
+                uint16_t *dst = out + ((size_t)b * T + t) * ((size_t)R * d) + (size_t)r * d;
+                if (e < 0) {
+                    for (int m = 0; m < d; ++m) dst[m] = 0;
+                } else {
+                    const uint16_t *src = V + ((size_t)b * T + (size_t)tau) * (size_t)v_row_stride
+                                            + (size_t)(r * rho);
+                    for (int m = 0; m < d; ++m) dst[m] = src[m];
+                }
+            }
+    return ORACLE_OK;
+}
