@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the ROSA retrieval step on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+A step is one pass of the retrieval hot path over one batch of synthetic
+input: discretisation (when the workload starts from hidden states), suffix
+matching, and the value-row read-out (when the workload has value rows).
+The default workload is ``zipf-256-131k``: 128 independent streams of
+T = 131072 symbols over 256 Zipf(1.1) symbols, query and key streams drawn
+independently with shared planted repeats.
+
+Metric: matched positions per second (streams x T / s), whole job.  Each
+rank processes its own full copy of the workload (weak scaling: the streams
+of a job are independent, so nothing is exchanged between ranks).
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events
+on the launching stream after an L2 flush (a 256 MiB memset outside the
+event pair); barrier + synchronize on both sides; max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ROSA matched positions/sec on 1 B200 (streams x T / s); achieved HBM GB/s vs peak"
+UNIT = "positions/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-streams", type=int, default=0,
+                    help="streams of the workload the CPU oracle is timed on (0 = auto, ~10-30 s)")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- workloads
+
+def build_workload(cfg: int, device, seed_offset: int = 0):
+    """Returns a dict with device inputs and the sizes of every op of a step."""
+    import torch
+    from suffix_automaton_retrieval_b200 import workloads as W
+
+    wl = {"cfg": cfg}
+    if cfg == 3:
+        c = W.CONFIGS[3]
+        T, width, ch, M, d, rho = c["T"], c["width"], c["channels"], c["M"], c["d"], c["rho"]
+        H, Wq, Wk = W.qwen_projection_inputs(T=T, width=width, channels=ch, device=device,
+                                             seed_h=3 + 1000 * seed_offset)
+        # projection = set-up, outside the timed step
+        wl["qvec"] = (H @ Wq).contiguous()
+        wl["kvec"] = (H @ Wk).contiguous()
+        del H
+        R = ch // M
+        wl.update(name=c["name"], B=1, R=R, T=T, K=2 ** M, g=2, S=R, same=False, M=M, d=d, rho=rho)
+        wl["V"] = W.value_rows(1, T, R * rho, seed=c["seed_v"] + 1000 * seed_offset, device=device)
+        wl["ops"] = ["discretize", "match", "gather"]
+        return wl
+    c = W.CONFIGS[cfg]
+    if seed_offset:
+        # other ranks draw the same recipe with shifted seeds
+        gen = {1: lambda: W.binary_iid(seed=1 + 1000 * seed_offset),
+               2: lambda: W.planted_copies(seed=2 + 1000 * seed_offset),
+               4: lambda: W.zipf_planted(seed_q=41 + 1000 * seed_offset, seed_k=42 + 1000 * seed_offset,
+                                         seed_plant=43 + 1000 * seed_offset),
+               5: lambda: W.markov(seed_q=51 + 1000 * seed_offset, seed_k=52 + 1000 * seed_offset)}[cfg]
+        sw = gen()
+    else:
+        sw = c["make"]()
+    wl.update(name=sw.name, B=sw.B, R=sw.R, T=sw.T, K=sw.K, g=sw.g, S=sw.S, same=sw.same_qk)
+    wl["q_host"], wl["k_host"] = sw.q, sw.k
+    wl["q"] = torch.from_numpy(sw.q).to(device)
+    wl["k"] = wl["q"] if sw.same_qk else torch.from_numpy(sw.k).to(device)
+    wl["ops"] = ["match"]
+    if "d" in c:
+        wl["d"], wl["rho"] = c["d"], c["rho"]
+        wl["V"] = W.value_rows(sw.B, sw.T, sw.R * c["rho"], seed=c["seed_v"] + 1000 * seed_offset, device=device)
+        wl["ops"].append("gather")
+    return wl
+
+
+def algorithmic_bytes(wl):
+    """Minimum bytes each op must move (read + write), per step."""
+    S, T = wl["S"], wl["T"]
+    out = {}
+    if "discretize" in wl["ops"]:
+        B, C = wl["qvec"].shape[0], wl["qvec"].shape[2]
+        out["discretize"] = 2 * (B * T * C * 2 + B * (C // wl["M"]) * T)
+    # q (1 B) + k (1 B, unless q = k) + three int32 outputs
+    out["match"] = S * T * ((1 if wl["same"] else 2) + 12)
+    if "gather" in wl["ops"]:
+        # end_idx (4 B) + d bf16 read + d bf16 written per (position, route)
+        out["gather"] = wl["B"] * T * wl["R"] * (4 + 2 * wl["d"] * 2)
+    return out
+
+
+class Runner:
+    """One step of the hot path through the binding, outputs preallocated."""
+
+    def __init__(self, wl, device):
+        import torch
+        import suffix_automaton_retrieval_b200.binding as rosa
+        self.rosa, self.wl, self.torch = rosa, wl, torch
+        S, T = wl["S"], wl["T"]
+        self.ws = rosa.alloc_workspace(S, T, wl["K"], device)
+        self.outs = tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))
+        if "discretize" in wl["ops"]:
+            B, _, C = wl["qvec"].shape
+            self.sq = torch.empty((B, C // wl["M"], T), dtype=torch.uint8, device=device)
+            self.sk = torch.empty_like(self.sq)
+        if "gather" in wl["ops"]:
+            self.gout = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
+
+    def launches(self):
+        wl = self.wl
+        n = self.rosa.match_launch_count(wl["S"], wl["T"], wl["K"], wl["same"])
+        n += 2 if "discretize" in wl["ops"] else 0
+        n += 1 if "gather" in wl["ops"] else 0
+        return n
+
+    def step(self, events=None):
+        rosa, wl = self.rosa, self.wl
+        ev = events or {}
+
+        def mark(name):
+            if name in ev:
+                ev[name].record()
+
+        if "discretize" in wl["ops"]:
+            mark("discretize0")
+            rosa.discretize(wl["qvec"], wl["M"], out=self.sq)
+            rosa.discretize(wl["kvec"], wl["M"], out=self.sk)
+            mark("discretize1")
+            q = self.sq.view(wl["S"], wl["T"])
+            k = self.sk.view(wl["S"], wl["T"])
+        else:
+            q, k = wl["q"], wl["k"]
+        mark("match0")
+        rosa.match(q, None if wl["same"] else k, K=wl["K"], g=wl["g"], out=self.outs, workspace=self.ws)
+        mark("match1")
+        if "gather" in wl["ops"]:
+            mark("gather0")
+            rosa.gather(wl["V"], self.outs[0], wl["R"], wl["d"], wl["rho"], out=self.gout)
+            mark("gather1")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1].split()[0]), float(f[2].split()[0]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- peaks
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- CPU oracle baseline
+
+def cpu_oracle_baseline(wl, target_seconds=(10.0, 30.0), forced_streams=0):
+    """Time the oracle (as it stands) on a bounded sample of this workload's
+    streams, on all host cores.  Returns positions/s and what was sampled."""
+    import oracle
+    if wl["cfg"] == 3:
+        q = oracle.discretize(wl["qvec"].cpu().view(__import__("torch").int16).numpy().view(np.uint16), wl["M"])
+        k = oracle.discretize(wl["kvec"].cpu().view(__import__("torch").int16).numpy().view(np.uint16), wl["M"])
+        q, k = q.reshape(wl["S"], wl["T"]), k.reshape(wl["S"], wl["T"])
+    else:
+        q, k = wl["q_host"], wl["k_host"]
+    cores = os.cpu_count() or 1
+    S = wl["S"]
+    n = forced_streams or min(S, cores)
+    while True:
+        t0 = time.perf_counter()
+        oracle.match_sam(q[:n], k[:n] if not wl["same"] else q[:n], g=wl["g"], threads=cores)
+        dt = time.perf_counter() - t0
+        if forced_streams or dt >= target_seconds[0] or n >= S:
+            break
+        n = min(S, max(n + 1, int(n * min(8.0, target_seconds[0] * 1.5 / max(dt, 1e-3)))))
+    used = min(cores, n)
+    return {"value": n * wl["T"] / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{n} of {S} streams x T={wl['T']} (full length), online suffix automaton, "
+                      f"{used} threads, {dt:.1f} s", "seconds": dt}
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+
+    from suffix_automaton_retrieval_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+
+    wl = build_workload(args.config, device, seed_offset=rank)
+    runner = Runner(wl, device)
+    ab = algorithmic_bytes(wl)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(3, args.warmup)):
+        runner.step()
+    torch.cuda.synchronize()
+
+    names = [o + s for o in wl["ops"] for s in ("0", "1")]
+    per_step = []
+    op_ms = {o: [] for o in wl["ops"]}
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_wall = time.perf_counter()
+    for _ in range(args.steps):
+        flush.zero_()
+        ev = {n: torch.cuda.Event(enable_timing=True) for n in names}
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        runner.step(ev)
+        e1.record(stream)
+        per_step.append((e0, e1, ev))
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    step_ms = [a.elapsed_time(b) for a, b, _ in per_step]
+    for _, _, ev in per_step:
+        for o in wl["ops"]:
+            op_ms[o].append(ev[o + "0"].elapsed_time(ev[o + "1"]))
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    positions = wl["S"] * wl["T"]
+    value = positions * args.steps * world / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    # roofline of the dominant op (the one with the largest share of the step)
+    mean_op = {o: statistics.mean(v) for o, v in op_ms.items()}
+    dom = max(mean_op, key=mean_op.get)
+    peak, peak_kind = load_peaks()
+    achieved = ab[dom] / (mean_op[dom] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"rosa_{dom}", "achieved": round(achieved, 2), "peak": peak,
+                "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 5),
+                "traffic": None, "algorithmic_bytes": ab[dom], "ms": round(mean_op[dom], 4),
+                "ops_ms": {o: round(v, 4) for o, v in mean_op.items()}}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(wl, device, args.steps)
+    if world > 1:
+        # every rank takes the same collective steps
+        ev_t = torch.tensor([e2e["value"] if e2e else 0.0], dtype=torch.float64, device=device)
+        dist.all_reduce(ev_t, op=dist.ReduceOp.MIN)
+        if e2e:
+            e2e["value"] = float(ev_t.item()) * world
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_baseline(wl, forced_streams=args.cpu_sample_streams)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": wl["name"], "streams": wl["S"], "T": wl["T"], "K": wl["K"], "g": wl["g"],
+                       "q_equals_k": wl["same"], "ops": wl["ops"], "parallelism": f"streams x{world} (weak)",
+                       "l2": "flushed before every timed step (256 MiB memset outside the events)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": runner.launches() * args.steps, "clocks": clocks,
+            "wall_s_timed_region": round(t_wall, 4),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def end_to_end(wl, device, steps):
+    """Same metric through the public API with host buffers: pinned host
+    inputs copied in, the step, outputs copied back, every step."""
+    import torch
+    rosa = __import__("suffix_automaton_retrieval_b200.binding", fromlist=["x"])
+    S, T = wl["S"], wl["T"]
+    stream = torch.cuda.current_stream(device)
+    if "discretize" in wl["ops"]:
+        hin = [wl["qvec"].cpu().pin_memory(), wl["kvec"].cpu().pin_memory(), wl["V"].cpu().pin_memory()]
+    elif "gather" in wl["ops"]:
+        hin = [torch.from_numpy(wl["q_host"]).pin_memory(),
+               torch.from_numpy(wl["k_host"]).pin_memory(), wl["V"].cpu().pin_memory()]
+    else:
+        hin = [torch.from_numpy(wl["q_host"]).pin_memory()]
+        if not wl["same"]:
+            hin.append(torch.from_numpy(wl["k_host"]).pin_memory())
+    din = [torch.empty_like(h, device=device) for h in hin]
+    ws = rosa.alloc_workspace(S, T, wl["K"], device)
+    outs = tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))
+    if "gather" in wl["ops"]:
+        gout = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
+        hout = [torch.empty(gout.shape, dtype=gout.dtype).pin_memory()]
+    else:
+        hout = [torch.empty((S, T), dtype=torch.int32).pin_memory() for _ in range(3)]
+
+    def one():
+        for h, d in zip(hin, din):
+            d.copy_(h, non_blocking=True)
+        if "discretize" in wl["ops"]:
+            sq = rosa.discretize(din[0], wl["M"])
+            sk = rosa.discretize(din[1], wl["M"])
+            q, k = sq.view(S, T), sk.view(S, T)
+        else:
+            q = din[0]
+            k = None if wl["same"] else din[1]
+        e, l, s = rosa.match(q, k, K=wl["K"], g=wl["g"], out=outs, workspace=ws)
+        if "gather" in wl["ops"]:
+            rosa.gather(din[-1], e, wl["R"], wl["d"], wl["rho"], out=gout)
+            hout[0].copy_(gout, non_blocking=True)
+        else:
+            for h, d in zip(hout, (e, l, s)):
+                h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    h2d = sum(h.numel() * h.element_size() for h in hin)
+    d2h = sum(h.numel() * h.element_size() for h in hout)
+    return {"value": S * T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle (plain online suffix automaton on
+    host threads, as it stands), timed on a bounded sample per step."""
+    if rank != 0:
+        return 0
+    from suffix_automaton_retrieval_b200 import workloads as W
+    import oracle
+    oracle.build()
+    cfg = args.config
+    if cfg == 3:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "qwen-proj-64 needs the GPU projection set-up; reference arm runs on symbol workloads"}))
+        return 0
+    sw = W.CONFIGS[cfg]["make"]()
+    cores = os.cpu_count() or 1
+    n = args.cpu_sample_streams or min(sw.S, cores)
+    # size the per-step sample so the whole run stays within a few minutes
+    t0 = time.perf_counter()
+    oracle.match_sam(sw.q[:n], sw.k[:n] if not sw.same_qk else sw.q[:n], g=sw.g, threads=cores)
+    probe = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    while probe * 2 < budget and n * 2 <= sw.S:
+        n *= 2
+        probe *= 2
+    while probe > budget and n > 1:
+        n = max(1, n // 2)
+        probe /= 2
+    qs, ks = sw.q[:n], (sw.q[:n] if sw.same_qk else sw.k[:n])
+    for _ in range(args.warmup):
+        oracle.match_sam(qs, ks, g=sw.g, threads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.match_sam(qs, ks, g=sw.g, threads=cores)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = n * sw.T * args.steps / total
+    used = min(cores, n)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+            "data": "synthetic",
+            "config": {"workload": sw.name, "streams": sw.S, "T": sw.T, "K": sw.K, "g": sw.g,
+                       "q_equals_k": sw.same_qk},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                             "sample": f"{n} of {sw.S} streams x T={sw.T} per step (full length)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)

@@ -1,0 +1,146 @@
+/*
+ * rosa.h -- C ABI of the B200-native ROSA retrieval step.
+ *
+ * The operation is the retrieval stage of "ROSA-Tuning: Enhancing Windowed
+ * Attention with Global Recall" (arXiv 2602.02499): binary discretisation of
+ * hidden states into multi-route symbol streams (section 3.2), the suffix
+ * retrieval destination tau of each position (section 3.3, Eq. 16; appendix
+ * B.3), and the read-out of value rows at tau (appendix C.4, Eq. 17).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers into memory the caller owns
+ *     (cudaMalloc, a torch tensor, ...).  The library allocates nothing and
+ *     keeps no state between calls.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the
+ *     call returns without waiting for it, except where stated.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned as ROSA_ERR_INVALID_ARG / ROSA_ERR_WORKSPACE; launch
+ *     failures are returned as ROSA_ERR_CUDA.  No call aborts the process or
+ *     throws across the ABI.
+ *   - bf16 tensors are passed as pointers to their 16-bit patterns
+ *     (rosa_bf16), IEEE bfloat16 layout.
+ */
+#ifndef ROSA_H_
+#define ROSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define ROSA_API __attribute__((visibility("default")))
+#else
+#define ROSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t rosa_bf16;
+
+typedef enum {
+    ROSA_OK = 0,
+    ROSA_ERR_INVALID_ARG = 1,   /* bad shape, range, alignment or NULL pointer */
+    ROSA_ERR_WORKSPACE = 2,     /* workspace missing or smaller than required */
+    ROSA_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
+    ROSA_ERR_DEVICE = 4,        /* a device-side check fired (see rosa_match_device_status) */
+    ROSA_ERR_INTERNAL = 5
+} rosa_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+ROSA_API const char *rosa_status_string(int status);
+
+/*
+ * Binary discretisation and multi-route packing (section 3.2, Eqs. 10-15;
+ * route layout of section 4.1).
+ *
+ *   x    [B, T, C] bf16, row-major (channel fastest).
+ *   sym  [B, R, T] uint8, R = C / M, written in full.
+ *   sym[b, r, t] = sum_{j<M} I[x[b, t, r*M + j] > 0] * 2^j
+ *
+ * The threshold is strict: +0, -0 and NaN give bit 0; +inf and positive
+ * subnormals give bit 1.  Requires 1 <= M <= 8, C % M == 0, B, T >= 0, C >= 1.
+ * Any alignment is accepted (16-byte aligned rows take the vector path).
+ */
+ROSA_API int rosa_discretize(const rosa_bf16 *x, int B, int T, int C, int M,
+                    uint8_t *sym, cudaStream_t stream);
+
+/*
+ * Bytes of workspace rosa_match needs for S streams of length T over an
+ * alphabet of K symbols (an upper bound valid whether or not q == k).
+ * Returns 0 for invalid sizes.
+ */
+ROSA_API size_t rosa_match_workspace_size(int S, int T, int K);
+
+/*
+ * Suffix retrieval (section 3.3, Eq. 16; appendix B.3), S independent
+ * streams (one per batch x route pair, section 4.1).
+ *
+ *   q, k  [S, T] uint8 query / key symbols, each < K.  Passing the same
+ *         pointer for q and k selects the self-retrieval form (q = k), which
+ *         needs half the work; distinct pointers with equal contents give the
+ *         same result.
+ *   v     [S, T] uint8 value symbols, or NULL to read them from k.
+ *   g     causal lag >= 1: key end i is admissible at query time t iff
+ *         i <= t - g.  g = 2 gives tau = i + 1 <= t - 1, the range of Eq. 16.
+ *
+ * For every stream s and position t, with L the length of the longest
+ * suffix of q[s, 0..t] that ends in k[s, .] at some admissible i, and i* the
+ * largest such i:
+ *   end_idx[s, t] = i*        (-1 if L = 0)   -- tau = end_idx + 1
+ *   len[s, t]     = L
+ *   sym[s, t]     = v[s, i*+1] (-1 if L = 0)
+ * Outputs are int32 [S, T], written in full.
+ *
+ * `workspace` is device memory of at least rosa_match_workspace_size(S, T, K)
+ * bytes, 256-byte aligned; its contents on entry do not matter and are
+ * clobbered.  Calls that share a workspace must not overlap on the GPU.
+ * Requires 1 <= K <= 256, g >= 1, S >= 0, T >= 0 and S*T*2 < 2^31.
+ * Symbols >= K are a caller error: they are masked to the alphabet's bit
+ * width and flagged in the workspace status word (rosa_match_device_status).
+ */
+ROSA_API int rosa_match(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+               int S, int T, int K, int g,
+               int32_t *end_idx, int32_t *len, int32_t *sym,
+               void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Number of kernel launches one rosa_match call with these arguments
+ * enqueues (q_is_k: 1 when q and k are the same pointer).  Host-only; lets a
+ * caller account for the work it submits.  Returns -1 for invalid sizes.
+ */
+ROSA_API int rosa_match_launch_count(int S, int T, int K, int q_is_k);
+
+/*
+ * Reads the device status word a previous rosa_match left in `workspace`
+ * (0 = no device-side check fired, otherwise a bit set of ROSA_DEV_*).
+ * Synchronises `stream`.  Returns ROSA_OK or ROSA_ERR_CUDA.
+ */
+#define ROSA_DEV_SYMBOL_RANGE 1u   /* some input symbol was >= K */
+ROSA_API int rosa_match_device_status(const void *workspace, cudaStream_t stream, uint32_t *status);
+
+/*
+ * Read-out of value rows at tau (appendix C.4 with the Eq. 17 mask).
+ *
+ *   V        [B, T, *] bf16 rows, row stride v_row_stride elements.
+ *   end_idx  [B*R, T] int32 from rosa_match (stream s = b*R + r).
+ *   out      [B, T, R*d] bf16, written in full.
+ *   out[b, t, r*d + m] = V[b, end_idx[b*R+r, t] + 1, r*v_route_stride + m]
+ *                        for m < d, or +0.0 when end_idx = -1.
+ * v_route_stride = d reads each route's own slice; 0 makes every route read
+ * the same d-wide row.  rosa_match only produces end_idx in [-1, T-2]; any
+ * value outside that range is treated like -1 (zero row), so no call reads
+ * outside V.  A bit-exact copy: no arithmetic on the values.
+ * Requires B, R, T >= 0, d >= 1, v_route_stride >= 0,
+ * (R-1)*v_route_stride + d <= v_row_stride.
+ */
+ROSA_API int rosa_gather(const rosa_bf16 *V, int64_t v_row_stride, int64_t v_route_stride,
+                const int32_t *end_idx, int B, int R, int T, int d,
+                rosa_bf16 *out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROSA_H_ */

@@ -1,0 +1,171 @@
+"""ctypes binding of ``librosa_b200.so`` (C ABI in ``include/rosa.h``).
+
+Argument marshalling only: every step of the retrieval runs in the CUDA
+library.  Tensors must be CUDA tensors; there is no CPU fallback, and
+importing this module fails loudly when the library has not been built.
+torch is used for device memory and the current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librosa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"CUDA library {LIB_PATH} is missing: build it with "
+        "`python -m suffix_automaton_retrieval_b200.build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+lib.rosa_status_string.argtypes = [_i]
+lib.rosa_status_string.restype = ctypes.c_char_p
+lib.rosa_discretize.argtypes = [_vp, _i, _i, _i, _i, _vp, _vp]
+lib.rosa_discretize.restype = _i
+lib.rosa_match_workspace_size.argtypes = [_i, _i, _i]
+lib.rosa_match_workspace_size.restype = ctypes.c_size_t
+lib.rosa_match.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.rosa_match.restype = _i
+lib.rosa_match_launch_count.argtypes = [_i, _i, _i, _i]
+lib.rosa_match_launch_count.restype = _i
+lib.rosa_match_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+lib.rosa_match_device_status.restype = _i
+lib.rosa_gather.argtypes = [_vp, _i64, _i64, _vp, _i, _i, _i, _i, _vp, _vp]
+lib.rosa_gather.restype = _i
+
+EXPORTED = ("rosa_status_string", "rosa_discretize", "rosa_match_workspace_size", "rosa_match",
+            "rosa_match_launch_count", "rosa_match_device_status", "rosa_gather")
+
+DEV_SYMBOL_RANGE = 1
+
+
+class RosaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def status_string(code: int) -> str:
+    return lib.rosa_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise RosaError(code, what)
+
+
+def _stream(device) -> _vp:
+    return _vp(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("the ROSA retrieval step runs on CUDA tensors only")
+
+
+def _ptr(t):
+    return _vp(t.data_ptr()) if t is not None and t.numel() > 0 else _vp(None)
+
+
+def discretize(x: torch.Tensor, M: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 ``[B, T, C]`` -> uint8 symbols ``[B, C // M, T]`` (Eqs. 10-15)."""
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 3:
+        raise ValueError("x must be a bf16 tensor [B, T, C]")
+    x = x.contiguous()
+    B, T, C = x.shape
+    if M < 1 or M > 8 or C % M:
+        raise ValueError("need 1 <= M <= 8 and C % M == 0")
+    if out is None:
+        out = torch.empty((B, C // M, T), dtype=torch.uint8, device=x.device)
+    _check(lib.rosa_discretize(_ptr(x), B, T, C, M, _ptr(out), _stream(x.device)), "rosa_discretize")
+    return out
+
+
+def match_workspace_size(S: int, T: int, K: int) -> int:
+    n = lib.rosa_match_workspace_size(S, T, K)
+    if n == 0:
+        raise ValueError(f"invalid match sizes S={S} T={T} K={K}")
+    return n
+
+
+def alloc_workspace(S: int, T: int, K: int, device) -> torch.Tensor:
+    return torch.empty(match_workspace_size(S, T, K), dtype=torch.uint8, device=device)
+
+
+def match(q: torch.Tensor, k: torch.Tensor | None = None, v: torch.Tensor | None = None, *, K: int = 256,
+          g: int = 2, out=None, workspace: torch.Tensor | None = None):
+    """Suffix retrieval over S streams (section 3.3, Eq. 16; appendix B.3).
+
+    ``q``, ``k``, ``v``: uint8 ``[S, T]`` CUDA tensors; ``k=None`` (or the
+    same tensor as ``q``) selects self-retrieval, ``v=None`` reads values
+    from ``k``.  Returns int32 ``(end_idx, len, sym)``, each ``[S, T]``.
+    """
+    _need_cuda(q, k, v, workspace)
+    same = k is None or k is q
+    if q.dtype != torch.uint8 or q.dim() != 2:
+        raise ValueError("q must be uint8 [S, T]")
+    q = q.contiguous()
+    k = q if same else k.contiguous()
+    S, T = q.shape
+    if k.shape != q.shape or k.dtype != torch.uint8:
+        raise ValueError("k must be uint8 with the shape of q")
+    if v is not None:
+        v = v.contiguous()
+        if v.shape != q.shape or v.dtype != torch.uint8:
+            raise ValueError("v must be uint8 with the shape of q")
+    if out is None:
+        out = tuple(torch.empty((S, T), dtype=torch.int32, device=q.device) for _ in range(3))
+    end_idx, ln, sym = out
+    if workspace is None:
+        workspace = alloc_workspace(S, T, K, q.device)
+    _check(lib.rosa_match(_ptr(q), _ptr(k), _ptr(v), S, T, K, g, _ptr(end_idx), _ptr(ln), _ptr(sym),
+                          _vp(workspace.data_ptr()), workspace.numel(), _stream(q.device)), "rosa_match")
+    return end_idx, ln, sym
+
+
+def match_launch_count(S: int, T: int, K: int, same: bool) -> int:
+    """Kernel launches one ``match`` call enqueues (reported by the library)."""
+    n = lib.rosa_match_launch_count(S, T, K, 1 if same else 0)
+    if n < 0:
+        raise ValueError("invalid match sizes")
+    return n
+
+
+def match_device_status(workspace: torch.Tensor) -> int:
+    st = ctypes.c_uint32(0)
+    _check(lib.rosa_match_device_status(_vp(workspace.data_ptr()), _stream(workspace.device),
+                                        ctypes.byref(st)), "rosa_match_device_status")
+    return st.value
+
+
+def gather(V: torch.Tensor, end_idx: torch.Tensor, R: int, d: int, rho: int | None = None,
+           out: torch.Tensor | None = None) -> torch.Tensor:
+    """Rows of ``V`` ``[B, T, W]`` at tau = end_idx + 1 -> ``[B, T, R*d]``
+    (appendix C.4, Eq. 17 mask).  Route r reads columns ``r*rho .. r*rho+d``
+    (``rho`` defaults to d; 0 shares one row)."""
+    _need_cuda(V, end_idx)
+    if V.dtype != torch.bfloat16 or V.dim() != 3 or V.stride(2) != 1:
+        raise ValueError("V must be bf16 [B, T, W] with unit inner stride")
+    if end_idx.dtype != torch.int32:
+        raise ValueError("end_idx must be int32")
+    B, T, _ = V.shape
+    rho = d if rho is None else rho
+    end_idx = end_idx.contiguous()
+    if end_idx.shape != (B * R, T):
+        raise ValueError("end_idx must be [B*R, T]")
+    if V.stride(0) != T * V.stride(1):
+        V = V.contiguous()
+    if out is None:
+        out = torch.empty((B, T, R * d), dtype=torch.bfloat16, device=V.device)
+    _check(lib.rosa_gather(_ptr(V), V.stride(1), rho, _ptr(end_idx), B, R, T, d, _ptr(out),
+                           _stream(V.device)), "rosa_gather")
+    return out

@@ -1,0 +1,773 @@
+// Position-parallel exact matcher for the ROSA retrieval destination.
+//
+// "ROSA-Tuning" (arXiv 2602.02499), section 3.3 Eq. (16) and appendix B.3:
+// for every stream and time t, the longest suffix of q[0..t] that occurs in
+// the key stream ending at an admissible position i <= t - g, and the most
+// recent such end i* (tau = i* + 1; -1 when nothing matches).  The pages run
+// one online suffix automaton per stream on a CPU core (sections 2.2, 4.1);
+// that is a chain of T dependent steps per stream.  Here the same quantity is
+// computed position-parallel:
+//
+//   D(t, i) = longest common suffix of q[0..t] and k[0..i]
+//           = longest common prefix of the reversed prefixes
+//             Q_t = q[t] q[t-1] .. q[0]  and  K_i = k[i] k[i-1] .. k[0].
+//
+// 1. Sort all reversed prefixes of a stream (keys, and queries when q != k)
+//    lexicographically: an LSD radix sort on the first D0 symbols packed in a
+//    64-bit word, then prefix doubling (sort each tied group by the rank of
+//    the prefix h symbols further back) until every group is a single string.
+// 2. Adjacent longest-common-prefix array of the sorted order.
+// 3. For a query at rank j, LCP with any other rank is the minimum of the
+//    adjacent LCPs in between, so the best admissible key lies at the nearest
+//    admissible rank on either side: L_t = max of the two.  The admissible
+//    keys with LCP >= L_t form a rank interval around j; i* is the largest
+//    admissible key position inside it.  Summaries over blocks of 32 and 1024
+//    ranks (smallest key position, smallest inner LCP) let long scans skip.
+//
+// All kernels are stream-segmented: items of stream s occupy [s*n, (s+1)*n).
+#include <climits>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/rosa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rosa {
+namespace {
+
+constexpr int kRadixThreads = 256;
+constexpr int kRadixIPT = 8;
+constexpr int kRadixTile = kRadixThreads * kRadixIPT;   // 2048 items per tile
+constexpr int kRadixBits = 8;
+constexpr int kRadixBins = 1 << kRadixBits;
+constexpr int kScanThreads = 1024;
+constexpr int kSmallGroup = 32;        // groups up to this size are sorted by one warp
+constexpr int kSmemSortCap = 4096;     // larger groups up to this size sort in shared memory
+constexpr int kLargeThreads = 512;
+constexpr int kL1 = 32;                // summary block sizes (ranks)
+constexpr int kL2 = 1024;
+
+int bits_for(int v) {   // number of bits to hold values 0..v
+    int b = 0;
+    while ((1 << b) <= v) ++b;
+    return b;
+}
+
+struct Geometry {
+    int S, T, K, g, n;
+    bool same;
+    int bps, D0, abits, keybits;
+    int64_t N;
+    int ntps, nb1, nb2;
+};
+
+Geometry make_geometry(int S, int T, int K, int g, bool same) {
+    Geometry G{};
+    G.S = S; G.T = T; G.K = K; G.g = g; G.same = same;
+    G.n = same ? T : 2 * T;
+    G.N = (int64_t)S * G.n;
+    G.bps = bits_for(K - 1);
+    if (G.bps < 1) G.bps = 1;
+    // D0 symbols of bps bits plus the available length (0..D0+1) must fit 64 bits
+    int d = 64 / G.bps;
+    while (d > 1 && d * G.bps + bits_for(d + 1) > 64) --d;
+    G.D0 = d;
+    G.abits = bits_for(d + 1);
+    G.keybits = d * G.bps + G.abits;
+    G.ntps = ceil_div(G.n, kRadixTile);
+    G.nb1 = ceil_div(G.n, kL1);
+    G.nb2 = ceil_div(G.n, kL2);
+    return G;
+}
+
+struct Workspace {
+    uint32_t *status;
+    int *counts;             // [2 buffers][2 kinds]
+    uint64_t *keys[2];
+    uint32_t *vals[2];
+    int32_t *rank;
+    int32_t *lcp;
+    uint32_t *k2;
+    uint32_t *hist;
+    int2 *lists[2][2];       // [buffer][0 = small, 1 = large]
+    int32_t *minpos1, *emin1, *minpos2, *emin2;
+    size_t bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Lays the workspace out from `base` (or only measures it when base == nullptr).
+Workspace carve(const Geometry &G, void *base) {
+    Workspace W{};
+    size_t off = 0;
+    char *b = static_cast<char *>(base);
+    auto take = [&](size_t bytes) -> void * {
+        void *p = b ? b + off : nullptr;
+        off += align256(bytes);
+        return p;
+    };
+    const size_t N = (size_t)G.N;
+    const size_t list_cap = N / 2 + 1;
+    W.status = (uint32_t *)take(256);
+    W.counts = (int *)take(4 * sizeof(int));
+    W.keys[0] = (uint64_t *)take(N * 8);
+    W.keys[1] = (uint64_t *)take(N * 8);
+    W.vals[0] = (uint32_t *)take(N * 4);
+    W.vals[1] = (uint32_t *)take(N * 4);
+    W.rank = (int32_t *)take(N * 4);
+    W.lcp = (int32_t *)take(N * 4);
+    W.k2 = (uint32_t *)take(N * 4);
+    W.hist = (uint32_t *)take((size_t)G.S * kRadixBins * G.ntps * 4);
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 2; ++j) W.lists[i][j] = (int2 *)take(list_cap * sizeof(int2));
+    W.minpos1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
+    W.emin1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
+    W.minpos2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
+    W.emin2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
+    W.bytes = off;
+    return W;
+}
+
+// ---------------------------------------------------------------------------
+// 1a. Round-0 keys: first D0 symbols of the reversed prefix, most significant
+//     first, zero-padded past the start, then min(p+1, D0+1) in the low bits so
+//     that a string that ends sorts before its extensions.
+// ---------------------------------------------------------------------------
+__global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
+                             uint64_t *__restrict__ keys, uint32_t *__restrict__ vals,
+                             uint32_t *__restrict__ status) {
+    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gi >= G.N) return;
+    const int s = (int)(gi / G.n);
+    const int x = (int)(gi - (int64_t)s * G.n);
+    const uint8_t *a;
+    int p;
+    if (x < G.T) { a = k + (int64_t)s * G.T; p = x; }
+    else         { a = q + (int64_t)s * G.T; p = x - G.T; }
+    const uint32_t symmask = (1u << G.bps) - 1u;
+    const int avail = min(p + 1, G.D0 + 1);
+    uint64_t chars = 0;
+    for (int m = 0; m < G.D0; ++m) {
+        uint32_t c = (m < avail) ? (uint32_t)a[p - m] : 0u;
+        chars = (chars << G.bps) | (c & symmask);
+    }
+    if ((uint32_t)a[p] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
+    keys[gi] = (chars << G.abits) | (uint64_t)avail;
+    vals[gi] = (uint32_t)x;
+}
+
+// ---------------------------------------------------------------------------
+// 1b. Segmented LSD radix sort, 8-bit digits, tiles of 2048 items that never
+//     straddle a stream.  hist layout: [stream][digit][tile-in-stream].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kRadixThreads)
+radix_hist_kernel(const uint64_t *__restrict__ keys, Geometry G, int shift, uint32_t *__restrict__ hist) {
+    __shared__ uint32_t cnt[kRadixBins];
+    const int tile = blockIdx.x;
+    const int s = tile / G.ntps, tt = tile - s * G.ntps;
+    cnt[threadIdx.x] = 0;
+    __syncthreads();
+    const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
+    const int lim = min(kRadixTile, G.n - tt * kRadixTile);
+    for (int i = threadIdx.x; i < lim; i += kRadixThreads)
+        atomicAdd(&cnt[(keys[base + i] >> shift) & (kRadixBins - 1)], 1u);
+    __syncthreads();
+    hist[((int64_t)s * kRadixBins + threadIdx.x) * G.ntps + tt] = cnt[threadIdx.x];
+}
+
+// Exclusive scan of one stream's [digit][tile] counts, in place.
+__global__ void __launch_bounds__(kScanThreads)
+radix_scan_kernel(uint32_t *__restrict__ hist, int ntps) {
+    __shared__ uint32_t ws[kScanThreads / 32 + 1];
+    uint32_t *h = hist + (int64_t)blockIdx.x * kRadixBins * ntps;
+    const int M = kRadixBins * ntps;
+    const int per = ceil_div(M, kScanThreads);
+    const int lo = min(M, threadIdx.x * per), hi = min(M, lo + per);
+    uint32_t sum = 0;
+    for (int i = lo; i < hi; ++i) sum += h[i];
+    uint32_t run = block_exclusive_scan<kScanThreads>(sum, ws, nullptr);
+    for (int i = lo; i < hi; ++i) {
+        const uint32_t c = h[i];
+        h[i] = run;
+        run += c;
+    }
+}
+
+// Stable scatter of one tile: items keep their tile order within a digit.
+__global__ void __launch_bounds__(kRadixThreads)
+radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restrict__ vin,
+                     uint64_t *__restrict__ kout, uint32_t *__restrict__ vout, Geometry G, int shift,
+                     const uint32_t *__restrict__ hist) {
+    __shared__ uint64_t sk[kRadixTile];
+    __shared__ uint32_t sv[kRadixTile];
+    __shared__ uint16_t wcnt[kRadixThreads / 32][kRadixBins];
+    __shared__ uint32_t running[kRadixBins];
+    __shared__ uint32_t tstart[kRadixBins];
+    __shared__ uint32_t gofs[kRadixBins];
+    __shared__ uint32_t wsum[kRadixThreads / 32 + 1];
+
+    const int tile = blockIdx.x;
+    const int s = tile / G.ntps, tt = tile - s * G.ntps;
+    const int64_t seg = (int64_t)s * G.n;
+    const int64_t base = seg + (int64_t)tt * kRadixTile;
+    const int lim = min(kRadixTile, G.n - tt * kRadixTile);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    gofs[threadIdx.x] = hist[((int64_t)s * kRadixBins + threadIdx.x) * G.ntps + tt];
+    running[threadIdx.x] = 0;
+    for (int w = 0; w < kRadixThreads / 32; ++w) wcnt[w][threadIdx.x] = 0;
+    __syncthreads();
+
+    uint64_t key[kRadixIPT];
+    uint32_t val[kRadixIPT];
+    uint32_t rnk[kRadixIPT];
+    int dig[kRadixIPT];
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {
+        const int i = u * kRadixThreads + threadIdx.x;
+        const bool ok = i < lim;
+        key[u] = ok ? kin[base + i] : 0ull;
+        val[u] = ok ? vin[base + i] : 0u;
+        dig[u] = ok ? (int)((key[u] >> shift) & (kRadixBins - 1)) : kRadixBins;
+        const unsigned peers = __match_any_sync(ROSA_FULL_MASK, dig[u]);
+        const unsigned wr = __popc(peers & lanemask_lt());
+        if (ok && wr == 0) wcnt[warp][dig[u]] = (uint16_t)__popc(peers);
+        __syncthreads();
+        if (ok) {
+            uint32_t pre = running[dig[u]];
+            for (int w = 0; w < warp; ++w) pre += wcnt[w][dig[u]];
+            rnk[u] = pre + wr;
+        }
+        __syncthreads();
+        {
+            uint32_t add = 0;
+            for (int w = 0; w < kRadixThreads / 32; ++w) {
+                add += wcnt[w][threadIdx.x];
+                wcnt[w][threadIdx.x] = 0;
+            }
+            running[threadIdx.x] += add;
+        }
+        __syncthreads();
+    }
+    (void)lane;
+    const uint32_t st = block_exclusive_scan<kRadixThreads>(running[threadIdx.x], wsum, nullptr);
+    tstart[threadIdx.x] = st;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {
+        if (dig[u] < kRadixBins) {
+            const uint32_t pos = tstart[dig[u]] + rnk[u];
+            sk[pos] = key[u];
+            sv[pos] = val[u];
+        }
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < lim; j += kRadixThreads) {
+        const uint64_t kk = sk[j];
+        const int d = (int)((kk >> shift) & (kRadixBins - 1));
+        const int64_t dst = seg + gofs[d] + (j - tstart[d]);
+        kout[dst] = kk;
+        vout[dst] = sv[j];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1c. Groups after round 0: rank = position of the group head; groups of more
+//     than one incomplete string (p + 1 > D0) go to the unresolved lists.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ? (int)x : (int)x - T; }
+
+__device__ __forceinline__ void push_group(int2 *small, int2 *large, int *counts_next, int64_t start, int size) {
+    if (size <= kSmallGroup) {
+        const int i = atomicAdd(&counts_next[0], 1);
+        small[i] = make_int2((int)start, size);
+    } else {
+        const int i = atomicAdd(&counts_next[1], 1);
+        large[i] = make_int2((int)start, size);
+    }
+}
+
+__global__ void groups0_kernel(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ sa, Geometry G,
+                               int32_t *__restrict__ rank, int2 *small, int2 *large, int *counts_next) {
+    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gi >= G.N) return;
+    const int s = (int)(gi / G.n);
+    const int j = (int)(gi - (int64_t)s * G.n);
+    const int64_t seg = (int64_t)s * G.n;
+    const uint64_t kk = keys[gi];
+    if (j > 0 && keys[gi - 1] == kk) return;   // not a group head
+    int e = j + 1;
+    while (e < G.n && keys[seg + e] == kk) ++e;
+    for (int m = j; m < e; ++m) rank[seg + sa[seg + m]] = j;
+    const int size = e - j;
+    if (size > 1 && item_pos(sa[gi], G.T) + 1 > G.D0) push_group(small, large, counts_next, gi, size);
+}
+
+// ---------------------------------------------------------------------------
+// 1d. Prefix doubling at depth h: sort each unresolved group by the rank of
+//     the same-kind prefix h symbols further back, then split into new groups.
+// ---------------------------------------------------------------------------
+__global__ void dbl_keys_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
+                                const int *__restrict__ counts, Geometry G, int64_t h,
+                                const uint32_t *__restrict__ sa, const int32_t *__restrict__ rank,
+                                uint32_t *__restrict__ k2) {
+    const int ns = counts[0], nl = counts[1];
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t gidx = wid; gidx < ns + nl; gidx += nw) {
+        const int2 gr = gidx < ns ? small[gidx] : large[gidx - ns];
+        const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
+        for (int m = lane; m < gr.y; m += 32) {
+            const uint32_t x = sa[gr.x + m];
+            k2[gr.x + m] = (uint32_t)rank[seg + x - h];
+        }
+    }
+}
+
+// One warp per group of at most 32: rank by counting on (k2, item id).
+__global__ void dbl_sort_small_kernel(const int2 *__restrict__ small, const int *__restrict__ counts,
+                                      uint32_t *__restrict__ sa, uint32_t *__restrict__ k2) {
+    const int ns = counts[0];
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t gidx = wid; gidx < ns; gidx += nw) {
+        const int2 gr = small[gidx];
+        const bool ok = lane < gr.y;
+        const uint64_t key = ok ? (((uint64_t)k2[gr.x + lane] << 32) | sa[gr.x + lane]) : ~0ull;
+        int r = 0;
+        for (int o = 0; o < 32; ++o) {
+            const uint64_t other = __shfl_sync(ROSA_FULL_MASK, key, o);
+            r += (other < key) ? 1 : 0;
+        }
+        __syncwarp();
+        if (ok) {
+            sa[gr.x + r] = (uint32_t)key;
+            k2[gr.x + r] = (uint32_t)(key >> 32);
+        }
+        __syncwarp();
+    }
+}
+
+// Ascending-only bitonic sort of n keys (virtual +inf padding to a power of 2).
+__device__ void bitonic_sort(uint64_t *a, int n) {
+    int np2 = 1;
+    while (np2 < n) np2 <<= 1;
+    for (int kk = 2; kk <= np2; kk <<= 1) {
+        const int half = kk >> 1;
+        for (int i = threadIdx.x; i < np2 / 2; i += blockDim.x) {
+            const int blk = i / half, off = i - blk * half;
+            const int lo = blk * kk + off, hi = blk * kk + kk - 1 - off;
+            if (hi < n && a[lo] > a[hi]) { const uint64_t t = a[lo]; a[lo] = a[hi]; a[hi] = t; }
+        }
+        __syncthreads();
+        for (int jj = kk >> 2; jj >= 1; jj >>= 1) {
+            for (int i = threadIdx.x; i < np2 / 2; i += blockDim.x) {
+                const int blk = i / jj, off = i - blk * jj;
+                const int lo = blk * 2 * jj + off, hi = lo + jj;
+                if (hi < n && a[lo] > a[hi]) { const uint64_t t = a[lo]; a[lo] = a[hi]; a[hi] = t; }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// One CTA per group of more than 32: shared memory up to kSmemSortCap, else
+// in place in the scratch key buffer (global memory).
+__global__ void __launch_bounds__(kLargeThreads)
+dbl_sort_large_kernel(const int2 *__restrict__ large, const int *__restrict__ counts,
+                      uint32_t *__restrict__ sa, uint32_t *__restrict__ k2, uint64_t *__restrict__ scratch) {
+    __shared__ uint64_t buf[kSmemSortCap];
+    const int nl = counts[1];
+    for (int gidx = blockIdx.x; gidx < nl; gidx += gridDim.x) {
+        const int2 gr = large[gidx];
+        uint64_t *a = gr.y <= kSmemSortCap ? buf : scratch + gr.x;
+        for (int m = threadIdx.x; m < gr.y; m += blockDim.x)
+            a[m] = ((uint64_t)k2[gr.x + m] << 32) | sa[gr.x + m];
+        __syncthreads();
+        bitonic_sort(a, gr.y);
+        for (int m = threadIdx.x; m < gr.y; m += blockDim.x) {
+            const uint64_t key = a[m];
+            sa[gr.x + m] = (uint32_t)key;
+            k2[gr.x + m] = (uint32_t)(key >> 32);
+        }
+        __syncthreads();
+    }
+}
+
+// Split sorted groups at k2 changes.  New group id = local head position;
+// new groups of more than one incomplete string (p + 1 > 2h) go on.
+__global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
+                                   const int *__restrict__ counts, Geometry G, int64_t h2,
+                                   const uint32_t *__restrict__ sa, const uint32_t *__restrict__ k2,
+                                   int32_t *__restrict__ rank, int2 *nsmall, int2 *nlarge, int *counts_next) {
+    const int ns = counts[0], nl = counts[1];
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t gidx = wid; gidx < ns + nl; gidx += nw) {
+        const int2 gr = gidx < ns ? small[gidx] : large[gidx - ns];
+        const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
+        const int jstart = (int)(gr.x - seg);
+        int carry = jstart;
+        for (int m0 = 0; m0 < gr.y; m0 += 32) {
+            const int m = m0 + lane;
+            const bool ok = m < gr.y;
+            const uint32_t kk = ok ? k2[gr.x + m] : 0u;
+            const bool head = ok && (m == 0 || k2[gr.x + m - 1] != kk);
+            int hp = head ? jstart + m : -1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(ROSA_FULL_MASK, hp, o);
+                if (lane >= o) hp = max(hp, y);
+            }
+            const int gid = max(hp, carry);
+            if (ok) {
+                const uint32_t x = sa[gr.x + m];
+                rank[seg + x] = gid;
+                const bool last = (m == gr.y - 1) || (k2[gr.x + m + 1] != kk);
+                if (last) {
+                    const int size = jstart + m - gid + 1;
+                    if (size > 1 && (int64_t)item_pos(x, G.T) + 1 > h2)
+                        push_group(nsmall, nlarge, counts_next, seg + gid, size);
+                }
+            }
+            carry = __shfl_sync(ROSA_FULL_MASK, gid, 31);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2. Adjacent LCP of the final order.  Ties never leave a round-0 key group,
+//    so keys[] (sorted in round 0) still holds the key of the item at each
+//    rank.
+// ---------------------------------------------------------------------------
+__global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
+                           const uint64_t *__restrict__ keys, const uint32_t *__restrict__ sa,
+                           int32_t *__restrict__ lcp) {
+    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gi >= G.N) return;
+    const int s = (int)(gi / G.n);
+    const int j = (int)(gi - (int64_t)s * G.n);
+    if (j == 0) { lcp[gi] = 0; return; }
+    const uint64_t k1 = keys[gi - 1], kk2 = keys[gi];
+    const uint64_t amask = (1ull << G.abits) - 1ull;
+    const int a1 = (int)(k1 & amask), a2 = (int)(kk2 & amask);
+    if (k1 != kk2) {
+        const uint64_t x = (k1 >> G.abits) ^ (kk2 >> G.abits);
+        int diff = G.D0;
+        if (x) diff = (__clzll((long long)x) - (64 - G.D0 * G.bps)) / G.bps;
+        lcp[gi] = min(diff, min(min(a1, G.D0), min(a2, G.D0)));
+        return;
+    }
+    if (a1 <= G.D0) { lcp[gi] = a1; return; }   // identical complete strings
+    const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
+    const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
+    const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
+    const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
+    int m = G.D0;
+    const int lim = min(p1, p2) + 1;
+    while (m < lim && s1[p1 - m] == s2[p2 - m]) ++m;
+    lcp[gi] = m;
+}
+
+// ---------------------------------------------------------------------------
+// 3a. Block summaries: smallest key position and smallest inner LCP (edges
+//     strictly inside the block) per 32 and per 1024 ranks.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
+    return (same || (int)x < T) ? (int)x : INT_MAX;
+}
+
+__global__ void __launch_bounds__(kL2)
+summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__restrict__ lcp,
+               int32_t *__restrict__ minpos1, int32_t *__restrict__ emin1,
+               int32_t *__restrict__ minpos2, int32_t *__restrict__ emin2) {
+    __shared__ int wpos[32], wemin[32], wfirst[32];
+    const int s = blockIdx.x / G.nb2, B2 = blockIdx.x - s * G.nb2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int j = B2 * kL2 + threadIdx.x;
+    const int64_t gi = (int64_t)s * G.n + j;
+    int pos = INT_MAX, l = INT_MAX;
+    if (j < G.n) {
+        pos = key_pos_or_inf(sa[gi], G.T, G.same);
+        l = lcp[gi];
+    }
+    const int first = __shfl_sync(ROSA_FULL_MASK, l, 0);
+    int mp = pos, me = lane == 0 ? INT_MAX : l;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        mp = min(mp, __shfl_xor_sync(ROSA_FULL_MASK, mp, o));
+        me = min(me, __shfl_xor_sync(ROSA_FULL_MASK, me, o));
+    }
+    const int b1 = B2 * (kL2 / kL1) + warp;
+    if (lane == 0) {
+        if (b1 < G.nb1) {
+            minpos1[(int64_t)s * G.nb1 + b1] = mp;
+            emin1[(int64_t)s * G.nb1 + b1] = me;
+        }
+        wpos[warp] = mp;
+        wemin[warp] = me;
+        wfirst[warp] = warp == 0 ? INT_MAX : first;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int p2 = wpos[lane], e2 = min(wemin[lane], wfirst[lane]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            p2 = min(p2, __shfl_xor_sync(ROSA_FULL_MASK, p2, o));
+            e2 = min(e2, __shfl_xor_sync(ROSA_FULL_MASK, e2, o));
+        }
+        if (lane == 0) {
+            minpos2[(int64_t)s * G.nb2 + B2] = p2;
+            emin2[(int64_t)s * G.nb2 + B2] = e2;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3b. Per-query resolution in rank order.
+// ---------------------------------------------------------------------------
+struct StreamView {
+    const uint32_t *sa;
+    const int32_t *lcp;
+    const int32_t *mp1, *em1, *mp2, *em2;
+    int n, T;
+    bool same;
+};
+
+__device__ __forceinline__ int kpos(const StreamView &v, int r) { return key_pos_or_inf(v.sa[r], v.T, v.same); }
+
+// LCP with the nearest admissible key (position <= X) at a lower rank than j,
+// or 0 if the running LCP falls to `stop` or below before one is found.
+__device__ int nearest_left(const StreamView &v, int j, int X, int stop) {
+    int m = INT_MAX, r = j - 1;
+    while (r >= 0) {
+        if ((r & (kL2 - 1)) == kL2 - 1) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em2[b]));
+                if (m <= stop) return 0;
+                r -= kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == kL1 - 1) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em1[b]));
+                if (m <= stop) return 0;
+                r -= kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r + 1]);
+        if (m <= stop) return 0;
+        if (kpos(v, r) <= X) return m;
+        --r;
+    }
+    return 0;
+}
+
+__device__ int nearest_right(const StreamView &v, int j, int X, int stop) {
+    int m = INT_MAX, r = j + 1;
+    while (r < v.n) {
+        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r], v.em2[b]));
+                if (m <= stop) return 0;
+                r += kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r], v.em1[b]));
+                if (m <= stop) return 0;
+                r += kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r]);
+        if (m <= stop) return 0;
+        if (kpos(v, r) <= X) return m;
+        ++r;
+    }
+    return 0;
+}
+
+// Largest admissible key position among ranks below j whose LCP with j is >= L.
+__device__ int latest_left(const StreamView &v, int j, int X, int L) {
+    int best = -1, m = INT_MAX, r = j - 1;
+    while (r >= 0) {
+        if ((r & (kL2 - 1)) == kL2 - 1) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em2[b]));
+                if (m < L) return best;
+                r -= kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == kL1 - 1) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em1[b]));
+                if (m < L) return best;
+                r -= kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r + 1]);
+        if (m < L) return best;
+        const int p = kpos(v, r);
+        if (p <= X) best = max(best, p);
+        --r;
+    }
+    return best;
+}
+
+__device__ int latest_right(const StreamView &v, int j, int X, int L) {
+    int best = -1, m = INT_MAX, r = j + 1;
+    while (r < v.n) {
+        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r], v.em2[b]));
+                if (m < L) return best;
+                r += kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r], v.em1[b]));
+                if (m < L) return best;
+                r += kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r]);
+        if (m < L) return best;
+        const int p = kpos(v, r);
+        if (p <= X) best = max(best, p);
+        ++r;
+    }
+    return best;
+}
+
+__global__ void resolve_kernel(Geometry G, const uint8_t *__restrict__ vsym, const uint32_t *__restrict__ sa,
+                               const int32_t *__restrict__ lcp, const int32_t *__restrict__ minpos1,
+                               const int32_t *__restrict__ emin1, const int32_t *__restrict__ minpos2,
+                               const int32_t *__restrict__ emin2, int32_t *__restrict__ end_idx,
+                               int32_t *__restrict__ len, int32_t *__restrict__ sym) {
+    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gi >= G.N) return;
+    const int s = (int)(gi / G.n);
+    const int j = (int)(gi - (int64_t)s * G.n);
+    const int64_t seg = (int64_t)s * G.n;
+    const uint32_t x = sa[gi];
+    if (!G.same && (int)x < G.T) return;          // key item: nothing to answer
+    const int t = G.same ? (int)x : (int)x - G.T;
+    const int64_t o = (int64_t)s * G.T + t;
+    const int X = t - G.g;
+    int L = 0, ib = -1;
+    if (X >= 0) {
+        StreamView v{sa + seg, lcp + seg, minpos1 + (int64_t)s * G.nb1, emin1 + (int64_t)s * G.nb1,
+                     minpos2 + (int64_t)s * G.nb2, emin2 + (int64_t)s * G.nb2, G.n, G.T, G.same};
+        const int bl = nearest_left(v, j, X, 0);
+        const int br = nearest_right(v, j, X, bl);
+        L = max(bl, br);
+        if (L > 0) ib = max(latest_left(v, j, X, L), latest_right(v, j, X, L));
+    }
+    if (L > 0 && ib >= 0) {
+        end_idx[o] = ib;
+        len[o] = L;
+        sym[o] = (int32_t)vsym[(int64_t)s * G.T + ib + 1];
+    } else {
+        end_idx[o] = -1;
+        len[o] = 0;
+        sym[o] = -1;
+    }
+}
+
+inline unsigned grid_for(int64_t n, int threads) { return (unsigned)ceil_div64(n, threads); }
+
+}  // namespace
+
+int match_launch_count(int S, int T, int K, bool same) {
+    if (S == 0 || T == 0) return 0;
+    const Geometry G = make_geometry(S, T, K, 1, same);
+    int rounds = 0;
+    for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
+    const int passes = ceil_div(G.keybits, kRadixBits);
+    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + lcp + summary + resolve
+    return 1 + 3 * passes + 1 + 4 * rounds + 3;
+}
+
+size_t match_workspace_bytes(int S, int T, int K, bool same) {
+    const Geometry G = make_geometry(S, T, K, 1, same);
+    return carve(G, nullptr).bytes;
+}
+
+cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int K, int g,
+                         int32_t *end_idx, int32_t *len, int32_t *sym, void *workspace, size_t ws_bytes,
+                         cudaStream_t st) {
+    const bool same = (q == k);
+    const Geometry G = make_geometry(S, T, K, g, same);
+    Workspace W = carve(G, workspace);
+    if (W.bytes > ws_bytes) return cudaErrorInvalidValue;
+    cudaError_t err;
+    if ((err = cudaMemsetAsync(W.status, 0, 256 + 256, st)) != cudaSuccess) return err;   // status + counts
+    if (S == 0 || T == 0) return cudaSuccess;
+    const uint8_t *vs = v ? v : k;
+
+    // 1a. keys
+    keys0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, W.keys[0], W.vals[0], W.status);
+    // 1b. radix sort over keybits, 8 bits per pass
+    int cur = 0;
+    const unsigned tiles = (unsigned)(G.S * G.ntps);
+    for (int shift = 0; shift < G.keybits; shift += kRadixBits) {
+        radix_hist_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], G, shift, W.hist);
+        radix_scan_kernel<<<(unsigned)G.S, kScanThreads, 0, st>>>(W.hist, G.ntps);
+        radix_scatter_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], W.vals[cur], W.keys[cur ^ 1],
+                                                              W.vals[cur ^ 1], G, shift, W.hist);
+        cur ^= 1;
+    }
+    uint64_t *keys = W.keys[cur];
+    uint64_t *scratch = W.keys[cur ^ 1];
+    uint32_t *sa = W.vals[cur];
+    // 1c. round-0 groups (lists buffer 0)
+    groups0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(keys, sa, G, W.rank, W.lists[0][0], W.lists[0][1],
+                                                       W.counts);
+    // 1d. doubling rounds while some string is longer than the sorted depth
+    int lb = 0;
+    const unsigned wgrid = kNumSMs * 8;   // 8 CTAs of 8 warps per SM, grid-stride over groups
+    for (int64_t h = G.D0; h < T; h *= 2) {
+        int *cnt = W.counts + 2 * lb;
+        int *cnt_next = W.counts + 2 * (lb ^ 1);
+        dbl_keys_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, h, sa, W.rank, W.k2);
+        dbl_sort_small_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], cnt, sa, W.k2);
+        dbl_sort_large_kernel<<<kNumSMs * 2, kLargeThreads, 0, st>>>(W.lists[lb][1], cnt, sa, W.k2, scratch);
+        if ((err = cudaMemsetAsync(cnt_next, 0, 2 * sizeof(int), st)) != cudaSuccess) return err;
+        dbl_regroup_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, 2 * h, sa, W.k2, W.rank,
+                                                  W.lists[lb ^ 1][0], W.lists[lb ^ 1][1], cnt_next);
+        lb ^= 1;
+    }
+    // 2. LCP
+    lcp_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, keys, sa, W.lcp);
+    // 3a. summaries
+    summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1,
+                                                                        W.minpos2, W.emin2);
+    // 3b. resolve
+    resolve_kernel<<<grid_for(G.N, 128), 128, 0, st>>>(G, vs, sa, W.lcp, W.minpos1, W.emin1, W.minpos2, W.emin2,
+                                                       end_idx, len, sym);
+    return cudaGetLastError();
+}
+
+}  // namespace rosa
