@@ -60,6 +60,7 @@ struct Geometry {
     int bps, D0, abits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
+    int wbits, ntw, nw;      // wavelet matrix: levels, 2048-element tiles and 64-bit words per stream
 };
 
 Geometry make_geometry(int S, int T, int K, int g, bool same) {
@@ -78,6 +79,11 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     G.ntps = ceil_div(G.n, kRadixTile);
     G.nb1 = ceil_div(G.n, kL1);
     G.nb2 = ceil_div(G.n, kL2);
+    int wb = 0;
+    while ((1 << wb) < T) ++wb;   // key positions 0..T-1
+    G.wbits = wb < 1 ? 1 : wb;
+    G.ntw = ceil_div(T, 2048);
+    G.nw = (T >> 6) + 1;
     return G;
 }
 
@@ -91,7 +97,14 @@ struct Workspace {
     uint32_t *k2;
     uint32_t *hist;
     int2 *lists[2][2];       // [buffer][0 = small, 1 = large]
-    int32_t *minpos1, *emin1, *minpos2, *emin2;
+    int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2;
+    int32_t *hard;           // ranks of queries left for the warp-cooperative phase
+    int32_t *kcount;         // keys before each rank (q != k)
+    int *ktile;              // keys per 2048-rank tile
+    uint32_t *wvals[2];      // wavelet level sequences
+    int *wcnt;               // [level][stream][tile] ones per wavelet tile
+    void *words;             // [stream][level][word] rank directory + bits (16 B each)
+    int *wz;                 // [stream][level] zeros per level
     size_t bytes;
 };
 
@@ -123,8 +136,17 @@ Workspace carve(const Geometry &G, void *base) {
         for (int j = 0; j < 2; ++j) W.lists[i][j] = (int2 *)take(list_cap * sizeof(int2));
     W.minpos1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
     W.emin1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
+    W.ein1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
     W.minpos2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.emin2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
+    W.hard = (int32_t *)take(N * 4);
+    W.kcount = (int32_t *)take(N * 4);
+    W.ktile = (int *)take((size_t)G.S * G.ntps * 4);
+    W.wvals[0] = (uint32_t *)take((size_t)G.S * G.T * 4);
+    W.wvals[1] = (uint32_t *)take((size_t)G.S * G.T * 4);
+    W.wcnt = (int *)take((size_t)G.wbits * G.S * G.ntw * 4);
+    W.words = take((size_t)G.S * G.wbits * G.nw * 16);
+    W.wz = (int *)take((size_t)G.S * G.wbits * 4);
     W.bytes = off;
     return W;
 }
@@ -475,7 +497,8 @@ __global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restr
 
 // ---------------------------------------------------------------------------
 // 3a. Block summaries: smallest key position and smallest inner LCP (edges
-//     strictly inside the block) per 32 and per 1024 ranks.
+//     strictly inside the block) per 32 and per 1024 ranks, and the LCP edge
+//     entering each 32-block from below.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
     return (same || (int)x < T) ? (int)x : INT_MAX;
@@ -483,7 +506,7 @@ __device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
 
 __global__ void __launch_bounds__(kL2)
 summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__restrict__ lcp,
-               int32_t *__restrict__ minpos1, int32_t *__restrict__ emin1,
+               int32_t *__restrict__ minpos1, int32_t *__restrict__ emin1, int32_t *__restrict__ ein1,
                int32_t *__restrict__ minpos2, int32_t *__restrict__ emin2) {
     __shared__ int wpos[32], wemin[32], wfirst[32];
     const int s = blockIdx.x / G.nb2, B2 = blockIdx.x - s * G.nb2;
@@ -507,6 +530,7 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
         if (b1 < G.nb1) {
             minpos1[(int64_t)s * G.nb1 + b1] = mp;
             emin1[(int64_t)s * G.nb1 + b1] = me;
+            ein1[(int64_t)s * G.nb1 + b1] = first;
         }
         wpos[warp] = mp;
         wemin[warp] = me;
@@ -528,163 +552,409 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
 }
 
 // ---------------------------------------------------------------------------
-// 3b. Per-query resolution in rank order.
+// 3b. Wavelet matrix over the key positions in rank order, for the query
+//     "largest key position <= X among ranks [lo, hi]" in O(log T).  One
+//     stable partition by bit per level, most significant bit first; each
+//     level stores its bits with the count of ones before every 64-bit word.
 // ---------------------------------------------------------------------------
+constexpr int kWTile = 2048;
+
+struct __align__(16) WWord {
+    uint32_t cum;
+    uint32_t pad;
+    unsigned long long bits;
+};
+
+// Keys per 2048-rank tile of the sorted order (q != k only).
+__global__ void __launch_bounds__(256)
+key_tile_count_kernel(Geometry G, const uint32_t *__restrict__ sa, int *__restrict__ ktile) {
+    __shared__ int red[8];
+    const int s = blockIdx.x / G.ntps, tt = blockIdx.x - s * G.ntps;
+    const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
+    const int lim = min(kRadixTile, G.n - tt * kRadixTile);
+    int c = 0;
+    for (int i = threadIdx.x; i < lim; i += 256) c += (int)sa[base + i] < G.T ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(ROSA_FULL_MASK, c, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        ktile[(int64_t)s * G.ntps + tt] = t;
+    }
+}
+
+// Level-0 sequence (key positions in rank order), the exclusive key count
+// before every rank (q != k), and the level-0 ones per wavelet tile.
+__global__ void __launch_bounds__(256)
+wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, const int *__restrict__ ktile,
+                       int32_t *__restrict__ kcount, uint32_t *__restrict__ a0, int *__restrict__ wcnt0) {
+    __shared__ int wk[8];
+    __shared__ int pre_s;
+    const int s = blockIdx.x / G.ntps, tt = blockIdx.x - s * G.ntps;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
+    const int lim = min(kRadixTile, G.n - tt * kRadixTile);
+    const int ntw = ceil_div(G.T, kWTile);
+    if (threadIdx.x == 0) {
+        int p = 0;
+        if (G.same) p = tt * kRadixTile;
+        else for (int i = 0; i < tt; ++i) p += ktile[(int64_t)s * G.ntps + i];
+        pre_s = p;
+    }
+    __syncthreads();
+    int run = pre_s;
+    for (int u = 0; u < kRadixIPT; ++u) {
+        const int i = u * 256 + threadIdx.x;
+        const bool ok = i < lim;
+        const uint32_t x = ok ? sa[base + i] : 0u;
+        const bool key = ok && (G.same || (int)x < G.T);
+        const unsigned bal = __ballot_sync(ROSA_FULL_MASK, key);
+        if (lane == 0) wk[warp] = __popc(bal);
+        __syncthreads();
+        int wpre = 0, rtot = 0;
+        for (int w = 0; w < 8; ++w) {
+            if (w < warp) wpre += wk[w];
+            rtot += wk[w];
+        }
+        const int kidx = run + wpre + __popc(bal & lanemask_lt());
+        if (ok && !G.same) kcount[base + i] = kidx;
+        if (key) {
+            a0[(int64_t)s * G.T + kidx] = x;
+            if ((x >> (nbits - 1)) & 1u) atomicAdd(&wcnt0[(int64_t)s * ntw + kidx / kWTile], 1);
+        }
+        run += rtot;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(256)
+wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__ in, uint32_t *__restrict__ out,
+                     int *__restrict__ wcnt, WWord *__restrict__ words, int *__restrict__ wz) {
+    __shared__ uint32_t ballots[kWTile / 32];
+    __shared__ int wones[8];
+    __shared__ int red_a[8], red_t[8];
+    const int ntw = ceil_div(G.T, kWTile), nw = (G.T >> 6) + 1;
+    const int s = blockIdx.x / ntw, tt = blockIdx.x - s * ntw;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int b = nbits - 1 - lv;
+    const int *cnt = wcnt + ((int64_t)lv * G.S + s) * ntw;
+    int a = 0, tot = 0;
+    for (int i = threadIdx.x; i < ntw; i += 256) {
+        const int c = cnt[i];
+        tot += c;
+        if (i < tt) a += c;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        a += __shfl_xor_sync(ROSA_FULL_MASK, a, o);
+        tot += __shfl_xor_sync(ROSA_FULL_MASK, tot, o);
+    }
+    if (lane == 0) { red_a[warp] = a; red_t[warp] = tot; }
+    __syncthreads();
+    int ones_before = 0, total_ones = 0;
+    for (int w = 0; w < 8; ++w) { ones_before += red_a[w]; total_ones += red_t[w]; }
+    const int Z = G.T - total_ones;
+    const int zeros_before = tt * kWTile - ones_before;
+    const int lim = min(kWTile, G.T - tt * kWTile);
+    const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
+    uint32_t *dst = out + (int64_t)s * G.T;
+    int *cnt_next = wcnt + ((int64_t)(lv + 1) * G.S + s) * ntw;
+    int run = 0;
+    for (int u = 0; u < kWTile / 256; ++u) {
+        const int i = u * 256 + threadIdx.x;
+        const bool ok = i < lim;
+        const uint32_t v = ok ? src[i] : 0u;
+        const int bit = ok ? (int)((v >> b) & 1u) : 0;
+        const unsigned bal = __ballot_sync(ROSA_FULL_MASK, bit);
+        if (lane == 0) {
+            ballots[u * 8 + warp] = bal;
+            wones[warp] = __popc(bal);
+        }
+        __syncthreads();
+        int wpre = 0, rtot = 0;
+        for (int w = 0; w < 8; ++w) {
+            if (w < warp) wpre += wones[w];
+            rtot += wones[w];
+        }
+        const int lo1 = run + wpre + __popc(bal & lanemask_lt());
+        if (ok) {
+            const int d = bit ? Z + ones_before + lo1 : zeros_before + (i - lo1);
+            dst[d] = v;
+            if (lv + 1 < nbits && ((v >> (b - 1)) & 1u)) atomicAdd(&cnt_next[d / kWTile], 1);
+        }
+        run += rtot;
+        __syncthreads();
+    }
+    if (threadIdx.x < 32) {
+        const int k = threadIdx.x;
+        const unsigned long long bits =
+            (unsigned long long)ballots[2 * k] | ((unsigned long long)ballots[2 * k + 1] << 32);
+        const int pc = __popcll(bits);
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(ROSA_FULL_MASK, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (k * 64 < lim) {
+            WWord w;
+            w.cum = (uint32_t)(ones_before + incl - pc);
+            w.pad = 0;
+            w.bits = bits;
+            words[((int64_t)s * nbits + lv) * nw + tt * 32 + k] = w;
+        }
+    }
+    if (threadIdx.x == 0) {
+        if (tt == ntw - 1 && (G.T & 63) == 0) {
+            WWord w;
+            w.cum = (uint32_t)total_ones;
+            w.pad = 0;
+            w.bits = 0ull;
+            words[((int64_t)s * nbits + lv) * nw + (G.T >> 6)] = w;
+        }
+        if (tt == 0) wz[(int64_t)s * nbits + lv] = Z;
+    }
+}
+
+__device__ __forceinline__ int wrank1(const WWord *W, int i) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(W + (i >> 6)));
+    const unsigned long long bits = ((unsigned long long)raw.w << 32) | raw.z;
+    const unsigned long long mask = (i & 63) ? ((1ull << (i & 63)) - 1ull) : 0ull;
+    return (int)raw.x + __popcll(bits & mask);
+}
+
+// Largest value <= X in positions [l, r) of the level-0 sequence, or -1.
+__device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, int l, int r, int X) {
+    if (l >= r || X < 0) return -1;
+    const int top = (1 << nbits) - 1;
+    if (X > top) X = top;
+    int alt_lv = -1, alt_l = 0, alt_r = 0;
+    bool alive = true;
+    for (int lv = 0; lv < nbits; ++lv) {
+        const int b = nbits - 1 - lv;
+        const WWord *Wl = W + (int64_t)lv * nw;
+        const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
+        const int zl = l - ol, zr = r - orr;
+        if ((X >> b) & 1) {
+            if (zr > zl) { alt_lv = lv; alt_l = zl; alt_r = zr; }
+            l = Z[lv] + ol;
+            r = Z[lv] + orr;
+        } else {
+            l = zl;
+            r = zr;
+        }
+        if (l >= r) { alive = false; break; }
+    }
+    if (alive) return X;
+    if (alt_lv < 0) return -1;
+    int val = (X >> (nbits - alt_lv)) << (nbits - alt_lv);
+    l = alt_l;
+    r = alt_r;
+    for (int lv = alt_lv + 1; lv < nbits; ++lv) {
+        const int b = nbits - 1 - lv;
+        const WWord *Wl = W + (int64_t)lv * nw;
+        const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
+        if (orr > ol) {
+            val |= 1 << b;
+            l = Z[lv] + ol;
+            r = Z[lv] + orr;
+        } else {
+            l -= ol;
+            r -= orr;
+        }
+    }
+    return val;
+}
+
+// ---------------------------------------------------------------------------
+// 3c. Per-query resolution.  Phase 1: one thread per query in rank order,
+//     with a budget of rank visits; queries that exhaust it go to a list.
+//     Phase 2: one warp per listed query, 32 ranks or 32 blocks per step.
+//     The most recent end comes from the visited ranks when the whole
+//     interval was visited, else from the wavelet matrix.
+// ---------------------------------------------------------------------------
+constexpr int kEasyBudget = 64;        // rank visits a thread spends before handing off
+
 struct StreamView {
     const uint32_t *sa;
     const int32_t *lcp;
-    const int32_t *mp1, *em1, *mp2, *em2;
-    int n, T;
+    const int32_t *mp1, *em1, *ein1, *mp2, *em2;
+    const int32_t *kcount;
+    const WWord *W;
+    const int *Z;
+    int n, T, nb1, nbits, nw;
     bool same;
 };
 
 __device__ __forceinline__ int kpos(const StreamView &v, int r) { return key_pos_or_inf(v.sa[r], v.T, v.same); }
 
-// LCP with the nearest admissible key (position <= X) at a lower rank than j,
-// or 0 if the running LCP falls to `stop` or below before one is found.
-__device__ int nearest_left(const StreamView &v, int j, int X, int stop) {
+// number of keys at ranks below r (r in [0, n])
+__device__ __forceinline__ int kc(const StreamView &v, int r) {
+    if (v.same) return r;
+    return r < v.n ? v.kcount[r] : v.T;
+}
+
+struct ResolveArgs {
+    const uint32_t *sa;
+    const int32_t *lcp, *mp1, *em1, *ein1, *mp2, *em2, *kcount;
+    const WWord *words;
+    const int *wz;
+    int nbits;
+};
+
+__device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const ResolveArgs &A) {
+    const int64_t seg = (int64_t)s * G.n;
+    const int nw = (G.T >> 6) + 1;
+    return StreamView{A.sa + seg, A.lcp + seg, A.mp1 + (int64_t)s * G.nb1, A.em1 + (int64_t)s * G.nb1,
+                      A.ein1 + (int64_t)s * G.nb1, A.mp2 + (int64_t)s * G.nb2, A.em2 + (int64_t)s * G.nb2,
+                      A.kcount ? A.kcount + seg : nullptr, A.words + (int64_t)s * A.nbits * nw,
+                      A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, A.nbits, nw, G.same};
+}
+
+// Serial scans with a shared visit budget; each returns false when the
+// budget ran out before its answer was known.
+// nearest_*: LCP with the nearest admissible key (position <= X) if > stop, else 0.
+__device__ bool nearest_left(const StreamView &v, int j, int X, int stop, int &budget, int &out) {
+    int m = INT_MAX, r = j - 1;
+    out = 0;
+    while (r >= 0) {
+        if (--budget < 0) return false;
+        if ((r & (kL2 - 1)) == kL2 - 1) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em2[b]));
+                if (m <= stop) return true;
+                r -= kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == kL1 - 1) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r + 1], v.em1[b]));
+                if (m <= stop) return true;
+                r -= kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r + 1]);
+        if (m <= stop) return true;
+        if (kpos(v, r) <= X) { out = m; return true; }
+        --r;
+    }
+    return true;
+}
+
+__device__ bool nearest_right(const StreamView &v, int j, int X, int stop, int &budget, int &out) {
+    int m = INT_MAX, r = j + 1;
+    out = 0;
+    while (r < v.n) {
+        if (--budget < 0) return false;
+        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
+            const int b = r / kL2;
+            if (v.mp2[b] > X) {
+                m = min(m, min(v.lcp[r], v.em2[b]));
+                if (m <= stop) return true;
+                r += kL2;
+                continue;
+            }
+        }
+        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
+            const int b = r / kL1;
+            if (v.mp1[b] > X) {
+                m = min(m, min(v.lcp[r], v.em1[b]));
+                if (m <= stop) return true;
+                r += kL1;
+                continue;
+            }
+        }
+        m = min(m, v.lcp[r]);
+        if (m <= stop) return true;
+        if (kpos(v, r) <= X) { out = m; return true; }
+        ++r;
+    }
+    return true;
+}
+
+// bound_*: walk away from j while the running LCP stays >= L.  `edge` gets
+// the last rank inside (j if none); `best` the largest admissible position
+// among visited ranks; `skipped` is set when a block holding admissible keys
+// was crossed without visiting its ranks.
+__device__ bool bound_left(const StreamView &v, int j, int X, int L, int &budget, int &edge, int &best,
+                           bool &skipped) {
     int m = INT_MAX, r = j - 1;
     while (r >= 0) {
+        if (--budget < 0) return false;
         if ((r & (kL2 - 1)) == kL2 - 1) {
             const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em2[b]));
-                if (m <= stop) return 0;
+            const int mm = min(m, min(v.lcp[r + 1], v.em2[b]));
+            if (mm >= L) {
+                m = mm;
+                skipped |= v.mp2[b] <= X;
                 r -= kL2;
                 continue;
             }
         }
         if ((r & (kL1 - 1)) == kL1 - 1) {
             const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em1[b]));
-                if (m <= stop) return 0;
+            const int mm = min(m, min(v.lcp[r + 1], v.em1[b]));
+            if (mm >= L) {
+                m = mm;
+                skipped |= v.mp1[b] <= X;
                 r -= kL1;
                 continue;
             }
         }
         m = min(m, v.lcp[r + 1]);
-        if (m <= stop) return 0;
-        if (kpos(v, r) <= X) return m;
+        if (m < L) break;
+        const int p = kpos(v, r);
+        if (p <= X) best = max(best, p);
         --r;
     }
-    return 0;
+    edge = r + 1;
+    return true;
 }
 
-__device__ int nearest_right(const StreamView &v, int j, int X, int stop) {
+__device__ bool bound_right(const StreamView &v, int j, int X, int L, int &budget, int &edge, int &best,
+                            bool &skipped) {
     int m = INT_MAX, r = j + 1;
     while (r < v.n) {
+        if (--budget < 0) return false;
         if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
             const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r], v.em2[b]));
-                if (m <= stop) return 0;
+            const int mm = min(m, min(v.lcp[r], v.em2[b]));
+            if (mm >= L) {
+                m = mm;
+                skipped |= v.mp2[b] <= X;
                 r += kL2;
                 continue;
             }
         }
         if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
             const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r], v.em1[b]));
-                if (m <= stop) return 0;
+            const int mm = min(m, min(v.lcp[r], v.em1[b]));
+            if (mm >= L) {
+                m = mm;
+                skipped |= v.mp1[b] <= X;
                 r += kL1;
                 continue;
             }
         }
         m = min(m, v.lcp[r]);
-        if (m <= stop) return 0;
-        if (kpos(v, r) <= X) return m;
-        ++r;
-    }
-    return 0;
-}
-
-// Largest admissible key position among ranks below j whose LCP with j is >= L.
-__device__ int latest_left(const StreamView &v, int j, int X, int L) {
-    int best = -1, m = INT_MAX, r = j - 1;
-    while (r >= 0) {
-        if ((r & (kL2 - 1)) == kL2 - 1) {
-            const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em2[b]));
-                if (m < L) return best;
-                r -= kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == kL1 - 1) {
-            const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em1[b]));
-                if (m < L) return best;
-                r -= kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r + 1]);
-        if (m < L) return best;
-        const int p = kpos(v, r);
-        if (p <= X) best = max(best, p);
-        --r;
-    }
-    return best;
-}
-
-__device__ int latest_right(const StreamView &v, int j, int X, int L) {
-    int best = -1, m = INT_MAX, r = j + 1;
-    while (r < v.n) {
-        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
-            const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r], v.em2[b]));
-                if (m < L) return best;
-                r += kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
-            const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r], v.em1[b]));
-                if (m < L) return best;
-                r += kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r]);
-        if (m < L) return best;
+        if (m < L) break;
         const int p = kpos(v, r);
         if (p <= X) best = max(best, p);
         ++r;
     }
-    return best;
+    edge = r - 1;
+    return true;
 }
 
-__global__ void resolve_kernel(Geometry G, const uint8_t *__restrict__ vsym, const uint32_t *__restrict__ sa,
-                               const int32_t *__restrict__ lcp, const int32_t *__restrict__ minpos1,
-                               const int32_t *__restrict__ emin1, const int32_t *__restrict__ minpos2,
-                               const int32_t *__restrict__ emin2, int32_t *__restrict__ end_idx,
-                               int32_t *__restrict__ len, int32_t *__restrict__ sym) {
-    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (gi >= G.N) return;
-    const int s = (int)(gi / G.n);
-    const int j = (int)(gi - (int64_t)s * G.n);
-    const int64_t seg = (int64_t)s * G.n;
-    const uint32_t x = sa[gi];
-    if (!G.same && (int)x < G.T) return;          // key item: nothing to answer
-    const int t = G.same ? (int)x : (int)x - G.T;
+__device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *vsym, int s, int t, int L, int ib,
+                                             int32_t *end_idx, int32_t *len, int32_t *sym) {
     const int64_t o = (int64_t)s * G.T + t;
-    const int X = t - G.g;
-    int L = 0, ib = -1;
-    if (X >= 0) {
-        StreamView v{sa + seg, lcp + seg, minpos1 + (int64_t)s * G.nb1, emin1 + (int64_t)s * G.nb1,
-                     minpos2 + (int64_t)s * G.nb2, emin2 + (int64_t)s * G.nb2, G.n, G.T, G.same};
-        const int bl = nearest_left(v, j, X, 0);
-        const int br = nearest_right(v, j, X, bl);
-        L = max(bl, br);
-        if (L > 0) ib = max(latest_left(v, j, X, L), latest_right(v, j, X, L));
-    }
     if (L > 0 && ib >= 0) {
         end_idx[o] = ib;
         len[o] = L;
@@ -693,6 +963,171 @@ __global__ void resolve_kernel(Geometry G, const uint8_t *__restrict__ vsym, con
         end_idx[o] = -1;
         len[o] = 0;
         sym[o] = -1;
+    }
+}
+
+__global__ void resolve_easy_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
+                                    int32_t *__restrict__ end_idx, int32_t *__restrict__ len,
+                                    int32_t *__restrict__ sym, int32_t *__restrict__ hard, int *hard_count) {
+    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gi >= G.N) return;
+    const int s = (int)(gi / G.n);
+    const int j = (int)(gi - (int64_t)s * G.n);
+    const uint32_t x = A.sa[gi];
+    if (!G.same && (int)x < G.T) return;          // key item: nothing to answer
+    const int t = G.same ? (int)x : (int)x - G.T;
+    const int X = t - G.g;
+    int L = 0, ib = -1;
+    if (X >= 0) {
+        const StreamView v = make_view(G, s, A);
+        int budget = kEasyBudget, bl = 0, br = 0;
+        bool ok = nearest_left(v, j, X, 0, budget, bl) && nearest_right(v, j, X, bl, budget, br);
+        if (ok) {
+            L = max(bl, br);
+            if (L > 0) {
+                int lo = j, hi = j, best = -1;
+                bool skipped = false;
+                ok = bound_left(v, j, X, L, budget, lo, best, skipped) &&
+                     bound_right(v, j, X, L, budget, hi, best, skipped);
+                if (ok) ib = skipped ? wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, lo), kc(v, hi + 1), X) : best;
+            }
+        }
+        if (!ok) {
+            hard[atomicAdd(hard_count, 1)] = (int32_t)gi;
+            return;
+        }
+    }
+    write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+}
+
+// ---- warp-cooperative scans -------------------------------------------------
+
+__device__ __forceinline__ int warp_prefix_min(int x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(ROSA_FULL_MASK, x, o);
+        if (lane >= o) x = min(x, y);
+    }
+    return x;
+}
+
+// NEAREST: LCP with the first admissible key in direction dir if > lim, else 0.
+// BOUND: the last rank in direction dir whose running LCP stays >= lim.
+enum ScanMode { NEAREST = 0, BOUND = 1 };
+
+// One step over up to 32 consecutive ranks: lane i visits first + dir*i when
+// i < cnt.  Returns true when the scan has ended (result set).
+template <int MODE>
+__device__ bool warp_fine(const StreamView &v, int first, int cnt, int dir, int X, int lim, int lane, int &carry,
+                          int &result) {
+    const int r = first + dir * lane;
+    const bool act = lane < cnt && r >= 0 && r < v.n;
+    int e = INT_MAX;
+    bool valid = false;
+    if (act) {
+        e = dir < 0 ? v.lcp[r + 1] : v.lcp[r];
+        if (MODE == NEAREST) valid = kpos(v, r) <= X;
+    } else if (lane < cnt) {
+        e = -1;   // ran off the stream: ends every scan
+    }
+    const int m = min(carry, warp_prefix_min(e, lane));
+    if (MODE == NEAREST) {
+        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && m <= lim);
+        const unsigned valm = __ballot_sync(ROSA_FULL_MASK, valid && m > lim);
+        const int fs = stopm ? __ffs(stopm) - 1 : 32;
+        const int fv = valm ? __ffs(valm) - 1 : 32;
+        if (fv < fs) {
+            result = __shfl_sync(ROSA_FULL_MASK, m, fv);
+            return true;
+        }
+        if (fs < 32) {
+            result = 0;
+            return true;
+        }
+    } else {
+        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && m < lim);
+        if (stopm) {
+            const int fs = __ffs(stopm) - 1;
+            result = first + dir * (fs - 1);
+            return true;
+        }
+        result = first + dir * (cnt - 1);
+    }
+    carry = __shfl_sync(ROSA_FULL_MASK, m, 31);
+    return false;
+}
+
+template <int MODE>
+__device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, int lane) {
+    int carry = INT_MAX;
+    int result = MODE == NEAREST ? 0 : j;
+    int next = j + dir;
+    if (next < 0 || next >= v.n) return result;
+    const int cnt = dir < 0 ? (next & (kL1 - 1)) + 1 : kL1 - (next & (kL1 - 1));
+    if (warp_fine<MODE>(v, next, cnt, dir, X, lim, lane, carry, result)) return result;
+    next += dir * cnt;
+    // `next` is now the last (dir < 0) or first (dir > 0) rank of block next / 32
+    while (next >= 0 && next < v.n) {
+        const int nb = next / kL1;
+        const int b = nb + dir * lane;
+        const bool inside = b >= 0 && b < v.nb1 && (b + 1) * kL1 <= v.n;
+        int bm = -1;
+        bool has_valid = true;
+        if (inside) {
+            const int edge = dir < 0 ? ((b + 1) * kL1 < v.n ? v.ein1[b + 1] : INT_MAX) : v.ein1[b];
+            bm = min(edge, v.em1[b]);
+            has_valid = v.mp1[b] <= X;
+        }
+        const int M = min(carry, warp_prefix_min(bm, lane));
+        const bool stop_here = MODE == NEAREST ? (!inside || has_valid || M <= lim) : (!inside || M < lim);
+        const unsigned sm = __ballot_sync(ROSA_FULL_MASK, stop_here);
+        const int f = sm ? __ffs(sm) - 1 : 32;
+        if (f > 0) {
+            carry = min(carry, __shfl_sync(ROSA_FULL_MASK, M, f - 1));
+            if (MODE == BOUND) {
+                const int bl = nb + dir * (f - 1);
+                result = dir < 0 ? bl * kL1 : bl * kL1 + kL1 - 1;
+            }
+            if (f == 32) {
+                next += dir * kL1 * 32;
+                continue;
+            }
+        }
+        const int bb = nb + dir * f;
+        const int first = dir < 0 ? bb * kL1 + kL1 - 1 : bb * kL1;
+        if (first < 0 || first >= v.n) break;
+        if (warp_fine<MODE>(v, first, kL1, dir, X, lim, lane, carry, result)) return result;
+        next = first + dir * kL1;
+    }
+    return result;
+}
+
+__global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
+                                    int32_t *__restrict__ end_idx, int32_t *__restrict__ len,
+                                    int32_t *__restrict__ sym, const int32_t *__restrict__ hard,
+                                    const int *__restrict__ hard_count) {
+    const int nh = *hard_count;
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t h = wid; h < nh; h += nw) {
+        const int64_t gi = hard[h];
+        const int s = (int)(gi / G.n);
+        const int j = (int)(gi - (int64_t)s * G.n);
+        const uint32_t x = A.sa[gi];
+        const int t = G.same ? (int)x : (int)x - G.T;
+        const int X = t - G.g;
+        const StreamView v = make_view(G, s, A);
+        const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
+        const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
+        const int L = max(bl, br);
+        int ib = -1;
+        if (L > 0) {
+            const int lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
+            const int hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
+            if (lane == 0) ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, lo), kc(v, hi + 1), X);
+        }
+        if (lane == 0) write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
     }
 }
 
@@ -706,8 +1141,9 @@ int match_launch_count(int S, int T, int K, bool same) {
     int rounds = 0;
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits, kRadixBits);
-    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + lcp + summary + resolve
-    return 1 + 3 * passes + 1 + 4 * rounds + 3;
+    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + lcp + summary
+    // + wavelet (key count when q != k, compaction, one per level) + 2 resolve
+    return 1 + 3 * passes + 1 + 4 * rounds + 2 + (same ? 0 : 1) + 1 + G.wbits + 2;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -762,11 +1198,23 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     // 2. LCP
     lcp_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, keys, sa, W.lcp);
     // 3a. summaries
-    summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1,
-                                                                        W.minpos2, W.emin2);
-    // 3b. resolve
-    resolve_kernel<<<grid_for(G.N, 128), 128, 0, st>>>(G, vs, sa, W.lcp, W.minpos1, W.emin1, W.minpos2, W.emin2,
-                                                       end_idx, len, sym);
+    summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
+                                                           W.minpos2, W.emin2);
+    // 3b. wavelet matrix over key positions in rank order
+    if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wbits * G.S * G.ntw * 4, st)) != cudaSuccess) return err;
+    if (!G.same) key_tile_count_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile);
+    wavelet_compact_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, G.wbits, sa, W.ktile, W.kcount, W.wvals[0],
+                                                                      W.wcnt);
+    WWord *words = static_cast<WWord *>(W.words);
+    for (int lv = 0; lv < G.wbits; ++lv)
+        wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, G.wbits, lv, W.wvals[lv & 1],
+                                                                       W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
+    // 3c. resolve: thread per query, then warp per query for the long scans
+    ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, G.same ? nullptr : W.kcount,
+                  words, W.wz, G.wbits};
+    int *hard_count = W.counts + 4;
+    resolve_easy_kernel<<<grid_for(G.N, 128), 128, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
+    resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
     return cudaGetLastError();
 }
 

@@ -49,7 +49,7 @@ int rosa_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int 
                int32_t *end_idx, int32_t *len, int32_t *sym, void *workspace, size_t ws_bytes,
                cudaStream_t stream) {
     if (!match_sizes_ok(S, T, K) || g < 1) return ROSA_ERR_INVALID_ARG;
-    if (S > 0 && (!q || !k || !end_idx || !len || !sym)) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)S * T > 0 && (!q || !k || !end_idx || !len || !sym)) return ROSA_ERR_INVALID_ARG;
     if (!workspace || !aligned(workspace, 256)) return ROSA_ERR_WORKSPACE;
     if (ws_bytes < rosa::match_workspace_bytes(S, T, K, q == k)) return ROSA_ERR_WORKSPACE;
     return cuda_status(rosa::launch_match(q, k, v, S, T, K, g, end_idx, len, sym, workspace, ws_bytes, stream));
