@@ -661,6 +661,12 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
     const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
     uint32_t *dst = out + (int64_t)s * G.T;
     int *cnt_next = wcnt + ((int64_t)(lv + 1) * G.S + s) * ntw;
+    // zeros of this tile land in one contiguous range and ones in another, so
+    // the next level's per-tile counts touch at most four tiles: count them here
+    __shared__ int nxt[4];
+    const int zr0 = zeros_before / kWTile, or0 = (Z + ones_before) / kWTile;
+    if (threadIdx.x < 4) nxt[threadIdx.x] = 0;
+    __syncthreads();
     int run = 0;
     for (int u = 0; u < kWTile / 256; ++u) {
         const int i = u * 256 + threadIdx.x;
@@ -682,10 +688,18 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         if (ok) {
             const int d = bit ? Z + ones_before + lo1 : zeros_before + (i - lo1);
             dst[d] = v;
-            if (lv + 1 < nbits && ((v >> (b - 1)) & 1u)) atomicAdd(&cnt_next[d / kWTile], 1);
+            if (lv + 1 < nbits && ((v >> (b - 1)) & 1u)) {
+                const int dt = d / kWTile;
+                atomicAdd(&nxt[bit ? 2 + (dt - or0) : (dt - zr0)], 1);
+            }
         }
         run += rtot;
         __syncthreads();
+    }
+    if (lv + 1 < nbits && threadIdx.x < 4) {
+        const int c = nxt[threadIdx.x];
+        const int dt = threadIdx.x < 2 ? zr0 + threadIdx.x : or0 + threadIdx.x - 2;
+        if (c) atomicAdd(&cnt_next[dt], c);
     }
     if (threadIdx.x < 32) {
         const int k = threadIdx.x;
@@ -769,13 +783,23 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
 }
 
 // ---------------------------------------------------------------------------
-// 3c. Per-query resolution.  Phase 1: one thread per query in rank order,
-//     with a budget of rank visits; queries that exhaust it go to a list.
-//     Phase 2: one warp per listed query, 32 ranks or 32 blocks per step.
-//     The most recent end comes from the visited ranks when the whole
-//     interval was visited, else from the wavelet matrix.
+// 3c. Per-query resolution.
+//     Phase 1 (resolve_tile_kernel): a CTA stages 1024 ranks plus 1024 on
+//     each side (key position, LCP edge) in shared memory and resolves the
+//     tile's queries there.  The nearest admissible key on each side gives L;
+//     the interval scan then continues from that key, so every rank is
+//     visited about once.  Queries whose scans would leave the staged window
+//     or exceed a visit budget go to a list.
+//     Phase 2 (resolve_hard_kernel): one warp per listed query scans global
+//     memory 32 ranks or 32 blocks per step for L and the interval bounds;
+//     the most recent admissible end comes from the wavelet matrix, 32
+//     queries per warp in parallel.
 // ---------------------------------------------------------------------------
-constexpr int kEasyBudget = 64;        // rank visits a thread spends before handing off
+constexpr int kRTile = 1024;
+constexpr int kRHalo = 1024;
+constexpr int kRWin = kRTile + 2 * kRHalo;
+constexpr int kRBudget = 1024;         // shared-memory rank visits per query
+constexpr int kRThreads = 256;
 
 struct StreamView {
     const uint32_t *sa;
@@ -813,145 +837,6 @@ __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const 
                       A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, A.nbits, nw, G.same};
 }
 
-// Serial scans with a shared visit budget; each returns false when the
-// budget ran out before its answer was known.
-// nearest_*: LCP with the nearest admissible key (position <= X) if > stop, else 0.
-__device__ bool nearest_left(const StreamView &v, int j, int X, int stop, int &budget, int &out) {
-    int m = INT_MAX, r = j - 1;
-    out = 0;
-    while (r >= 0) {
-        if (--budget < 0) return false;
-        if ((r & (kL2 - 1)) == kL2 - 1) {
-            const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em2[b]));
-                if (m <= stop) return true;
-                r -= kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == kL1 - 1) {
-            const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r + 1], v.em1[b]));
-                if (m <= stop) return true;
-                r -= kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r + 1]);
-        if (m <= stop) return true;
-        if (kpos(v, r) <= X) { out = m; return true; }
-        --r;
-    }
-    return true;
-}
-
-__device__ bool nearest_right(const StreamView &v, int j, int X, int stop, int &budget, int &out) {
-    int m = INT_MAX, r = j + 1;
-    out = 0;
-    while (r < v.n) {
-        if (--budget < 0) return false;
-        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
-            const int b = r / kL2;
-            if (v.mp2[b] > X) {
-                m = min(m, min(v.lcp[r], v.em2[b]));
-                if (m <= stop) return true;
-                r += kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
-            const int b = r / kL1;
-            if (v.mp1[b] > X) {
-                m = min(m, min(v.lcp[r], v.em1[b]));
-                if (m <= stop) return true;
-                r += kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r]);
-        if (m <= stop) return true;
-        if (kpos(v, r) <= X) { out = m; return true; }
-        ++r;
-    }
-    return true;
-}
-
-// bound_*: walk away from j while the running LCP stays >= L.  `edge` gets
-// the last rank inside (j if none); `best` the largest admissible position
-// among visited ranks; `skipped` is set when a block holding admissible keys
-// was crossed without visiting its ranks.
-__device__ bool bound_left(const StreamView &v, int j, int X, int L, int &budget, int &edge, int &best,
-                           bool &skipped) {
-    int m = INT_MAX, r = j - 1;
-    while (r >= 0) {
-        if (--budget < 0) return false;
-        if ((r & (kL2 - 1)) == kL2 - 1) {
-            const int b = r / kL2;
-            const int mm = min(m, min(v.lcp[r + 1], v.em2[b]));
-            if (mm >= L) {
-                m = mm;
-                skipped |= v.mp2[b] <= X;
-                r -= kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == kL1 - 1) {
-            const int b = r / kL1;
-            const int mm = min(m, min(v.lcp[r + 1], v.em1[b]));
-            if (mm >= L) {
-                m = mm;
-                skipped |= v.mp1[b] <= X;
-                r -= kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r + 1]);
-        if (m < L) break;
-        const int p = kpos(v, r);
-        if (p <= X) best = max(best, p);
-        --r;
-    }
-    edge = r + 1;
-    return true;
-}
-
-__device__ bool bound_right(const StreamView &v, int j, int X, int L, int &budget, int &edge, int &best,
-                            bool &skipped) {
-    int m = INT_MAX, r = j + 1;
-    while (r < v.n) {
-        if (--budget < 0) return false;
-        if ((r & (kL2 - 1)) == 0 && r + kL2 - 1 < v.n) {
-            const int b = r / kL2;
-            const int mm = min(m, min(v.lcp[r], v.em2[b]));
-            if (mm >= L) {
-                m = mm;
-                skipped |= v.mp2[b] <= X;
-                r += kL2;
-                continue;
-            }
-        }
-        if ((r & (kL1 - 1)) == 0 && r + kL1 - 1 < v.n) {
-            const int b = r / kL1;
-            const int mm = min(m, min(v.lcp[r], v.em1[b]));
-            if (mm >= L) {
-                m = mm;
-                skipped |= v.mp1[b] <= X;
-                r += kL1;
-                continue;
-            }
-        }
-        m = min(m, v.lcp[r]);
-        if (m < L) break;
-        const int p = kpos(v, r);
-        if (p <= X) best = max(best, p);
-        ++r;
-    }
-    edge = r - 1;
-    return true;
-}
-
 __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *vsym, int s, int t, int L, int ib,
                                              int32_t *end_idx, int32_t *len, int32_t *sym) {
     const int64_t o = (int64_t)s * G.T + t;
@@ -966,41 +851,119 @@ __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *v
     }
 }
 
-__global__ void resolve_easy_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
-                                    int32_t *__restrict__ end_idx, int32_t *__restrict__ len,
-                                    int32_t *__restrict__ sym, int32_t *__restrict__ hard, int *hard_count) {
-    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (gi >= G.N) return;
-    const int s = (int)(gi / G.n);
-    const int j = (int)(gi - (int64_t)s * G.n);
-    const uint32_t x = A.sa[gi];
-    if (!G.same && (int)x < G.T) return;          // key item: nothing to answer
-    const int t = G.same ? (int)x : (int)x - G.T;
-    const int X = t - G.g;
-    int L = 0, ib = -1;
-    if (X >= 0) {
-        const StreamView v = make_view(G, s, A);
-        int budget = kEasyBudget, bl = 0, br = 0;
-        bool ok = nearest_left(v, j, X, 0, budget, bl) && nearest_right(v, j, X, bl, budget, br);
-        if (ok) {
-            L = max(bl, br);
-            if (L > 0) {
-                int lo = j, hi = j, best = -1;
-                bool skipped = false;
-                ok = bound_left(v, j, X, L, budget, lo, best, skipped) &&
-                     bound_right(v, j, X, L, budget, hi, best, skipped);
-                if (ok) ib = skipped ? wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, lo), kc(v, hi + 1), X) : best;
-            }
-        }
-        if (!ok) {
-            hard[atomicAdd(hard_count, 1)] = (int32_t)gi;
-            return;
+// One query in the staged window.  kp[i]: key position of local rank i or
+// INT_MAX (query item or outside the stream); lc[i]: LCP edge between local
+// ranks i-1 and i (0 at the stream start, -1 past the stream end).  Returns
+// false when the answer needs ranks outside the window or the budget ran out.
+__device__ bool resolve_in_window(const int *kp, const int *lc, int jl, int X, int &L, int &ib) {
+    int budget = kRBudget;
+    // nearest admissible key below j
+    int mL = 0, rL = -1;
+    {
+        int m = INT_MAX, r = jl - 1;
+        for (;;) {
+            if (r < 0 || --budget < 0) return false;
+            m = min(m, lc[r + 1]);
+            if (m <= 0) break;
+            if (kp[r] <= X) { mL = m; rL = r; break; }
+            --r;
         }
     }
-    write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+    // nearest admissible key above j that beats mL; remember where it stopped
+    int mR = 0, rR = -1, rstop, mstop;
+    {
+        int m = INT_MAX, r = jl + 1;
+        for (;;) {
+            if (r >= kRWin || --budget < 0) return false;
+            m = min(m, lc[r]);
+            if (m <= mL) { rstop = r; mstop = m; break; }
+            if (kp[r] <= X) { mR = m; rR = r; rstop = r; mstop = m; break; }
+            ++r;
+        }
+    }
+    L = max(mL, mR);
+    ib = -1;
+    if (L == 0) return true;
+    int best = -1;
+    if (mR > mL) {
+        // only the upper side reaches L; ranks between j and rR hold no admissible key
+        best = kp[rR];
+        int m = L, r = rR + 1;
+        for (;;) {
+            if (r >= kRWin || --budget < 0) return false;
+            m = min(m, lc[r]);
+            if (m < L) break;
+            if (kp[r] <= X) best = max(best, kp[r]);
+            ++r;
+        }
+    } else {
+        // lower side reaches L at rL; continue below it
+        best = kp[rL];
+        {
+            int m = L, r = rL - 1;
+            for (;;) {
+                if (r < 0 || --budget < 0) return false;
+                m = min(m, lc[r + 1]);
+                if (m < L) break;
+                if (kp[r] <= X) best = max(best, kp[r]);
+                --r;
+            }
+        }
+        // upper side: ranks before rstop hold no admissible key; if the running
+        // LCP at rstop is still L, the interval continues there
+        if (mstop == L) {
+            int m = L, r = rstop;
+            for (;;) {
+                if (r >= kRWin || --budget < 0) return false;
+                m = min(m, lc[r]);
+                if (m < L) break;
+                if (kp[r] <= X) best = max(best, kp[r]);
+                ++r;
+            }
+        }
+    }
+    ib = best;
+    return true;
 }
 
-// ---- warp-cooperative scans -------------------------------------------------
+__global__ void __launch_bounds__(kRThreads)
+resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
+                    int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
+                    int *hard_count) {
+    __shared__ int kp[kRWin];
+    __shared__ int lc[kRWin];
+    const int ntr = ceil_div(G.n, kRTile);
+    const int s = blockIdx.x / ntr, tt = blockIdx.x - s * ntr;
+    const int64_t seg = (int64_t)s * G.n;
+    const int w0 = tt * kRTile - kRHalo;
+    for (int i = threadIdx.x; i < kRWin; i += kRThreads) {
+        const int r = w0 + i;
+        int p = INT_MAX, l = -1;
+        if (r >= 0 && r < G.n) {
+            p = key_pos_or_inf(A.sa[seg + r], G.T, G.same);
+            l = A.lcp[seg + r];
+        }
+        kp[i] = p;
+        lc[i] = l;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kRTile; i += kRThreads) {
+        const int j = tt * kRTile + i;
+        if (j >= G.n) break;
+        const uint32_t x = A.sa[seg + j];
+        if (!G.same && (int)x < G.T) continue;     // key item: nothing to answer
+        const int t = G.same ? (int)x : (int)x - G.T;
+        const int X = t - G.g;
+        int L = 0, ib = -1;
+        if (X >= 0 && !resolve_in_window(kp, lc, j - w0, X, L, ib)) {
+            hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + j);
+            continue;
+        }
+        write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+    }
+}
+
+// ---- warp-cooperative scans over global memory ------------------------------
 
 __device__ __forceinline__ int warp_prefix_min(int x, int lane) {
 #pragma unroll
@@ -1102,6 +1065,8 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
     return result;
 }
 
+// Each warp takes 32 listed queries: the scans run warp-wide one query at a
+// time, then every lane answers its own query's wavelet lookup.
 __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                                     int32_t *__restrict__ end_idx, int32_t *__restrict__ len,
                                     int32_t *__restrict__ sym, const int32_t *__restrict__ hard,
@@ -1110,24 +1075,33 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, const uint8_t *__
     const int lane = threadIdx.x & 31;
     const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t h = wid; h < nh; h += nw) {
-        const int64_t gi = hard[h];
-        const int s = (int)(gi / G.n);
-        const int j = (int)(gi - (int64_t)s * G.n);
-        const uint32_t x = A.sa[gi];
-        const int t = G.same ? (int)x : (int)x - G.T;
-        const int X = t - G.g;
-        const StreamView v = make_view(G, s, A);
-        const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
-        const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
-        const int L = max(bl, br);
-        int ib = -1;
-        if (L > 0) {
-            const int lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
-            const int hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
-            if (lane == 0) ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, lo), kc(v, hi + 1), X);
+    for (int64_t h0 = wid * 32; h0 < nh; h0 += nw * 32) {
+        const int cnt = (nh - h0) < 32 ? (int)(nh - h0) : 32;
+        int my_s = 0, my_t = 0, my_L = 0, my_lo = 0, my_hi = 0, my_X = -1;
+        for (int q = 0; q < cnt; ++q) {
+            const int64_t gi = hard[h0 + q];
+            const int s = (int)(gi / G.n);
+            const int j = (int)(gi - (int64_t)s * G.n);
+            const uint32_t x = A.sa[gi];
+            const int t = G.same ? (int)x : (int)x - G.T;
+            const int X = t - G.g;
+            const StreamView v = make_view(G, s, A);
+            const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
+            const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
+            const int L = max(bl, br);
+            int lo = j, hi = j;
+            if (L > 0) {
+                lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
+                hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
+            }
+            if (lane == q) { my_s = s; my_t = t; my_L = L; my_lo = lo; my_hi = hi; my_X = X; }
         }
-        if (lane == 0) write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+        if (lane < cnt) {
+            const StreamView v = make_view(G, my_s, A);
+            int ib = -1;
+            if (my_L > 0) ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, my_lo), kc(v, my_hi + 1), my_X);
+            write_result(G, vsym, my_s, my_t, my_L, ib, end_idx, len, sym);
+        }
     }
 }
 
@@ -1213,7 +1187,8 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, G.same ? nullptr : W.kcount,
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
-    resolve_easy_kernel<<<grid_for(G.N, 128), 128, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
+    resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, 0, st>>>(G, A, vs, end_idx, len, sym,
+                                                                                      W.hard, hard_count);
     resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
     return cudaGetLastError();
 }
