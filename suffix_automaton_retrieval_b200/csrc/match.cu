@@ -798,7 +798,6 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
 constexpr int kRTile = 1024;
 constexpr int kRHalo = 1024;
 constexpr int kRWin = kRTile + 2 * kRHalo;
-constexpr int kRBudget = 1024;         // shared-memory rank visits per query
 constexpr int kRThreads = 256;
 
 struct StreamView {
@@ -851,102 +850,165 @@ __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *v
     }
 }
 
-// One query in the staged window.  kp[i]: key position of local rank i or
-// INT_MAX (query item or outside the stream); lc[i]: LCP edge between local
-// ranks i-1 and i (0 at the stream start, -1 past the stream end).  Returns
-// false when the answer needs ranks outside the window or the budget ran out.
-__device__ bool resolve_in_window(const int *kp, const int *lc, int jl, int X, int &L, int &ib) {
-    int budget = kRBudget;
+// One query in the staged window (local ranks 0..kRWin-1).
+//   kp[i]  key position of local rank i, INT_MAX for query items and ranks
+//          outside the stream;
+//   lc[i]  LCP edge between local ranks i-1 and i (0 at the stream start,
+//          -1 past the stream end); lc[kRWin] is the edge just past the window;
+//   sp[k][i] min(lc[i .. i+2^k-1]) capped to 255 (u8);
+//   bkp[b] smallest key position among local ranks 32b..32b+31.
+// Returns 0 when answered (L, lo, hi filled; hi < lo when L = 0), 1 when the
+// answer needs ranks outside the window or the visit budget ran out.
+constexpr int kSpLevels = 12;          // 2^11 <= kRWin
+constexpr int kNearBudget = 256;       // shared-memory visits for the nearest-key scans
+
+struct WinSmem {
+    int kp[kRWin];
+    int lc[kRWin + 1];
+    int bkp[kRWin / 32];
+    uint8_t sp[kSpLevels][kRWin];
+};
+
+__device__ __forceinline__ int sp_min(const WinSmem &w, int l, int r) {   // inclusive, l <= r
+    const int k = 31 - __clz(r - l + 1);
+    return min((int)w.sp[k][l], (int)w.sp[k][r - (1 << k) + 1]);
+}
+
+// exact LCP between local ranks a < b: min(lc[a+1..b]) (long runs use the int array)
+__device__ __forceinline__ int lcp_between(const WinSmem &w, int a, int b) {
+    const int c = sp_min(w, a + 1, b);
+    if (c < 255) return c;
+    int m = INT_MAX;
+    for (int i = a + 1; i <= b; ++i) m = min(m, w.lc[i]);
+    return m;
+}
+
+__device__ int resolve_window(const WinSmem &w, bool window_at_start, bool window_at_end, int jl, int X,
+                              int &L, int &lo, int &hi) {
+    int budget = kNearBudget;
     // nearest admissible key below j
-    int mL = 0, rL = -1;
+    int mL = 0;
     {
-        int m = INT_MAX, r = jl - 1;
+        int r = jl - 1;
         for (;;) {
-            if (r < 0 || --budget < 0) return false;
-            m = min(m, lc[r + 1]);
-            if (m <= 0) break;
-            if (kp[r] <= X) { mL = m; rL = r; break; }
+            if (r < 0) {
+                if (!window_at_start) return 1;
+                break;
+            }
+            if (--budget < 0) return 1;
+            if ((r & 31) == 31) {
+                const int b = r >> 5;
+                if (w.bkp[b] > X) {
+                    if (sp_min(w, r - 31, jl) == 0) break;   // no match reaches past this block
+                    r -= 32;
+                    continue;
+                }
+            }
+            if (w.kp[r] <= X) {
+                mL = lcp_between(w, r, jl);
+                break;
+            }
+            if (w.lc[r] == 0) break;                        // nothing further shares a symbol
             --r;
         }
     }
-    // nearest admissible key above j that beats mL; remember where it stopped
-    int mR = 0, rR = -1, rstop, mstop;
+    // nearest admissible key above j; only matters when it beats mL
+    int mR = 0;
     {
-        int m = INT_MAX, r = jl + 1;
+        int r = jl + 1;
         for (;;) {
-            if (r >= kRWin || --budget < 0) return false;
-            m = min(m, lc[r]);
-            if (m <= mL) { rstop = r; mstop = m; break; }
-            if (kp[r] <= X) { mR = m; rR = r; rstop = r; mstop = m; break; }
+            if (r >= kRWin) {
+                if (!window_at_end) return 1;
+                break;
+            }
+            if (--budget < 0) return 1;
+            if (w.lc[r] <= mL) break;                       // running LCP cannot beat mL any more
+            if ((r & 31) == 0 && r + 31 < kRWin) {
+                const int b = r >> 5;
+                if (w.bkp[b] > X) {
+                    if (sp_min(w, jl + 1, r + 31) <= mL) break;
+                    r += 32;
+                    continue;
+                }
+            }
+            if (w.kp[r] <= X) {
+                mR = lcp_between(w, jl, r);
+                break;
+            }
             ++r;
         }
     }
     L = max(mL, mR);
-    ib = -1;
-    if (L == 0) return true;
-    int best = -1;
-    if (mR > mL) {
-        // only the upper side reaches L; ranks between j and rR hold no admissible key
-        best = kp[rR];
-        int m = L, r = rR + 1;
-        for (;;) {
-            if (r >= kRWin || --budget < 0) return false;
-            m = min(m, lc[r]);
-            if (m < L) break;
-            if (kp[r] <= X) best = max(best, kp[r]);
-            ++r;
+    lo = jl;
+    hi = jl - 1;
+    if (L == 0) return 0;
+    if (L < 255) {
+        int cur = jl;
+        for (int k = kSpLevels - 1; k >= 0; --k) {
+            const int c = cur - (1 << k);
+            if (c >= 0 && w.sp[k][c + 1] >= L) cur = c;
         }
+        // cur is the lowest rank with min(lc[cur+1..jl]) >= L inside the window
+        if (cur == 0 && !window_at_start && w.lc[0] >= L) return 1;
+        lo = cur;
+        cur = jl;
+        for (int k = kSpLevels - 1; k >= 0; --k) {
+            const int c = cur + (1 << k);
+            if (c < kRWin && w.sp[k][cur + 1] >= L) cur = c;
+        }
+        if (cur == kRWin - 1 && w.lc[kRWin] >= L) return 1;
+        hi = cur;
     } else {
-        // lower side reaches L at rL; continue below it
-        best = kp[rL];
-        {
-            int m = L, r = rL - 1;
-            for (;;) {
-                if (r < 0 || --budget < 0) return false;
-                m = min(m, lc[r + 1]);
-                if (m < L) break;
-                if (kp[r] <= X) best = max(best, kp[r]);
-                --r;
-            }
-        }
-        // upper side: ranks before rstop hold no admissible key; if the running
-        // LCP at rstop is still L, the interval continues there
-        if (mstop == L) {
-            int m = L, r = rstop;
-            for (;;) {
-                if (r >= kRWin || --budget < 0) return false;
-                m = min(m, lc[r]);
-                if (m < L) break;
-                if (kp[r] <= X) best = max(best, kp[r]);
-                ++r;
-            }
-        }
+        int r = jl;
+        while (r > 0 && w.lc[r] >= L) --r;
+        if (r == 0 && !window_at_start && w.lc[0] >= L) return 1;
+        lo = r;
+        r = jl;
+        while (r + 1 < kRWin && w.lc[r + 1] >= L) ++r;
+        if (r == kRWin - 1 && w.lc[kRWin] >= L) return 1;
+        hi = r;
     }
-    ib = best;
-    return true;
+    return 0;
 }
 
 __global__ void __launch_bounds__(kRThreads)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
                     int *hard_count) {
-    __shared__ int kp[kRWin];
-    __shared__ int lc[kRWin];
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    WinSmem &w = *reinterpret_cast<WinSmem *>(smem_raw);
     const int ntr = ceil_div(G.n, kRTile);
     const int s = blockIdx.x / ntr, tt = blockIdx.x - s * ntr;
     const int64_t seg = (int64_t)s * G.n;
     const int w0 = tt * kRTile - kRHalo;
-    for (int i = threadIdx.x; i < kRWin; i += kRThreads) {
+    for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
         const int r = w0 + i;
         int p = INT_MAX, l = -1;
         if (r >= 0 && r < G.n) {
-            p = key_pos_or_inf(A.sa[seg + r], G.T, G.same);
+            if (i < kRWin) p = key_pos_or_inf(A.sa[seg + r], G.T, G.same);
             l = A.lcp[seg + r];
         }
-        kp[i] = p;
-        lc[i] = l;
+        if (i < kRWin) {
+            w.kp[i] = p;
+            w.sp[0][i] = (uint8_t)(l < 0 ? 0 : (l > 255 ? 255 : l));
+        }
+        w.lc[i] = l;
     }
     __syncthreads();
+    for (int k = 1; k < kSpLevels; ++k) {
+        const int h = 1 << (k - 1);
+        for (int i = threadIdx.x; i < kRWin; i += kRThreads)
+            w.sp[k][i] = (i + 2 * h - 1 < kRWin) ? min(w.sp[k - 1][i], w.sp[k - 1][i + h]) : 0;
+        __syncthreads();
+    }
+    for (int b = threadIdx.x; b < kRWin / 32; b += kRThreads) {
+        int m = INT_MAX;
+        for (int i = 0; i < 32; ++i) m = min(m, w.kp[b * 32 + i]);
+        w.bkp[b] = m;
+    }
+    __syncthreads();
+    const bool at_start = w0 <= 0, at_end = w0 + kRWin >= G.n;
+    const StreamView v = make_view(G, s, A);
     for (int i = threadIdx.x; i < kRTile; i += kRThreads) {
         const int j = tt * kRTile + i;
         if (j >= G.n) break;
@@ -955,9 +1017,20 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         const int t = G.same ? (int)x : (int)x - G.T;
         const int X = t - G.g;
         int L = 0, ib = -1;
-        if (X >= 0 && !resolve_in_window(kp, lc, j - w0, X, L, ib)) {
-            hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + j);
-            continue;
+        if (X >= 0) {
+            int lo, hi;
+            if (resolve_window(w, at_start, at_end, j - w0, X, L, lo, hi)) {
+                hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + j);
+                continue;
+            }
+            if (L > 0) {
+                if (hi - lo < 64) {
+                    for (int r = lo; r <= hi; ++r)
+                        if (w.kp[r] <= X) ib = max(ib, w.kp[r]);
+                } else {
+                    ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, w0 + lo), kc(v, w0 + hi + 1), X);
+                }
+            }
         }
         write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
     }
@@ -1184,11 +1257,14 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
         wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, G.wbits, lv, W.wvals[lv & 1],
                                                                        W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
     // 3c. resolve: thread per query, then warp per query for the long scans
+    if ((err = cudaFuncSetAttribute(resolve_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)sizeof(WinSmem))) != cudaSuccess)
+        return err;
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, G.same ? nullptr : W.kcount,
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
-    resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, 0, st>>>(G, A, vs, end_idx, len, sym,
-                                                                                      W.hard, hard_count);
+    resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
+        G, A, vs, end_idx, len, sym, W.hard, hard_count);
     resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
     return cudaGetLastError();
 }
