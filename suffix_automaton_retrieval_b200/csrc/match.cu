@@ -99,6 +99,7 @@ struct Workspace {
     int2 *lists[2][2];       // [buffer][0 = small, 1 = large]
     int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2;
     int32_t *hard;           // ranks of queries left for the warp-cooperative phase
+    int32_t *wq;             // output slots of queries waiting for a wavelet lookup
     int32_t *kcount;         // keys before each rank (q != k)
     int *ktile;              // keys per 2048-rank tile
     uint32_t *wvals[2];      // wavelet level sequences
@@ -140,6 +141,7 @@ Workspace carve(const Geometry &G, void *base) {
     W.minpos2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.emin2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.hard = (int32_t *)take(N * 4);
+    W.wq = (int32_t *)take((size_t)G.S * G.T * 4);
     W.kcount = (int32_t *)take(N * 4);
     W.ktile = (int *)take((size_t)G.S * G.ntps * 4);
     W.wvals[0] = (uint32_t *)take((size_t)G.S * G.T * 4);
@@ -466,9 +468,11 @@ __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *_
 //    so keys[] (sorted in round 0) still holds the key of the item at each
 //    rank.
 // ---------------------------------------------------------------------------
+constexpr int kLcpSerial = 24;         // symbols past D0 one thread compares before handing off
+
 __global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
                            const uint64_t *__restrict__ keys, const uint32_t *__restrict__ sa,
-                           int32_t *__restrict__ lcp) {
+                           int32_t *__restrict__ lcp, int32_t *__restrict__ long_list, int *long_count) {
     const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (gi >= G.N) return;
     const int s = (int)(gi / G.n);
@@ -491,8 +495,41 @@ __global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restr
     const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
     int m = G.D0;
     const int lim = min(p1, p2) + 1;
-    while (m < lim && s1[p1 - m] == s2[p2 - m]) ++m;
+    const int stop = min(lim, G.D0 + kLcpSerial);
+    while (m < stop && s1[p1 - m] == s2[p2 - m]) ++m;
     lcp[gi] = m;
+    if (m == stop && m < lim) long_list[atomicAdd(long_count, 1)] = (int32_t)gi;   // still equal: a warp finishes it
+}
+
+// Long common prefixes (repeats): one warp per pair, 32 symbols per step.
+__global__ void lcp_long_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
+                                const uint32_t *__restrict__ sa, int32_t *__restrict__ lcp,
+                                const int32_t *__restrict__ long_list, const int *__restrict__ long_count) {
+    const int nl = *long_count;
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t e = wid; e < nl; e += nw) {
+        const int64_t gi = long_list[e];
+        const int s = (int)(gi / G.n);
+        const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
+        const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
+        const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
+        const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
+        const int lim = min(p1, p2) + 1;
+        int m = lcp[gi];
+        for (;;) {
+            const int i = m + lane;
+            const bool diff = i >= lim || s1[p1 - i] != s2[p2 - i];
+            const unsigned dm = __ballot_sync(ROSA_FULL_MASK, diff);
+            if (dm) {
+                m += __ffs(dm) - 1;
+                break;
+            }
+            m += 32;
+        }
+        if (lane == 0) lcp[gi] = m;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -603,8 +640,12 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
         else for (int i = 0; i < tt; ++i) p += ktile[(int64_t)s * G.ntps + i];
         pre_s = p;
     }
+    // this tile's keys take consecutive key indices, so they touch at most two wavelet tiles
+    __shared__ int ones[2];
+    if (threadIdx.x < 2) ones[threadIdx.x] = 0;
     __syncthreads();
     int run = pre_s;
+    const int t0 = run / kWTile;
     for (int u = 0; u < kRadixIPT; ++u) {
         const int i = u * 256 + threadIdx.x;
         const bool ok = i < lim;
@@ -622,11 +663,12 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
         if (ok && !G.same) kcount[base + i] = kidx;
         if (key) {
             a0[(int64_t)s * G.T + kidx] = x;
-            if ((x >> (nbits - 1)) & 1u) atomicAdd(&wcnt0[(int64_t)s * ntw + kidx / kWTile], 1);
+            if ((x >> (nbits - 1)) & 1u) atomicAdd(&ones[kidx / kWTile - t0], 1);
         }
         run += rtot;
         __syncthreads();
     }
+    if (threadIdx.x < 2 && ones[threadIdx.x]) atomicAdd(&wcnt0[(int64_t)s * ntw + t0 + threadIdx.x], ones[threadIdx.x]);
 }
 
 __global__ void __launch_bounds__(256)
@@ -971,10 +1013,22 @@ __device__ int resolve_window(const WinSmem &w, bool window_at_start, bool windo
     return 0;
 }
 
+// Parks a query whose interval is too wide to scan: its key range goes into
+// the output slots until wavelet_query_kernel replaces it with the answer.
+__device__ __forceinline__ void defer_wavelet(const Geometry &G, int s, int t, int L, int klo, int khi,
+                                              int32_t *end_idx, int32_t *len, int32_t *sym, int32_t *wq,
+                                              int *wq_count) {
+    const int64_t o = (int64_t)s * G.T + t;
+    len[o] = L;
+    end_idx[o] = klo;
+    sym[o] = khi;
+    wq[atomicAdd(wq_count, 1)] = (int32_t)o;
+}
+
 __global__ void __launch_bounds__(kRThreads)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
-                    int *hard_count) {
+                    int *hard_count, int32_t *__restrict__ wq, int *wq_count) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     WinSmem &w = *reinterpret_cast<WinSmem *>(smem_raw);
     const int ntr = ceil_div(G.n, kRTile);
@@ -1028,7 +1082,8 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                     for (int r = lo; r <= hi; ++r)
                         if (w.kp[r] <= X) ib = max(ib, w.kp[r]);
                 } else {
-                    ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, w0 + lo), kc(v, w0 + hi + 1), X);
+                    defer_wavelet(G, s, t, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), end_idx, len, sym, wq, wq_count);
+                    continue;
                 }
             }
         }
@@ -1138,43 +1193,55 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
     return result;
 }
 
-// Each warp takes 32 listed queries: the scans run warp-wide one query at a
-// time, then every lane answers its own query's wavelet lookup.
-__global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
-                                    int32_t *__restrict__ end_idx, int32_t *__restrict__ len,
-                                    int32_t *__restrict__ sym, const int32_t *__restrict__ hard,
-                                    const int *__restrict__ hard_count) {
+// One warp per listed query: scans for L and the interval bounds; the most
+// recent admissible end is left to wavelet_query_kernel.
+__global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
+                                    int32_t *__restrict__ len, int32_t *__restrict__ sym,
+                                    const int32_t *__restrict__ hard, const int *__restrict__ hard_count,
+                                    int32_t *__restrict__ wq, int *wq_count) {
     const int nh = *hard_count;
     const int lane = threadIdx.x & 31;
     const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t h0 = wid * 32; h0 < nh; h0 += nw * 32) {
-        const int cnt = (nh - h0) < 32 ? (int)(nh - h0) : 32;
-        int my_s = 0, my_t = 0, my_L = 0, my_lo = 0, my_hi = 0, my_X = -1;
-        for (int q = 0; q < cnt; ++q) {
-            const int64_t gi = hard[h0 + q];
-            const int s = (int)(gi / G.n);
-            const int j = (int)(gi - (int64_t)s * G.n);
-            const uint32_t x = A.sa[gi];
-            const int t = G.same ? (int)x : (int)x - G.T;
-            const int X = t - G.g;
-            const StreamView v = make_view(G, s, A);
-            const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
-            const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
-            const int L = max(bl, br);
-            int lo = j, hi = j;
-            if (L > 0) {
-                lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
-                hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
-            }
-            if (lane == q) { my_s = s; my_t = t; my_L = L; my_lo = lo; my_hi = hi; my_X = X; }
+    for (int64_t h = wid; h < nh; h += nw) {
+        const int64_t gi = hard[h];
+        const int s = (int)(gi / G.n);
+        const int j = (int)(gi - (int64_t)s * G.n);
+        const uint32_t x = A.sa[gi];
+        const int t = G.same ? (int)x : (int)x - G.T;
+        const int X = t - G.g;
+        const StreamView v = make_view(G, s, A);
+        const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
+        const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
+        const int L = max(bl, br);
+        if (L > 0) {
+            const int lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
+            const int hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
+            if (lane == 0) defer_wavelet(G, s, t, L, kc(v, lo), kc(v, hi + 1), end_idx, len, sym, wq, wq_count);
+        } else if (lane == 0) {
+            const int64_t o = (int64_t)s * G.T + t;
+            end_idx[o] = -1;
+            len[o] = 0;
+            sym[o] = -1;
         }
-        if (lane < cnt) {
-            const StreamView v = make_view(G, my_s, A);
-            int ib = -1;
-            if (my_L > 0) ib = wavelet_max_le(v.W, v.Z, v.nbits, v.nw, kc(v, my_lo), kc(v, my_hi + 1), my_X);
-            write_result(G, vsym, my_s, my_t, my_L, ib, end_idx, len, sym);
-        }
+    }
+}
+
+// Largest admissible key position inside each parked query's key range.
+__global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
+                                     int32_t *__restrict__ end_idx, int32_t *__restrict__ sym,
+                                     const int32_t *__restrict__ wq, const int *__restrict__ wq_count) {
+    const int nq = *wq_count;
+    const int nw = (G.T >> 6) + 1;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t o = wq[i];
+        const int s = (int)(o / G.T);
+        const int t = (int)(o - (int64_t)s * G.T);
+        const int klo = end_idx[o], khi = sym[o];
+        const WWord *W = A.words + (int64_t)s * A.nbits * nw;
+        const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nbits, A.nbits, nw, klo, khi, t - G.g);
+        end_idx[o] = ib;
+        sym[o] = ib >= 0 ? (int32_t)vsym[(int64_t)s * G.T + ib + 1] : -1;
     }
 }
 
@@ -1188,9 +1255,9 @@ int match_launch_count(int S, int T, int K, bool same) {
     int rounds = 0;
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits, kRadixBits);
-    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + lcp + summary
-    // + wavelet (key count when q != k, compaction, one per level) + 2 resolve
-    return 1 + 3 * passes + 1 + 4 * rounds + 2 + (same ? 0 : 1) + 1 + G.wbits + 2;
+    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + 2 lcp + summary
+    // + wavelet (key count when q != k, compaction, one per level) + 3 resolve
+    return 1 + 3 * passes + 1 + 4 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 3;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1243,7 +1310,8 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
         lb ^= 1;
     }
     // 2. LCP
-    lcp_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, keys, sa, W.lcp);
+    lcp_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, keys, sa, W.lcp, W.hard, W.counts + 6);
+    lcp_long_kernel<<<kNumSMs * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
     // 3a. summaries
     summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
                                                            W.minpos2, W.emin2);
@@ -1263,9 +1331,11 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, G.same ? nullptr : W.kcount,
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
+    int *wq_count = W.counts + 5;
     resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
-        G, A, vs, end_idx, len, sym, W.hard, hard_count);
-    resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, len, sym, W.hard, hard_count);
+        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
+    resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
+    wavelet_query_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
     return cudaGetLastError();
 }
 
