@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--streams", type=int, default=0,
+                    help="profiling aid: keep only the first N streams of a symbol workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-streams", type=int, default=0,
@@ -97,6 +99,24 @@ def build_workload(cfg: int, device, seed_offset: int = 0):
         wl["V"] = W.value_rows(sw.B, sw.T, sw.R * c["rho"], seed=c["seed_v"] + 1000 * seed_offset, device=device)
         wl["ops"].append("gather")
     return wl
+
+
+def shrink_streams(wl, S):
+    """Keep the first S streams (whole batches when the workload has value rows)."""
+    if "V" in wl:
+        B = max(1, S // wl["R"])
+        S = B * wl["R"]
+        wl["V"] = wl["V"][:B].contiguous()
+        wl["B"] = B
+    else:
+        wl["R"] = S
+        wl["B"] = 1
+    wl["S"] = S
+    wl["q_host"] = wl["q_host"][:S]
+    wl["k_host"] = wl["q_host"] if wl["same"] else wl["k_host"][:S]
+    wl["q"] = wl["q"][:S].contiguous()
+    wl["k"] = wl["q"] if wl["same"] else wl["k"][:S].contiguous()
+    wl["name"] += f"[{S} streams]"
 
 
 def algorithmic_bytes(wl):
@@ -277,6 +297,8 @@ def main():
         dist.barrier()
 
     wl = build_workload(args.config, device, seed_offset=rank)
+    if args.streams and wl["cfg"] != 3 and args.streams < wl["S"]:
+        shrink_streams(wl, args.streams)
     runner = Runner(wl, device)
     ab = algorithmic_bytes(wl)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)

@@ -902,12 +902,15 @@ __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *v
 // Returns 0 when answered (L, lo, hi filled; hi < lo when L = 0), 1 when the
 // answer needs ranks outside the window or the visit budget ran out.
 constexpr int kSpLevels = 12;          // 2^11 <= kRWin
-constexpr int kNearBudget = 256;       // shared-memory visits for the nearest-key scans
+constexpr int kNearBudget = 48;        // shared-memory visits for the nearest-key scans
 
 struct WinSmem {
     int kp[kRWin];
     int lc[kRWin + 1];
     int bkp[kRWin / 32];
+    int qj[kRTile];          // local rank of each query of the tile
+    int qt[kRTile];          // its time index t
+    int nq;
     uint8_t sp[kSpLevels][kRWin];
 };
 
@@ -1060,15 +1063,37 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         for (int i = 0; i < 32; ++i) m = min(m, w.kp[b * 32 + i]);
         w.bkp[b] = m;
     }
+    // compact the tile's query items so that every lane has one to answer
+    if (threadIdx.x == 0) w.nq = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int i0 = 0; i0 < kRTile; i0 += kRThreads) {
+        const int i = i0 + threadIdx.x;
+        const int j = tt * kRTile + i;
+        uint32_t x = 0;
+        bool isq = false;
+        if (j < G.n) {
+            x = A.sa[seg + j];
+            isq = G.same || (int)x >= G.T;
+        }
+        const unsigned bal = __ballot_sync(ROSA_FULL_MASK, isq);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&w.nq, __popc(bal));
+        base = __shfl_sync(ROSA_FULL_MASK, base, 0);
+        if (isq) {
+            const int slot = base + __popc(bal & lanemask_lt());
+            w.qj[slot] = i + kRHalo;
+            w.qt[slot] = G.same ? (int)x : (int)x - G.T;
+        }
+    }
     __syncthreads();
     const bool at_start = w0 <= 0, at_end = w0 + kRWin >= G.n;
     const StreamView v = make_view(G, s, A);
-    for (int i = threadIdx.x; i < kRTile; i += kRThreads) {
-        const int j = tt * kRTile + i;
-        if (j >= G.n) break;
-        const uint32_t x = A.sa[seg + j];
-        if (!G.same && (int)x < G.T) continue;     // key item: nothing to answer
-        const int t = G.same ? (int)x : (int)x - G.T;
+    const int nq = w.nq;
+    for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
+        const int jl = w.qj[qi];
+        const int j = w0 + jl;
+        const int t = w.qt[qi];
         const int X = t - G.g;
         int L = 0, ib = -1;
         if (X >= 0) {
