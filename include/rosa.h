@@ -121,6 +121,31 @@ ROSA_API int rosa_match_launch_count(int S, int T, int K, int q_is_k);
 ROSA_API int rosa_match_device_status(const void *workspace, cudaStream_t stream, uint32_t *status);
 
 /*
+ * rosa_match without a workspace argument: the same retrieval, with its
+ * scratch memory taken from a fixed device array inside this library
+ * (ROSA_NOALLOC_SCRATCH_BYTES, 64 MiB, reserved on every GPU that loads the
+ * library until the process exits).  There is no counterpart on the pages;
+ * it exists for callers that cannot allocate device memory where they run
+ * the retrieval (hosts that own all device allocations, serving loops that
+ * must not call cudaMalloc/cudaFree because those can synchronise the
+ * device).  Inputs and outputs are the caller's, as for rosa_match.
+ *
+ * Sizes whose workspace (rosa_match_workspace_size) exceeds the array are
+ * rejected with ROSA_ERR_WORKSPACE before anything touches the GPU; the
+ * array holds about 500 000 positions (S*T), e.g. 16 streams of 16384 with
+ * q != k over 256 symbols.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents: calls that overlap on the GPU (different streams or
+ * threads) race and must be serialised by the caller.
+ */
+#define ROSA_NOALLOC_SCRATCH_BYTES (64u << 20)
+ROSA_API int rosa_match_noalloc(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                                int S, int T, int K, int g,
+                                int32_t *end_idx, int32_t *len, int32_t *sym, cudaStream_t stream);
+
+/*
  * Read-out of value rows at tau (appendix C.4 with the Eq. 17 mask).
  *
  *   V        [B, T, *] bf16 rows, row stride v_row_stride elements.
