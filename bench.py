@@ -234,6 +234,20 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- peaks
 
+def reduce_over_ranks(local_ms: float, local_units: float, device=None):
+    """Whole-job timing across ranks: the slowest rank's time and the units
+    all ranks processed.  A no-op without an initialised process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return local_ms, local_units
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -336,14 +350,9 @@ def main():
     for _, _, ev in per_step:
         for o in wl["ops"]:
             op_ms[o].append(ev[o + "0"].elapsed_time(ev[o + "1"]))
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-
     positions = wl["S"] * wl["T"]
-    value = positions * args.steps * world / (total_ms / 1e3)
+    total_ms, units = reduce_over_ranks(sum(step_ms), positions * args.steps, device)
+    value = units / (total_ms / 1e3)
     ms_per_step = total_ms / args.steps
 
     # roofline of the dominant op (the one with the largest share of the step)
@@ -359,12 +368,10 @@ def main():
     e2e = None
     if not args.no_e2e:
         e2e = end_to_end(wl, device, args.steps)
-    if world > 1:
         # every rank takes the same collective steps
-        ev_t = torch.tensor([e2e["value"] if e2e else 0.0], dtype=torch.float64, device=device)
-        dist.all_reduce(ev_t, op=dist.ReduceOp.MIN)
-        if e2e:
-            e2e["value"] = float(ev_t.item()) * world
+        e_ms, e_units = reduce_over_ranks(e2e["ms_per_step"] * args.steps, positions * args.steps, device)
+        e2e["value"] = e_units / (e_ms / 1e3)
+        e2e["ms_per_step"] = e_ms / args.steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

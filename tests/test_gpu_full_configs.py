@@ -1,0 +1,130 @@
+"""Parity at the full sizes of the five workloads, in the launch
+configuration the benchmark times (one rosa_match over all streams, one
+workspace, preallocated outputs).  The CPU oracle checks whole sampled
+streams bit for bit (its online suffix automaton is linear in T); the
+independent invariant checker covers sampled positions; gathered rows are
+compared bitwise for sampled routes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.invariants import check_stream
+from suffix_automaton_retrieval_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def rosa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from suffix_automaton_retrieval_b200 import build
+    build.build()
+    import suffix_automaton_retrieval_b200.binding as b
+    return b
+
+
+def _bits(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _run_match(rosa, q, k, K, g, same):
+    S, T = q.shape
+    ws = rosa.alloc_workspace(S, T, K, DEV)
+    outs = tuple(torch.empty((S, T), dtype=torch.int32, device=DEV) for _ in range(3))
+    rosa.match(q, None if same else k, K=K, g=g, out=outs, workspace=ws)
+    torch.cuda.synchronize()
+    assert rosa.match_device_status(ws) == 0
+    return [o.cpu().numpy() for o in outs]
+
+
+def _check_streams(got, qh, kh, g, streams, tag, sample_pos=40):
+    want = oracle.match_sam(qh[streams], kh[streams], g=g)
+    for name, a, b in zip(("end_idx", "len", "sym"), got, want):
+        sub = a[streams]
+        if not np.array_equal(sub, b):
+            bad = np.argwhere(sub != b)
+            s, t = bad[0]
+            raise AssertionError(f"{tag}: {name} differs at {len(bad)} places; first stream {streams[s]} t={t}: "
+                                 f"gpu={sub[s, t]} oracle={b[s, t]}")
+    s0 = streams[0]
+    check_stream(qh[s0], kh[s0], kh[s0], g, got[0][s0], got[1][s0], got[2][s0], full=False, sample=sample_pos)
+
+
+def _symbol_case(rosa, w, n_streams):
+    q = torch.from_numpy(w.q).to(DEV)
+    k = q if w.same_qk else torch.from_numpy(w.k).to(DEV)
+    got = _run_match(rosa, q, k, w.K, w.g, w.same_qk)
+    rng = np.random.default_rng(0)
+    streams = np.sort(rng.choice(w.S, size=min(n_streams, w.S), replace=False))
+    _check_streams(got, w.q, w.k, w.g, streams, w.name)
+    return got, streams
+
+
+def test_full_binary_4k(rosa):
+    w = workloads.binary_iid()
+    q = torch.from_numpy(w.q).to(DEV)
+    got = _run_match(rosa, q, q, w.K, w.g, True)
+    want = oracle.match_brute(w.q, w.q, g=w.g)      # the definition, exhaustively
+    for a, b in zip(got, want):
+        assert np.array_equal(a, b)
+    w64 = workloads.binary_iid(T=64)
+    q = torch.from_numpy(w64.q).to(DEV)
+    got = _run_match(rosa, q, q, w64.K, w64.g, True)
+    for a, b in zip(got, oracle.match_brute(w64.q, w64.q, g=w64.g)):
+        assert np.array_equal(a, b)
+
+
+def test_full_planted_16(rosa):
+    _symbol_case(rosa, workloads.planted_copies(), 8)
+
+
+def test_full_zipf_256_131k(rosa):
+    got, _ = _symbol_case(rosa, workloads.zipf_planted(), 4)
+    assert got[1].max() >= 16          # the planted repeats are found
+
+
+def test_full_markov_4_train_with_gather(rosa):
+    c = workloads.CONFIGS[5]
+    w = workloads.markov()
+    got, streams = _symbol_case(rosa, w, 12)
+    V = workloads.value_rows(w.B, w.T, w.R * c["rho"], seed=c["seed_v"], device=DEV)
+    end = torch.from_numpy(got[0]).to(DEV)
+    out = rosa.gather(V, end, w.R, c["d"], c["rho"])
+    torch.cuda.synchronize()
+    d, rho = c["d"], c["rho"]
+    want_end = oracle.match_sam(w.q[streams], w.k[streams], g=w.g)[0]
+    for i, s in enumerate(streams[:4]):
+        b, r = divmod(int(s), w.R)
+        vslice = _bits(V[b:b + 1, :, r * rho:r * rho + d].contiguous())
+        want = oracle.gather(vslice, want_end[i:i + 1], 1, d, d)
+        assert np.array_equal(_bits(out[b:b + 1, :, r * d:(r + 1) * d].contiguous()), want), (b, r)
+
+
+def test_full_qwen_proj_64_path(rosa):
+    c = workloads.CONFIGS[3]
+    T, width, ch, M, d, rho = c["T"], c["width"], c["channels"], c["M"], c["d"], c["rho"]
+    H, Wq, Wk = workloads.qwen_projection_inputs(T=T, width=width, channels=ch, device=DEV)
+    qv, kv = (H @ Wq).contiguous(), (H @ Wk).contiguous()
+    del H
+    R = ch // M
+    V = workloads.value_rows(1, T, R * rho, seed=c["seed_v"], device=DEV)
+    sq, sk = rosa.discretize(qv, M), rosa.discretize(kv, M)
+    got = _run_match(rosa, sq.view(R, T), sk.view(R, T), 2 ** M, 2, False)
+    end = torch.from_numpy(got[0]).to(DEV)
+    out = rosa.gather(V, end, R, d, rho)
+    torch.cuda.synchronize()
+    oq, ok = oracle.discretize(_bits(qv), M), oracle.discretize(_bits(kv), M)
+    assert np.array_equal(sq.cpu().numpy(), oq) and np.array_equal(sk.cpu().numpy(), ok)
+    qh, kh = oq.reshape(R, T), ok.reshape(R, T)
+    streams = np.array([0, 17, 40, 63])
+    _check_streams(got, qh, kh, 2, streams, "qwen-proj-64")
+    want_end = oracle.match_sam(qh[streams], kh[streams], g=2)[0]
+    for i, r in enumerate(streams[:2]):
+        vslice = _bits(V[:, :, r * rho:r * rho + d].contiguous())
+        want = oracle.gather(vslice, want_end[i:i + 1], 1, d, d)
+        assert np.array_equal(_bits(out[:, :, r * d:(r + 1) * d].contiguous()), want), r
