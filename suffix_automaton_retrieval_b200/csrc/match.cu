@@ -41,7 +41,6 @@ constexpr int kRadixIPT = 8;
 constexpr int kRadixTile = kRadixThreads * kRadixIPT;   // 2048 items per tile
 constexpr int kRadixBits = 8;
 constexpr int kRadixBins = 1 << kRadixBits;
-constexpr int kScanThreads = 1024;
 constexpr int kSmallGroup = 32;        // groups up to this size are sorted by one warp
 constexpr int kSmemSortCap = 4096;     // larger groups up to this size sort in shared memory
 constexpr int kLargeThreads = 512;
@@ -183,8 +182,11 @@ __global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__res
 
 // ---------------------------------------------------------------------------
 // 1b. Segmented LSD radix sort, 8-bit digits, tiles of 2048 items that never
-//     straddle a stream.  hist layout: [stream][digit][tile-in-stream].
+//     straddle a stream.  hist layout: [stream][tile-in-stream][digit].
 // ---------------------------------------------------------------------------
+constexpr int kRadixWarps = kRadixThreads / 32;
+constexpr int kWarpItems = kRadixTile / kRadixWarps;   // 256 contiguous items per warp
+
 __global__ void __launch_bounds__(kRadixThreads)
 radix_hist_kernel(const uint64_t *__restrict__ keys, Geometry G, int shift, uint32_t *__restrict__ hist) {
     __shared__ uint32_t cnt[kRadixBins];
@@ -197,39 +199,38 @@ radix_hist_kernel(const uint64_t *__restrict__ keys, Geometry G, int shift, uint
     for (int i = threadIdx.x; i < lim; i += kRadixThreads)
         atomicAdd(&cnt[(keys[base + i] >> shift) & (kRadixBins - 1)], 1u);
     __syncthreads();
-    hist[((int64_t)s * kRadixBins + threadIdx.x) * G.ntps + tt] = cnt[threadIdx.x];
+    hist[((int64_t)s * G.ntps + tt) * kRadixBins + threadIdx.x] = cnt[threadIdx.x];
 }
 
-// Exclusive scan of one stream's [digit][tile] counts, in place.
-__global__ void __launch_bounds__(kScanThreads)
+// Per stream: turn the [tile][digit] counts into each tile's first output
+// slot per digit (digit-major order, tiles in order within a digit).
+__global__ void __launch_bounds__(kRadixBins)
 radix_scan_kernel(uint32_t *__restrict__ hist, int ntps) {
-    __shared__ uint32_t ws[kScanThreads / 32 + 1];
-    uint32_t *h = hist + (int64_t)blockIdx.x * kRadixBins * ntps;
-    const int M = kRadixBins * ntps;
-    const int per = ceil_div(M, kScanThreads);
-    const int lo = min(M, threadIdx.x * per), hi = min(M, lo + per);
-    uint32_t sum = 0;
-    for (int i = lo; i < hi; ++i) sum += h[i];
-    uint32_t run = block_exclusive_scan<kScanThreads>(sum, ws, nullptr);
-    for (int i = lo; i < hi; ++i) {
-        const uint32_t c = h[i];
-        h[i] = run;
+    __shared__ uint32_t ws[kRadixBins / 32 + 1];
+    uint32_t *h = hist + (int64_t)blockIdx.x * ntps * kRadixBins + threadIdx.x;
+    uint32_t total = 0;
+    for (int t = 0; t < ntps; ++t) total += h[(int64_t)t * kRadixBins];
+    uint32_t run = block_exclusive_scan<kRadixBins>(total, ws, nullptr);
+    for (int t = 0; t < ntps; ++t) {
+        const uint32_t c = h[(int64_t)t * kRadixBins];
+        h[(int64_t)t * kRadixBins] = run;
         run += c;
     }
 }
 
-// Stable scatter of one tile: items keep their tile order within a digit.
+// Stable scatter of one tile.  Warp w owns items [256w, 256w+256) of the
+// tile; ranks come from warp-private digit counters, so the whole tile needs
+// only three block barriers.
 __global__ void __launch_bounds__(kRadixThreads)
 radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restrict__ vin,
                      uint64_t *__restrict__ kout, uint32_t *__restrict__ vout, Geometry G, int shift,
                      const uint32_t *__restrict__ hist) {
     __shared__ uint64_t sk[kRadixTile];
     __shared__ uint32_t sv[kRadixTile];
-    __shared__ uint16_t wcnt[kRadixThreads / 32][kRadixBins];
-    __shared__ uint32_t running[kRadixBins];
+    __shared__ uint32_t wcnt[kRadixWarps][kRadixBins];   // per-warp digit counts, then per-warp offsets
     __shared__ uint32_t tstart[kRadixBins];
     __shared__ uint32_t gofs[kRadixBins];
-    __shared__ uint32_t wsum[kRadixThreads / 32 + 1];
+    __shared__ uint32_t wsum[kRadixWarps + 1];
 
     const int tile = blockIdx.x;
     const int s = tile / G.ntps, tt = tile - s * G.ntps;
@@ -238,53 +239,58 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
     const int lim = min(kRadixTile, G.n - tt * kRadixTile);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    gofs[threadIdx.x] = hist[((int64_t)s * kRadixBins + threadIdx.x) * G.ntps + tt];
-    running[threadIdx.x] = 0;
-    for (int w = 0; w < kRadixThreads / 32; ++w) wcnt[w][threadIdx.x] = 0;
+    gofs[threadIdx.x] = hist[((int64_t)s * G.ntps + tt) * kRadixBins + threadIdx.x];
+#pragma unroll
+    for (int w = 0; w < kRadixWarps; ++w) wcnt[w][threadIdx.x] = 0;
     __syncthreads();
 
     uint64_t key[kRadixIPT];
     uint32_t val[kRadixIPT];
-    uint32_t rnk[kRadixIPT];
     int dig[kRadixIPT];
+    const int wbase = warp * kWarpItems;
+    // pass 1: warp-private digit counts (a digit's leader lane owns its counter)
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
-        const int i = u * kRadixThreads + threadIdx.x;
+        const int i = wbase + u * 32 + lane;
         const bool ok = i < lim;
         key[u] = ok ? kin[base + i] : 0ull;
         val[u] = ok ? vin[base + i] : 0u;
         dig[u] = ok ? (int)((key[u] >> shift) & (kRadixBins - 1)) : kRadixBins;
         const unsigned peers = __match_any_sync(ROSA_FULL_MASK, dig[u]);
-        const unsigned wr = __popc(peers & lanemask_lt());
-        if (ok && wr == 0) wcnt[warp][dig[u]] = (uint16_t)__popc(peers);
-        __syncthreads();
-        if (ok) {
-            uint32_t pre = running[dig[u]];
-            for (int w = 0; w < warp; ++w) pre += wcnt[w][dig[u]];
-            rnk[u] = pre + wr;
-        }
-        __syncthreads();
-        {
-            uint32_t add = 0;
-            for (int w = 0; w < kRadixThreads / 32; ++w) {
-                add += wcnt[w][threadIdx.x];
-                wcnt[w][threadIdx.x] = 0;
-            }
-            running[threadIdx.x] += add;
-        }
-        __syncthreads();
+        if (ok && (peers & lanemask_lt()) == 0) wcnt[warp][dig[u]] += __popc(peers);
+        __syncwarp();
     }
-    (void)lane;
-    const uint32_t st = block_exclusive_scan<kRadixThreads>(running[threadIdx.x], wsum, nullptr);
-    tstart[threadIdx.x] = st;
     __syncthreads();
+    // digit totals -> tile start per digit; per-warp offsets within the digit
+    {
+        const int d = threadIdx.x;
+        uint32_t tot = 0;
+#pragma unroll
+        for (int w = 0; w < kRadixWarps; ++w) tot += wcnt[w][d];
+        const uint32_t st = block_exclusive_scan<kRadixThreads>(tot, wsum, nullptr);
+        tstart[d] = st;
+        uint32_t run = st;
+#pragma unroll
+        for (int w = 0; w < kRadixWarps; ++w) {
+            const uint32_t c = wcnt[w][d];
+            wcnt[w][d] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    // pass 2: place each item at its stable slot in shared memory
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
+        const unsigned peers = __match_any_sync(ROSA_FULL_MASK, dig[u]);
+        const unsigned before = __popc(peers & lanemask_lt());
         if (dig[u] < kRadixBins) {
-            const uint32_t pos = tstart[dig[u]] + rnk[u];
+            const uint32_t pos = wcnt[warp][dig[u]] + before;
             sk[pos] = key[u];
             sv[pos] = val[u];
         }
+        __syncwarp();
+        if (dig[u] < kRadixBins && before == 0) wcnt[warp][dig[u]] += __popc(peers);
+        __syncwarp();
     }
     __syncthreads();
     for (int j = threadIdx.x; j < lim; j += kRadixThreads) {
@@ -892,129 +898,39 @@ __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *v
     }
 }
 
-// One query in the staged window (local ranks 0..kRWin-1).
+__device__ __forceinline__ int warp_prefix_min(int x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(ROSA_FULL_MASK, x, o);
+        if (lane >= o) x = min(x, y);
+    }
+    return x;
+}
+
+// Staged window of one resolve tile (local ranks 0..kRWin-1):
 //   kp[i]  key position of local rank i, INT_MAX for query items and ranks
 //          outside the stream;
 //   lc[i]  LCP edge between local ranks i-1 and i (0 at the stream start,
 //          -1 past the stream end); lc[kRWin] is the edge just past the window;
 //   sp[k][i] min(lc[i .. i+2^k-1]) capped to 255 (u8);
-//   bkp[b] smallest key position among local ranks 32b..32b+31.
-// Returns 0 when answered (L, lo, hi filled; hi < lo when L = 0), 1 when the
-// answer needs ranks outside the window or the visit budget ran out.
+//   per query of the tile: local rank qj, time index qt, match length qL.
+// Queries are resolved in three uniform phases (see resolve_tile_kernel).
 constexpr int kSpLevels = 12;          // 2^11 <= kRWin
-constexpr int kNearBudget = 48;        // shared-memory visits for the nearest-key scans
+constexpr int kProbe = 16;             // ranks a lane probes on each side before its warp helps
+constexpr int kWarpSteps = 24;         // 32-rank steps of a warp-cooperative scan (768 ranks)
+constexpr int kNeedWarp = -1;          // qL codes
+constexpr int kNeedHard = -2;
 
 struct WinSmem {
     int kp[kRWin];
     int lc[kRWin + 1];
-    int bkp[kRWin / 32];
-    int qj[kRTile];          // local rank of each query of the tile
-    int qt[kRTile];          // its time index t
-    int nq;
+    int qt[kRTile];
+    int qL[kRTile];
+    int16_t qj[kRTile];
+    int16_t bq[kRTile];
+    int nq, nb;
     uint8_t sp[kSpLevels][kRWin];
 };
-
-__device__ __forceinline__ int sp_min(const WinSmem &w, int l, int r) {   // inclusive, l <= r
-    const int k = 31 - __clz(r - l + 1);
-    return min((int)w.sp[k][l], (int)w.sp[k][r - (1 << k) + 1]);
-}
-
-// exact LCP between local ranks a < b: min(lc[a+1..b]) (long runs use the int array)
-__device__ __forceinline__ int lcp_between(const WinSmem &w, int a, int b) {
-    const int c = sp_min(w, a + 1, b);
-    if (c < 255) return c;
-    int m = INT_MAX;
-    for (int i = a + 1; i <= b; ++i) m = min(m, w.lc[i]);
-    return m;
-}
-
-__device__ int resolve_window(const WinSmem &w, bool window_at_start, bool window_at_end, int jl, int X,
-                              int &L, int &lo, int &hi) {
-    int budget = kNearBudget;
-    // nearest admissible key below j
-    int mL = 0;
-    {
-        int r = jl - 1;
-        for (;;) {
-            if (r < 0) {
-                if (!window_at_start) return 1;
-                break;
-            }
-            if (--budget < 0) return 1;
-            if ((r & 31) == 31) {
-                const int b = r >> 5;
-                if (w.bkp[b] > X) {
-                    if (sp_min(w, r - 31, jl) == 0) break;   // no match reaches past this block
-                    r -= 32;
-                    continue;
-                }
-            }
-            if (w.kp[r] <= X) {
-                mL = lcp_between(w, r, jl);
-                break;
-            }
-            if (w.lc[r] == 0) break;                        // nothing further shares a symbol
-            --r;
-        }
-    }
-    // nearest admissible key above j; only matters when it beats mL
-    int mR = 0;
-    {
-        int r = jl + 1;
-        for (;;) {
-            if (r >= kRWin) {
-                if (!window_at_end) return 1;
-                break;
-            }
-            if (--budget < 0) return 1;
-            if (w.lc[r] <= mL) break;                       // running LCP cannot beat mL any more
-            if ((r & 31) == 0 && r + 31 < kRWin) {
-                const int b = r >> 5;
-                if (w.bkp[b] > X) {
-                    if (sp_min(w, jl + 1, r + 31) <= mL) break;
-                    r += 32;
-                    continue;
-                }
-            }
-            if (w.kp[r] <= X) {
-                mR = lcp_between(w, jl, r);
-                break;
-            }
-            ++r;
-        }
-    }
-    L = max(mL, mR);
-    lo = jl;
-    hi = jl - 1;
-    if (L == 0) return 0;
-    if (L < 255) {
-        int cur = jl;
-        for (int k = kSpLevels - 1; k >= 0; --k) {
-            const int c = cur - (1 << k);
-            if (c >= 0 && w.sp[k][c + 1] >= L) cur = c;
-        }
-        // cur is the lowest rank with min(lc[cur+1..jl]) >= L inside the window
-        if (cur == 0 && !window_at_start && w.lc[0] >= L) return 1;
-        lo = cur;
-        cur = jl;
-        for (int k = kSpLevels - 1; k >= 0; --k) {
-            const int c = cur + (1 << k);
-            if (c < kRWin && w.sp[k][cur + 1] >= L) cur = c;
-        }
-        if (cur == kRWin - 1 && w.lc[kRWin] >= L) return 1;
-        hi = cur;
-    } else {
-        int r = jl;
-        while (r > 0 && w.lc[r] >= L) --r;
-        if (r == 0 && !window_at_start && w.lc[0] >= L) return 1;
-        lo = r;
-        r = jl;
-        while (r + 1 < kRWin && w.lc[r + 1] >= L) ++r;
-        if (r == kRWin - 1 && w.lc[kRWin] >= L) return 1;
-        hi = r;
-    }
-    return 0;
-}
 
 // Parks a query whose interval is too wide to scan: its key range goes into
 // the output slots until wavelet_query_kernel replaces it with the answer.
@@ -1028,6 +944,76 @@ __device__ __forceinline__ void defer_wavelet(const Geometry &G, int s, int t, i
     wq[atomicAdd(wq_count, 1)] = (int32_t)o;
 }
 
+// Warp-cooperative nearest admissible key in direction dir, 32 ranks per
+// step: the LCP with it when that exceeds lim, 0 when the running LCP falls
+// to lim first, kNeedHard when the answer lies beyond the window or the steps.
+__device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int lim, int lane) {
+    int carry = INT_MAX;
+    for (int step = 0; step < kWarpSteps; ++step) {
+        const int r = jl + dir * (1 + step * 32 + lane);
+        int e;
+        bool valid;
+        if (dir < 0) {
+            e = r >= -1 ? w.lc[r + 1] : kNeedHard;
+            valid = r >= 0 && w.kp[r] <= X;
+        } else {
+            e = r <= kRWin ? w.lc[r] : kNeedHard;
+            valid = r < kRWin && w.kp[r] <= X;
+        }
+        const int pm = min(carry, warp_prefix_min(e, lane));
+        const unsigned sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
+        const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid && pm > lim);
+        const int fs = sm ? __ffs(sm) - 1 : 32;
+        const int fv = vm ? __ffs(vm) - 1 : 32;
+        if (fv < fs) return __shfl_sync(ROSA_FULL_MASK, pm, fv);
+        if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
+        carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
+    }
+    return kNeedHard;
+}
+
+// Interval of local ranks around jl whose LCP with jl is >= L.  Returns false
+// when it may extend beyond the window.
+__device__ bool window_bounds(const WinSmem &w, bool at_start, int jl, int L, int &lo, int &hi) {
+    if (L < 255) {
+        int cur = jl;
+#pragma unroll
+        for (int k = kSpLevels - 1; k >= 0; --k) {
+            const int c = cur - (1 << k);
+            if (c >= 0 && w.sp[k][c + 1] >= L) cur = c;
+        }
+        if (cur == 0 && !at_start && w.lc[0] >= L) return false;
+        lo = cur;
+        cur = jl;
+#pragma unroll
+        for (int k = kSpLevels - 1; k >= 0; --k) {
+            const int c = cur + (1 << k);
+            if (c < kRWin && w.sp[k][cur + 1] >= L) cur = c;
+        }
+        if (cur == kRWin - 1 && w.lc[kRWin] >= L) return false;
+        hi = cur;
+    } else {   // long matches: exact edges (such intervals are short)
+        int r = jl;
+        while (r > 0 && w.lc[r] >= L) --r;
+        if (r == 0 && !at_start && w.lc[0] >= L) return false;
+        lo = r;
+        r = jl;
+        while (r + 1 < kRWin && w.lc[r + 1] >= L) ++r;
+        if (r == kRWin - 1 && w.lc[kRWin] >= L) return false;
+        hi = r;
+    }
+    return true;
+}
+
+// One CTA per 1024 ranks of a stream, with 1024 ranks of context on each side.
+//   Phase A: each lane probes 16 ranks on each side of its query for the
+//            nearest admissible key (fixed trip count, no divergence).
+//   Phase B: queries the probes could not settle get a warp each, scanning
+//            32 ranks per step in shared memory.
+//   Phase C: each lane finds its interval bounds by binary lifting on the
+//            sparse table, then i* by a 16-rank probe or, for wider
+//            intervals, a deferred wavelet lookup.
+// Queries whose answer needs ranks outside the window go to the hard list.
 __global__ void __launch_bounds__(kRThreads)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
@@ -1038,6 +1024,8 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const int s = blockIdx.x / ntr, tt = blockIdx.x - s * ntr;
     const int64_t seg = (int64_t)s * G.n;
     const int w0 = tt * kRTile - kRHalo;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; }
     for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
         const int r = w0 + i;
         int p = INT_MAX, l = -1;
@@ -1058,15 +1046,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
             w.sp[k][i] = (i + 2 * h - 1 < kRWin) ? min(w.sp[k - 1][i], w.sp[k - 1][i + h]) : 0;
         __syncthreads();
     }
-    for (int b = threadIdx.x; b < kRWin / 32; b += kRThreads) {
-        int m = INT_MAX;
-        for (int i = 0; i < 32; ++i) m = min(m, w.kp[b * 32 + i]);
-        w.bkp[b] = m;
-    }
     // compact the tile's query items so that every lane has one to answer
-    if (threadIdx.x == 0) w.nq = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
     for (int i0 = 0; i0 < kRTile; i0 += kRThreads) {
         const int i = i0 + threadIdx.x;
         const int j = tt * kRTile + i;
@@ -1082,34 +1062,87 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         base = __shfl_sync(ROSA_FULL_MASK, base, 0);
         if (isq) {
             const int slot = base + __popc(bal & lanemask_lt());
-            w.qj[slot] = i + kRHalo;
+            w.qj[slot] = (int16_t)(i + kRHalo);
             w.qt[slot] = G.same ? (int)x : (int)x - G.T;
         }
     }
     __syncthreads();
-    const bool at_start = w0 <= 0, at_end = w0 + kRWin >= G.n;
-    const StreamView v = make_view(G, s, A);
     const int nq = w.nq;
+    // Phase A
     for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
         const int jl = w.qj[qi];
-        const int j = w0 + jl;
+        const int X = w.qt[qi] - G.g;
+        int L = 0;
+        if (X >= 0) {
+            int m = INT_MAX, Ll = -1;
+#pragma unroll
+            for (int k = 1; k <= kProbe; ++k) {
+                const int r = jl - k;                  // jl >= kRHalo, so r >= 0
+                m = min(m, w.lc[r + 1]);
+                const int c = w.kp[r];
+                if (Ll < 0) Ll = (m <= 0) ? 0 : (c <= X ? m : -1);
+            }
+            int Lr = -1;
+            if (Ll >= 0) {
+                m = INT_MAX;
+#pragma unroll
+                for (int k = 1; k <= kProbe; ++k) {
+                    const int r = jl + k;              // jl + kProbe < kRWin
+                    m = min(m, w.lc[r]);
+                    const int c = w.kp[r];
+                    if (Lr < 0) Lr = (m <= Ll) ? 0 : (c <= X ? m : -1);
+                }
+            }
+            if (Ll < 0 || Lr < 0) {
+                L = kNeedWarp;
+                w.bq[atomicAdd(&w.nb, 1)] = (int16_t)qi;
+            } else {
+                L = max(Ll, Lr);
+            }
+        }
+        w.qL[qi] = L;
+    }
+    __syncthreads();
+    // Phase B
+    const int nb = w.nb;
+    for (int bi = warp; bi < nb; bi += kRThreads / 32) {
+        const int qi = w.bq[bi];
+        const int jl = w.qj[qi];
+        const int X = w.qt[qi] - G.g;
+        const int Ll = warp_nearest_smem(w, jl, X, -1, 0, lane);
+        int L = Ll;
+        if (Ll != kNeedHard) {
+            const int Lr = warp_nearest_smem(w, jl, X, +1, Ll, lane);
+            L = Lr == kNeedHard ? kNeedHard : max(Ll, Lr);
+        }
+        if (lane == 0) w.qL[qi] = L;
+    }
+    __syncthreads();
+    // Phase C
+    const bool at_start = w0 <= 0;
+    const StreamView v = make_view(G, s, A);
+    for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
+        const int jl = w.qj[qi];
         const int t = w.qt[qi];
         const int X = t - G.g;
-        int L = 0, ib = -1;
-        if (X >= 0) {
-            int lo, hi;
-            if (resolve_window(w, at_start, at_end, j - w0, X, L, lo, hi)) {
-                hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + j);
-                continue;
-            }
-            if (L > 0) {
-                if (hi - lo < 64) {
-                    for (int r = lo; r <= hi; ++r)
-                        if (w.kp[r] <= X) ib = max(ib, w.kp[r]);
-                } else {
-                    defer_wavelet(G, s, t, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), end_idx, len, sym, wq, wq_count);
-                    continue;
+        const int L = w.qL[qi];
+        int lo = 0, hi = -1;
+        if (L == kNeedHard || (L > 0 && !window_bounds(w, at_start, jl, L, lo, hi))) {
+            hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + w0 + jl);
+            continue;
+        }
+        int ib = -1;
+        if (L > 0) {
+            if (hi - lo < kProbe) {
+#pragma unroll
+                for (int k = 0; k < kProbe; ++k) {
+                    const int r = lo + k;              // lo <= jl < kRWin - kProbe
+                    const int c = r <= hi ? w.kp[r] : INT_MAX;
+                    if (c <= X) ib = max(ib, c);
                 }
+            } else {
+                defer_wavelet(G, s, t, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), end_idx, len, sym, wq, wq_count);
+                continue;
             }
         }
         write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
@@ -1118,14 +1151,6 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
 
 // ---- warp-cooperative scans over global memory ------------------------------
 
-__device__ __forceinline__ int warp_prefix_min(int x, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(ROSA_FULL_MASK, x, o);
-        if (lane >= o) x = min(x, y);
-    }
-    return x;
-}
 
 // NEAREST: LCP with the first admissible key in direction dir if > lim, else 0.
 // BOUND: the last rank in direction dir whose running LCP stays >= lim.
@@ -1309,7 +1334,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     const unsigned tiles = (unsigned)(G.S * G.ntps);
     for (int shift = 0; shift < G.keybits; shift += kRadixBits) {
         radix_hist_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], G, shift, W.hist);
-        radix_scan_kernel<<<(unsigned)G.S, kScanThreads, 0, st>>>(W.hist, G.ntps);
+        radix_scan_kernel<<<(unsigned)G.S, kRadixBins, 0, st>>>(W.hist, G.ntps);
         radix_scatter_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], W.vals[cur], W.keys[cur ^ 1],
                                                               W.vals[cur ^ 1], G, shift, W.hist);
         cur ^= 1;
