@@ -337,47 +337,47 @@ __global__ void groups0_kernel(const uint64_t *__restrict__ keys, const uint32_t
 // ---------------------------------------------------------------------------
 // 1d. Prefix doubling at depth h: sort each unresolved group by the rank of
 //     the same-kind prefix h symbols further back, then split into new groups.
+//     Groups of up to 32 members (nearly all of them) take one thread each;
+//     larger ones a warp (keys, regroup) and a CTA (sort).  Within a round all
+//     keys are read before any rank changes (separate launches).
 // ---------------------------------------------------------------------------
-__global__ void dbl_keys_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
-                                const int *__restrict__ counts, Geometry G, int64_t h,
-                                const uint32_t *__restrict__ sa, const int32_t *__restrict__ rank,
-                                uint32_t *__restrict__ k2) {
+__device__ __forceinline__ uint64_t pair_key(uint32_t k2, uint32_t x) { return ((uint64_t)k2 << 32) | x; }
+
+// Small groups: one thread computes its members' keys and insertion-sorts
+// them in place.  Large groups: one warp computes the keys.
+__global__ void dbl_keys_sort_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
+                                     const int *__restrict__ counts, Geometry G, int64_t h, uint32_t *__restrict__ sa,
+                                     const int32_t *__restrict__ rank, uint32_t *__restrict__ k2) {
     const int ns = counts[0], nl = counts[1];
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t nth = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t gidx = tid; gidx < ns; gidx += nth) {
+        const int2 gr = small[gidx];
+        const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
+        uint32_t *gs = sa + gr.x;
+        uint32_t *gk = k2 + gr.x;
+        for (int m = 0; m < gr.y; ++m) {
+            const uint32_t x = gs[m];
+            const uint32_t kk = (uint32_t)rank[seg + x - h];
+            const uint64_t key = pair_key(kk, x);
+            int i = m - 1;
+            while (i >= 0 && pair_key(gk[i], gs[i]) > key) {
+                gk[i + 1] = gk[i];
+                gs[i + 1] = gs[i];
+                --i;
+            }
+            gk[i + 1] = kk;
+            gs[i + 1] = x;
+        }
+    }
     const int lane = threadIdx.x & 31;
-    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t gidx = wid; gidx < ns + nl; gidx += nw) {
-        const int2 gr = gidx < ns ? small[gidx] : large[gidx - ns];
+    for (int64_t gidx = tid >> 5; gidx < nl; gidx += nth >> 5) {
+        const int2 gr = large[gidx];
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
         for (int m = lane; m < gr.y; m += 32) {
             const uint32_t x = sa[gr.x + m];
             k2[gr.x + m] = (uint32_t)rank[seg + x - h];
         }
-    }
-}
-
-// One warp per group of at most 32: rank by counting on (k2, item id).
-__global__ void dbl_sort_small_kernel(const int2 *__restrict__ small, const int *__restrict__ counts,
-                                      uint32_t *__restrict__ sa, uint32_t *__restrict__ k2) {
-    const int ns = counts[0];
-    const int lane = threadIdx.x & 31;
-    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t gidx = wid; gidx < ns; gidx += nw) {
-        const int2 gr = small[gidx];
-        const bool ok = lane < gr.y;
-        const uint64_t key = ok ? (((uint64_t)k2[gr.x + lane] << 32) | sa[gr.x + lane]) : ~0ull;
-        int r = 0;
-        for (int o = 0; o < 32; ++o) {
-            const uint64_t other = __shfl_sync(ROSA_FULL_MASK, key, o);
-            r += (other < key) ? 1 : 0;
-        }
-        __syncwarp();
-        if (ok) {
-            sa[gr.x + r] = (uint32_t)key;
-            k2[gr.x + r] = (uint32_t)(key >> 32);
-        }
-        __syncwarp();
     }
 }
 
@@ -414,8 +414,7 @@ dbl_sort_large_kernel(const int2 *__restrict__ large, const int *__restrict__ co
     for (int gidx = blockIdx.x; gidx < nl; gidx += gridDim.x) {
         const int2 gr = large[gidx];
         uint64_t *a = gr.y <= kSmemSortCap ? buf : scratch + gr.x;
-        for (int m = threadIdx.x; m < gr.y; m += blockDim.x)
-            a[m] = ((uint64_t)k2[gr.x + m] << 32) | sa[gr.x + m];
+        for (int m = threadIdx.x; m < gr.y; m += blockDim.x) a[m] = pair_key(k2[gr.x + m], sa[gr.x + m]);
         __syncthreads();
         bitonic_sort(a, gr.y);
         for (int m = threadIdx.x; m < gr.y; m += blockDim.x) {
@@ -434,11 +433,26 @@ __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *_
                                    const uint32_t *__restrict__ sa, const uint32_t *__restrict__ k2,
                                    int32_t *__restrict__ rank, int2 *nsmall, int2 *nlarge, int *counts_next) {
     const int ns = counts[0], nl = counts[1];
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t nth = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t gidx = tid; gidx < ns; gidx += nth) {
+        const int2 gr = small[gidx];
+        const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
+        const int jstart = (int)(gr.x - seg);
+        int head = 0;
+        for (int m = 0; m < gr.y; ++m) {
+            const uint32_t kk = k2[gr.x + m];
+            if (m > 0 && kk != k2[gr.x + m - 1]) head = m;
+            const uint32_t x = sa[gr.x + m];
+            rank[seg + x] = jstart + head;
+            const bool last = (m == gr.y - 1) || (k2[gr.x + m + 1] != kk);
+            if (last && m > head && (int64_t)item_pos(x, G.T) + 1 > h2)
+                push_group(nsmall, nlarge, counts_next, gr.x + head, m - head + 1);
+        }
+    }
     const int lane = threadIdx.x & 31;
-    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t gidx = wid; gidx < ns + nl; gidx += nw) {
-        const int2 gr = gidx < ns ? small[gidx] : large[gidx - ns];
+    for (int64_t gidx = tid >> 5; gidx < nl; gidx += nth >> 5) {
+        const int2 gr = large[gidx];
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
         const int jstart = (int)(gr.x - seg);
         int carry = jstart;
@@ -1305,9 +1319,9 @@ int match_launch_count(int S, int T, int K, bool same) {
     int rounds = 0;
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits, kRadixBits);
-    // keys0 + 3 per radix pass + groups0 + 4 per doubling round + 2 lcp + summary
+    // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
     // + wavelet (key count when q != k, compaction, one per level) + 3 resolve
-    return 1 + 3 * passes + 1 + 4 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 3;
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 3;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1351,8 +1365,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     for (int64_t h = G.D0; h < T; h *= 2) {
         int *cnt = W.counts + 2 * lb;
         int *cnt_next = W.counts + 2 * (lb ^ 1);
-        dbl_keys_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, h, sa, W.rank, W.k2);
-        dbl_sort_small_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], cnt, sa, W.k2);
+        dbl_keys_sort_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, h, sa, W.rank, W.k2);
         dbl_sort_large_kernel<<<kNumSMs * 2, kLargeThreads, 0, st>>>(W.lists[lb][1], cnt, sa, W.k2, scratch);
         if ((err = cudaMemsetAsync(cnt_next, 0, 2 * sizeof(int), st)) != cudaSuccess) return err;
         dbl_regroup_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, 2 * h, sa, W.k2, W.rank,
