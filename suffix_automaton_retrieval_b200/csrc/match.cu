@@ -694,9 +694,12 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
 __global__ void __launch_bounds__(256)
 wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__ in, uint32_t *__restrict__ out,
                      int *__restrict__ wcnt, WWord *__restrict__ words, int *__restrict__ wz) {
+    // warp w owns elements [256w, 256w + 256) of the tile: its ones count
+    // gives the warp's offsets, so the tile needs only two block barriers
     __shared__ uint32_t ballots[kWTile / 32];
     __shared__ int wones[8];
     __shared__ int red_a[8], red_t[8];
+    __shared__ int nxt[4];
     const int ntw = ceil_div(G.T, kWTile), nw = (G.T >> 6) + 1;
     const int s = blockIdx.x / ntw, tt = blockIdx.x - s * ntw;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -713,55 +716,56 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         a += __shfl_xor_sync(ROSA_FULL_MASK, a, o);
         tot += __shfl_xor_sync(ROSA_FULL_MASK, tot, o);
     }
-    if (lane == 0) { red_a[warp] = a; red_t[warp] = tot; }
-    __syncthreads();
-    int ones_before = 0, total_ones = 0;
-    for (int w = 0; w < 8; ++w) { ones_before += red_a[w]; total_ones += red_t[w]; }
-    const int Z = G.T - total_ones;
-    const int zeros_before = tt * kWTile - ones_before;
     const int lim = min(kWTile, G.T - tt * kWTile);
     const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
-    uint32_t *dst = out + (int64_t)s * G.T;
-    int *cnt_next = wcnt + ((int64_t)(lv + 1) * G.S + s) * ntw;
-    // zeros of this tile land in one contiguous range and ones in another, so
-    // the next level's per-tile counts touch at most four tiles: count them here
-    __shared__ int nxt[4];
-    const int zr0 = zeros_before / kWTile, or0 = (Z + ones_before) / kWTile;
+    uint32_t v[8];
+    unsigned bal[8];
+    int mine = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int i = warp * 256 + u * 32 + lane;
+        const bool ok = i < lim;
+        v[u] = ok ? src[i] : 0u;
+        bal[u] = __ballot_sync(ROSA_FULL_MASK, ok && ((v[u] >> b) & 1u));
+        mine += __popc(bal[u]);
+    }
+    if (lane == 0) {
+        red_a[warp] = a;
+        red_t[warp] = tot;
+        wones[warp] = mine;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ballots[warp * 8 + u] = bal[u];
+    }
     if (threadIdx.x < 4) nxt[threadIdx.x] = 0;
     __syncthreads();
-    int run = 0;
-    for (int u = 0; u < kWTile / 256; ++u) {
-        const int i = u * 256 + threadIdx.x;
-        const bool ok = i < lim;
-        const uint32_t v = ok ? src[i] : 0u;
-        const int bit = ok ? (int)((v >> b) & 1u) : 0;
-        const unsigned bal = __ballot_sync(ROSA_FULL_MASK, bit);
-        if (lane == 0) {
-            ballots[u * 8 + warp] = bal;
-            wones[warp] = __popc(bal);
-        }
-        __syncthreads();
-        int wpre = 0, rtot = 0;
-        for (int w = 0; w < 8; ++w) {
-            if (w < warp) wpre += wones[w];
-            rtot += wones[w];
-        }
-        const int lo1 = run + wpre + __popc(bal & lanemask_lt());
-        if (ok) {
+    int ones_before = 0, total_ones = 0, wpre = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) {
+        ones_before += red_a[w2];
+        total_ones += red_t[w2];
+        if (w2 < warp) wpre += wones[w2];
+    }
+    const int Z = G.T - total_ones;
+    const int zeros_before = tt * kWTile - ones_before;
+    // zeros of this tile land in one contiguous range and ones in another, so
+    // the next level's per-tile counts touch at most four tiles
+    const int zr0 = zeros_before / kWTile, or0 = (Z + ones_before) / kWTile;
+    uint32_t *dst = out + (int64_t)s * G.T;
+    int run = wpre;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int i = warp * 256 + u * 32 + lane;
+        const int bit = (bal[u] >> lane) & 1;
+        const int lo1 = run + __popc(bal[u] & lanemask_lt());
+        if (i < lim) {
             const int d = bit ? Z + ones_before + lo1 : zeros_before + (i - lo1);
-            dst[d] = v;
-            if (lv + 1 < nbits && ((v >> (b - 1)) & 1u)) {
+            dst[d] = v[u];
+            if (lv + 1 < nbits && ((v[u] >> (b - 1)) & 1u)) {
                 const int dt = d / kWTile;
                 atomicAdd(&nxt[bit ? 2 + (dt - or0) : (dt - zr0)], 1);
             }
         }
-        run += rtot;
-        __syncthreads();
-    }
-    if (lv + 1 < nbits && threadIdx.x < 4) {
-        const int c = nxt[threadIdx.x];
-        const int dt = threadIdx.x < 2 ? zr0 + threadIdx.x : or0 + threadIdx.x - 2;
-        if (c) atomicAdd(&cnt_next[dt], c);
+        run += __popc(bal[u]);
     }
     if (threadIdx.x < 32) {
         const int k = threadIdx.x;
@@ -775,20 +779,26 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
             if (lane >= o) incl += y;
         }
         if (k * 64 < lim) {
-            WWord w;
-            w.cum = (uint32_t)(ones_before + incl - pc);
-            w.pad = 0;
-            w.bits = bits;
-            words[((int64_t)s * nbits + lv) * nw + tt * 32 + k] = w;
+            WWord wd;
+            wd.cum = (uint32_t)(ones_before + incl - pc);
+            wd.pad = 0;
+            wd.bits = bits;
+            words[((int64_t)s * nbits + lv) * nw + tt * 32 + k] = wd;
         }
+    }
+    __syncthreads();
+    if (lv + 1 < nbits && threadIdx.x < 4) {
+        const int c = nxt[threadIdx.x];
+        const int dt = threadIdx.x < 2 ? zr0 + threadIdx.x : or0 + threadIdx.x - 2;
+        if (c) atomicAdd(&wcnt[((int64_t)(lv + 1) * G.S + s) * ntw + dt], c);
     }
     if (threadIdx.x == 0) {
         if (tt == ntw - 1 && (G.T & 63) == 0) {
-            WWord w;
-            w.cum = (uint32_t)total_ones;
-            w.pad = 0;
-            w.bits = 0ull;
-            words[((int64_t)s * nbits + lv) * nw + (G.T >> 6)] = w;
+            WWord wd;
+            wd.cum = (uint32_t)total_ones;
+            wd.pad = 0;
+            wd.bits = 0ull;
+            words[((int64_t)s * nbits + lv) * nw + (G.T >> 6)] = wd;
         }
         if (tt == 0) wz[(int64_t)s * nbits + lv] = Z;
     }
@@ -929,11 +939,13 @@ __device__ __forceinline__ int warp_prefix_min(int x, int lane) {
 //   sp[k][i] min(lc[i .. i+2^k-1]) capped to 255 (u8);
 //   per query of the tile: local rank qj, time index qt, match length qL.
 // Queries are resolved in three uniform phases (see resolve_tile_kernel).
-constexpr int kSpLevels = 12;          // 2^11 <= kRWin
+constexpr int kSpLevels = 11;          // lifting reaches 2^11 - 1 ranks: a whole side of the window
 constexpr int kProbe = 16;             // ranks a lane probes on each side before its warp helps
 constexpr int kWarpSteps = 24;         // 32-rank steps of a warp-cooperative scan (768 ranks)
 constexpr int kNeedWarp = -1;          // qL codes
 constexpr int kNeedHard = -2;
+
+constexpr int kWarpScanMax = 256;      // widest interval a warp scans in shared memory
 
 struct WinSmem {
     int kp[kRWin];
@@ -942,7 +954,9 @@ struct WinSmem {
     int qL[kRTile];
     int16_t qj[kRTile];
     int16_t bq[kRTile];
-    int nq, nb;
+    int16_t dlo[kRTile];     // phase D: interval bounds of queries a warp finishes
+    int16_t dhi[kRTile];     // (their query indices reuse bq)
+    int nq, nb, nd;
     uint8_t sp[kSpLevels][kRWin];
 };
 
@@ -1039,7 +1053,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const int64_t seg = (int64_t)s * G.n;
     const int w0 = tt * kRTile - kRHalo;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; }
+    if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; w.nd = 0; }
     for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
         const int r = w0 + i;
         int p = INT_MAX, l = -1;
@@ -1154,12 +1168,35 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                     const int c = r <= hi ? w.kp[r] : INT_MAX;
                     if (c <= X) ib = max(ib, c);
                 }
+            } else if (hi - lo < kWarpScanMax) {
+                const int d = atomicAdd(&w.nd, 1);
+                w.bq[d] = (int16_t)qi;
+                w.dlo[d] = (int16_t)lo;
+                w.dhi[d] = (int16_t)hi;
+                w.qL[qi] = L;
+                continue;
             } else {
                 defer_wavelet(G, s, t, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), end_idx, len, sym, wq, wq_count);
                 continue;
             }
         }
         write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+    }
+    __syncthreads();
+    // Phase D: mid-size intervals, one warp each, 32 ranks per step
+    const int nd = w.nd;
+    for (int di = warp; di < nd; di += kRThreads / 32) {
+        const int qi = w.bq[di];
+        const int lo = w.dlo[di], hi = w.dhi[di];
+        const int X = w.qt[qi] - G.g;
+        int best = -1;
+        for (int r = lo + lane; r <= hi; r += 32) {
+            const int c = w.kp[r];
+            if (c <= X) best = max(best, c);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
+        if (lane == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
     }
 }
 
