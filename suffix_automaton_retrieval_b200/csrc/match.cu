@@ -96,7 +96,7 @@ struct Workspace {
     uint32_t *k2;
     uint32_t *hist;
     int2 *lists[2][2];       // [buffer][0 = small, 1 = large]
-    int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2;
+    int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2, *ein2;
     int32_t *hard;           // ranks of queries left for the warp-cooperative phase
     int32_t *wq;             // output slots of queries waiting for a wavelet lookup
     int32_t *kcount;         // keys before each rank (q != k)
@@ -139,6 +139,7 @@ Workspace carve(const Geometry &G, void *base) {
     W.ein1 = (int32_t *)take((size_t)G.S * G.nb1 * 4);
     W.minpos2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.emin2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
+    W.ein2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.hard = (int32_t *)take(N * 4);
     W.wq = (int32_t *)take((size_t)G.S * G.T * 4);
     W.kcount = (int32_t *)take(N * 4);
@@ -221,7 +222,7 @@ radix_scan_kernel(uint32_t *__restrict__ hist, int ntps) {
 // Stable scatter of one tile.  Warp w owns items [256w, 256w+256) of the
 // tile; ranks come from warp-private digit counters, so the whole tile needs
 // only three block barriers.
-__global__ void __launch_bounds__(kRadixThreads)
+__global__ void __launch_bounds__(kRadixThreads, 4)
 radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restrict__ vin,
                      uint64_t *__restrict__ kout, uint32_t *__restrict__ vout, Geometry G, int shift,
                      const uint32_t *__restrict__ hist) {
@@ -246,18 +247,26 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
 
     uint64_t key[kRadixIPT];
     uint32_t val[kRadixIPT];
-    int dig[kRadixIPT];
+    unsigned peer[kRadixIPT];
     const int wbase = warp * kWarpItems;
-    // pass 1: warp-private digit counts (a digit's leader lane owns its counter)
+    const unsigned lt = lanemask_lt();
+    // pass 1: lanes holding the same digit (8 ballots, one per digit bit);
+    // each digit's lowest lane adds the group size to the warp's counter
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
         const int i = wbase + u * 32 + lane;
         const bool ok = i < lim;
         key[u] = ok ? kin[base + i] : 0ull;
         val[u] = ok ? vin[base + i] : 0u;
-        dig[u] = ok ? (int)((key[u] >> shift) & (kRadixBins - 1)) : kRadixBins;
-        const unsigned peers = __match_any_sync(ROSA_FULL_MASK, dig[u]);
-        if (ok && (peers & lanemask_lt()) == 0) wcnt[warp][dig[u]] += __popc(peers);
+        const unsigned d = (unsigned)(key[u] >> shift) & (kRadixBins - 1);
+        unsigned pm = __ballot_sync(ROSA_FULL_MASK, ok);
+#pragma unroll
+        for (int bit = 0; bit < kRadixBits; ++bit) {
+            const unsigned bm = __ballot_sync(ROSA_FULL_MASK, (d >> bit) & 1u);
+            pm &= ((d >> bit) & 1u) ? bm : ~bm;
+        }
+        peer[u] = pm;
+        if (ok && (pm & lt) == 0) wcnt[warp][d] += __popc(pm);
         __syncwarp();
     }
     __syncthreads();
@@ -281,15 +290,16 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
     // pass 2: place each item at its stable slot in shared memory
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
-        const unsigned peers = __match_any_sync(ROSA_FULL_MASK, dig[u]);
-        const unsigned before = __popc(peers & lanemask_lt());
-        if (dig[u] < kRadixBins) {
-            const uint32_t pos = wcnt[warp][dig[u]] + before;
+        const bool ok = wbase + u * 32 + lane < lim;
+        const unsigned d = (unsigned)(key[u] >> shift) & (kRadixBins - 1);
+        const unsigned before = __popc(peer[u] & lt);
+        if (ok) {
+            const uint32_t pos = wcnt[warp][d] + before;
             sk[pos] = key[u];
             sv[pos] = val[u];
         }
         __syncwarp();
-        if (dig[u] < kRadixBins && before == 0) wcnt[warp][dig[u]] += __popc(peers);
+        if (ok && before == 0) wcnt[warp][d] += __popc(peer[u]);
         __syncwarp();
     }
     __syncthreads();
@@ -564,7 +574,7 @@ __device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
 __global__ void __launch_bounds__(kL2)
 summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__restrict__ lcp,
                int32_t *__restrict__ minpos1, int32_t *__restrict__ emin1, int32_t *__restrict__ ein1,
-               int32_t *__restrict__ minpos2, int32_t *__restrict__ emin2) {
+               int32_t *__restrict__ minpos2, int32_t *__restrict__ emin2, int32_t *__restrict__ ein2) {
     __shared__ int wpos[32], wemin[32], wfirst[32];
     const int s = blockIdx.x / G.nb2, B2 = blockIdx.x - s * G.nb2;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -604,6 +614,7 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
         if (lane == 0) {
             minpos2[(int64_t)s * G.nb2 + B2] = p2;
             emin2[(int64_t)s * G.nb2 + B2] = e2;
+            ein2[(int64_t)s * G.nb2 + B2] = first;
         }
     }
 }
@@ -875,11 +886,11 @@ constexpr int kRThreads = 256;
 struct StreamView {
     const uint32_t *sa;
     const int32_t *lcp;
-    const int32_t *mp1, *em1, *ein1, *mp2, *em2;
+    const int32_t *mp1, *em1, *ein1, *mp2, *em2, *ein2;
     const int32_t *kcount;
     const WWord *W;
     const int *Z;
-    int n, T, nb1, nbits, nw;
+    int n, T, nb1, nb2, nbits, nw;
     bool same;
 };
 
@@ -893,7 +904,7 @@ __device__ __forceinline__ int kc(const StreamView &v, int r) {
 
 struct ResolveArgs {
     const uint32_t *sa;
-    const int32_t *lcp, *mp1, *em1, *ein1, *mp2, *em2, *kcount;
+    const int32_t *lcp, *mp1, *em1, *ein1, *mp2, *em2, *ein2, *kcount;
     const WWord *words;
     const int *wz;
     int nbits;
@@ -904,8 +915,9 @@ __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const 
     const int nw = (G.T >> 6) + 1;
     return StreamView{A.sa + seg, A.lcp + seg, A.mp1 + (int64_t)s * G.nb1, A.em1 + (int64_t)s * G.nb1,
                       A.ein1 + (int64_t)s * G.nb1, A.mp2 + (int64_t)s * G.nb2, A.em2 + (int64_t)s * G.nb2,
-                      A.kcount ? A.kcount + seg : nullptr, A.words + (int64_t)s * A.nbits * nw,
-                      A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, A.nbits, nw, G.same};
+                      A.ein2 + (int64_t)s * G.nb2, A.kcount ? A.kcount + seg : nullptr,
+                      A.words + (int64_t)s * A.nbits * nw, A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, G.nb2,
+                      A.nbits, nw, G.same};
 }
 
 __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *vsym, int s, int t, int L, int ib,
@@ -1260,6 +1272,33 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
     next += dir * cnt;
     // `next` is now the last (dir < 0) or first (dir > 0) rank of block next / 32
     while (next >= 0 && next < v.n) {
+        if ((dir < 0 && (next & (kL2 - 1)) == kL2 - 1) || (dir > 0 && (next & (kL2 - 1)) == 0)) {
+            // at a 1024-rank boundary: try to cross up to 32 whole 1024-blocks at once
+            const int nb2 = next / kL2;
+            const int b2 = nb2 + dir * lane;
+            const bool in2 = b2 >= 0 && b2 < v.nb2 && (b2 + 1) * kL2 <= v.n;
+            int bm2 = -1;
+            bool hv2 = true;
+            if (in2) {
+                const int edge = dir < 0 ? ((b2 + 1) * kL2 < v.n ? v.ein2[b2 + 1] : INT_MAX) : v.ein2[b2];
+                bm2 = min(edge, v.em2[b2]);
+                hv2 = v.mp2[b2] <= X;
+            }
+            const int M2 = min(carry, warp_prefix_min(bm2, lane));
+            const bool st2 = MODE == NEAREST ? (!in2 || hv2 || M2 <= lim) : (!in2 || M2 < lim);
+            const unsigned sm2 = __ballot_sync(ROSA_FULL_MASK, st2);
+            const int f2 = sm2 ? __ffs(sm2) - 1 : 32;
+            if (f2 > 0) {
+                carry = min(carry, __shfl_sync(ROSA_FULL_MASK, M2, f2 - 1));
+                if (MODE == BOUND) {
+                    const int bl = nb2 + dir * (f2 - 1);
+                    result = dir < 0 ? bl * kL2 : bl * kL2 + kL2 - 1;
+                }
+                next += dir * kL2 * f2;
+                if (f2 == 32) continue;
+                if (next < 0 || next >= v.n) break;
+            }
+        }
         const int nb = next / kL1;
         const int b = nb + dir * lane;
         const bool inside = b >= 0 && b < v.nb1 && (b + 1) * kL1 <= v.n;
@@ -1414,7 +1453,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     lcp_long_kernel<<<kNumSMs * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
     // 3a. summaries
     summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
-                                                           W.minpos2, W.emin2);
+                                                           W.minpos2, W.emin2, W.ein2);
     // 3b. wavelet matrix over key positions in rank order
     if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wbits * G.S * G.ntw * 4, st)) != cudaSuccess) return err;
     if (!G.same) key_tile_count_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile);
@@ -1428,7 +1467,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     if ((err = cudaFuncSetAttribute(resolve_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)sizeof(WinSmem))) != cudaSuccess)
         return err;
-    ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, G.same ? nullptr : W.kcount,
+    ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.same ? nullptr : W.kcount,
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
