@@ -99,6 +99,7 @@ struct Workspace {
     int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2, *ein2;
     int32_t *hard;           // ranks of queries left for the warp-cooperative phase
     int32_t *wq;             // output slots of queries waiting for a wavelet lookup
+    int32_t *hardb;          // ranks of queries whose interval runs past their window
     int32_t *kcount;         // keys before each rank (q != k)
     int *ktile;              // keys per 2048-rank tile
     uint32_t *wvals[2];      // wavelet level sequences
@@ -142,6 +143,7 @@ Workspace carve(const Geometry &G, void *base) {
     W.ein2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.hard = (int32_t *)take(N * 4);
     W.wq = (int32_t *)take((size_t)G.S * G.T * 4);
+    W.hardb = (int32_t *)take((size_t)G.S * G.T * 4);
     W.kcount = (int32_t *)take(N * 4);
     W.ktile = (int *)take((size_t)G.S * G.ntps * 4);
     W.wvals[0] = (uint32_t *)take((size_t)G.S * G.T * 4);
@@ -1012,9 +1014,9 @@ __device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int l
     return kNeedHard;
 }
 
-// Interval of local ranks around jl whose LCP with jl is >= L.  Returns false
-// when it may extend beyond the window.
-__device__ bool window_bounds(const WinSmem &w, bool at_start, int jl, int L, int &lo, int &hi) {
+// Interval of local ranks around jl whose LCP with jl is >= L.  A side that
+// may extend beyond the window is returned as -1.
+__device__ void window_bounds(const WinSmem &w, bool at_start, int jl, int L, int &lo, int &hi) {
     if (L < 255) {
         int cur = jl;
 #pragma unroll
@@ -1022,27 +1024,22 @@ __device__ bool window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
             const int c = cur - (1 << k);
             if (c >= 0 && w.sp[k][c + 1] >= L) cur = c;
         }
-        if (cur == 0 && !at_start && w.lc[0] >= L) return false;
-        lo = cur;
+        lo = (cur == 0 && !at_start && w.lc[0] >= L) ? -1 : cur;
         cur = jl;
 #pragma unroll
         for (int k = kSpLevels - 1; k >= 0; --k) {
             const int c = cur + (1 << k);
             if (c < kRWin && w.sp[k][cur + 1] >= L) cur = c;
         }
-        if (cur == kRWin - 1 && w.lc[kRWin] >= L) return false;
-        hi = cur;
+        hi = (cur == kRWin - 1 && w.lc[kRWin] >= L) ? -1 : cur;
     } else {   // long matches: exact edges (such intervals are short)
         int r = jl;
         while (r > 0 && w.lc[r] >= L) --r;
-        if (r == 0 && !at_start && w.lc[0] >= L) return false;
-        lo = r;
+        lo = (r == 0 && !at_start && w.lc[0] >= L) ? -1 : r;
         r = jl;
         while (r + 1 < kRWin && w.lc[r + 1] >= L) ++r;
-        if (r == kRWin - 1 && w.lc[kRWin] >= L) return false;
-        hi = r;
+        hi = (r == kRWin - 1 && w.lc[kRWin] >= L) ? -1 : r;
     }
-    return true;
 }
 
 // One CTA per 1024 ranks of a stream, with 1024 ranks of context on each side.
@@ -1057,7 +1054,8 @@ __device__ bool window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
 __global__ void __launch_bounds__(kRThreads)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
-                    int *hard_count, int32_t *__restrict__ wq, int *wq_count) {
+                    int *hard_count, int32_t *__restrict__ hardb, int *hardb_count, int32_t *__restrict__ wq,
+                    int *wq_count) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     WinSmem &w = *reinterpret_cast<WinSmem *>(smem_raw);
     const int ntr = ceil_div(G.n, kRTile);
@@ -1167,9 +1165,21 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         const int X = t - G.g;
         const int L = w.qL[qi];
         int lo = 0, hi = -1;
-        if (L == kNeedHard || (L > 0 && !window_bounds(w, at_start, jl, L, lo, hi))) {
+        if (L == kNeedHard) {
             hard[atomicAdd(hard_count, 1)] = (int32_t)(seg + w0 + jl);
             continue;
+        }
+        if (L > 0) {
+            window_bounds(w, at_start, jl, L, lo, hi);
+            if (lo < 0 || hi < 0) {
+                // L is known; only the interval's far end lies outside the window
+                const int64_t o = (int64_t)s * G.T + t;
+                len[o] = L;
+                end_idx[o] = lo < 0 ? -1 : w0 + lo;
+                sym[o] = hi < 0 ? -1 : w0 + hi;
+                hardb[atomicAdd(hardb_count, 1)] = (int32_t)(seg + w0 + jl);
+                continue;
+            }
         }
         int ib = -1;
         if (L > 0) {
@@ -1367,6 +1377,39 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restri
     }
 }
 
+// Queries whose L is known but whose interval runs past the staged window:
+// one warp scans outward from the window edge on each open side, then the
+// query is parked for the wavelet lookup.
+__global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
+                                      const int32_t *__restrict__ len, int32_t *__restrict__ sym,
+                                      const int32_t *__restrict__ hardb, const int *__restrict__ hardb_count,
+                                      int32_t *__restrict__ wq, int *wq_count) {
+    const int nh = *hardb_count;
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t h = wid; h < nh; h += nw) {
+        const int64_t gi = hardb[h];
+        const int s = (int)(gi / G.n);
+        const int j = (int)(gi - (int64_t)s * G.n);
+        const uint32_t x = A.sa[gi];
+        const int t = G.same ? (int)x : (int)x - G.T;
+        const int X = t - G.g;
+        const int64_t o = (int64_t)s * G.T + t;
+        const int L = len[o];
+        int lo = end_idx[o], hi = sym[o];
+        const int w0 = (j / kRTile) * kRTile - kRHalo;
+        const StreamView v = make_view(G, s, A);
+        if (lo < 0) lo = warp_scan<BOUND>(v, w0, -1, X, L, lane);
+        if (hi < 0) hi = warp_scan<BOUND>(v, w0 + kRWin - 1, +1, X, L, lane);
+        if (lane == 0) {
+            end_idx[o] = kc(v, lo);
+            sym[o] = kc(v, hi + 1);
+            wq[atomicAdd(wq_count, 1)] = (int32_t)o;
+        }
+    }
+}
+
 // Largest admissible key position inside each parked query's key range.
 __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                                      int32_t *__restrict__ end_idx, int32_t *__restrict__ sym,
@@ -1396,8 +1439,8 @@ int match_launch_count(int S, int T, int K, bool same) {
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
-    // + wavelet (key count when q != k, compaction, one per level) + 3 resolve
-    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 3;
+    // + wavelet (key count when q != k, compaction, one per level) + 4 resolve
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 4;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1471,9 +1514,12 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
+    int *hardb_count = W.counts + 7;
     resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
-        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
+        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.hardb, hardb_count, W.wq, wq_count);
     resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
+    resolve_bounds_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardb, hardb_count, W.wq,
+                                                        wq_count);
     wavelet_query_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
     return cudaGetLastError();
 }
