@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--streams", type=int, default=0,
                     help="profiling aid: keep only the first N streams of a symbol workload")
+    ap.add_argument("--no-graph", action="store_true", help="launch every kernel eagerly instead of graph replay")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-streams", type=int, default=0,
@@ -158,30 +159,51 @@ class Runner:
         n += 1 if "gather" in wl["ops"] else 0
         return n
 
-    def step(self, events=None):
+        self.graphs = None
+
+    def _op(self, name):
         rosa, wl = self.rosa, self.wl
-        ev = events or {}
-
-        def mark(name):
-            if name in ev:
-                ev[name].record()
-
-        if "discretize" in wl["ops"]:
-            mark("discretize0")
+        if name == "discretize":
             rosa.discretize(wl["qvec"], wl["M"], out=self.sq)
             rosa.discretize(wl["kvec"], wl["M"], out=self.sk)
-            mark("discretize1")
-            q = self.sq.view(wl["S"], wl["T"])
-            k = self.sk.view(wl["S"], wl["T"])
-        else:
-            q, k = wl["q"], wl["k"]
-        mark("match0")
-        rosa.match(q, None if wl["same"] else k, K=wl["K"], g=wl["g"], out=self.outs, workspace=self.ws)
-        mark("match1")
-        if "gather" in wl["ops"]:
-            mark("gather0")
+        elif name == "match":
+            if "discretize" in wl["ops"]:
+                q, k = self.sq.view(wl["S"], wl["T"]), self.sk.view(wl["S"], wl["T"])
+            else:
+                q, k = wl["q"], wl["k"]
+            rosa.match(q, None if wl["same"] else k, K=wl["K"], g=wl["g"], out=self.outs, workspace=self.ws)
+        elif name == "gather":
             rosa.gather(wl["V"], self.outs[0], wl["R"], wl["d"], wl["rho"], out=self.gout)
-            mark("gather1")
+
+    def capture(self):
+        """Capture each op of the step as a CUDA graph (after eager warm-up),
+        so a step is a few graph launches instead of ~100 kernel launches."""
+        torch = self.torch
+        self.graphs = {}
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for op in self.wl["ops"]:
+                self._op(op)
+        torch.cuda.current_stream().wait_stream(side)
+        for op in self.wl["ops"]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._op(op)
+            self.graphs[op] = g
+        torch.cuda.synchronize()
+
+    def step(self, events=None):
+        ev = events or {}
+        for op in self.wl["ops"]:
+            if op + "0" in ev:
+                ev[op + "0"].record()
+            if self.graphs:
+                self.graphs[op].replay()
+            else:
+                self._op(op)
+            if op + "1" in ev:
+                ev[op + "1"].record()
 
 
 # --------------------------------------------------------------------------- clocks
@@ -321,6 +343,10 @@ def main():
     for _ in range(max(3, args.warmup)):
         runner.step()
     torch.cuda.synchronize()
+    if not args.no_graph:
+        runner.capture()
+        runner.step()
+        torch.cuda.synchronize()
 
     names = [o + s for o in wl["ops"] for s in ("0", "1")]
     per_step = []
@@ -384,6 +410,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
             "config": {"workload": wl["name"], "streams": wl["S"], "T": wl["T"], "K": wl["K"], "g": wl["g"],
                        "q_equals_k": wl["same"], "ops": wl["ops"], "parallelism": f"streams x{world} (weak)",
+                       "launch": "eager" if args.no_graph else "one CUDA graph per op",
                        "l2": "flushed before every timed step (256 MiB memset outside the events)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": runner.launches() * args.steps, "clocks": clocks,

@@ -27,6 +27,7 @@
 // All kernels are stream-segmented: items of stream s occupy [s*n, (s+1)*n).
 #include <climits>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/rosa.h"
@@ -883,7 +884,7 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
 constexpr int kRTile = 1024;
 constexpr int kRHalo = 1024;
 constexpr int kRWin = kRTile + 2 * kRHalo;
-constexpr int kRThreads = 256;
+constexpr int kRThreads = 512;
 
 struct StreamView {
     const uint32_t *sa;
@@ -1430,6 +1431,21 @@ __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *_
 
 inline unsigned grid_for(int64_t n, int threads) { return (unsigned)ceil_div64(n, threads); }
 
+// The resolve tile needs more than 48 KB of shared memory; opt in once per
+// device (a host-side attribute, so later calls, captured or not, skip it).
+cudaError_t tile_smem_optin() {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(resolve_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(WinSmem));
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    return e;
+}
+
 }  // namespace
 
 int match_launch_count(int S, int T, int K, bool same) {
@@ -1507,9 +1523,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
         wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, G.wbits, lv, W.wvals[lv & 1],
                                                                        W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
     // 3c. resolve: thread per query, then warp per query for the long scans
-    if ((err = cudaFuncSetAttribute(resolve_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)sizeof(WinSmem))) != cudaSuccess)
-        return err;
+    if ((err = tile_smem_optin()) != cudaSuccess) return err;
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.same ? nullptr : W.kcount,
                   words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
