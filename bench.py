@@ -151,6 +151,7 @@ class Runner:
             self.sk = torch.empty_like(self.sq)
         if "gather" in wl["ops"]:
             self.gout = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
+        self.graphs = None
 
     def launches(self):
         wl = self.wl
@@ -158,8 +159,6 @@ class Runner:
         n += 2 if "discretize" in wl["ops"] else 0
         n += 1 if "gather" in wl["ops"] else 0
         return n
-
-        self.graphs = None
 
     def _op(self, name):
         rosa, wl = self.rosa, self.wl
