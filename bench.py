@@ -269,6 +269,14 @@ def reduce_over_ranks(local_ms: float, local_units: float, device=None):
     return float(t.item()), float(u.item())
 
 
+# DRAM bytes (read + write) of one rosa_match call, from an ncu capture of the
+# same kernels (dram__bytes_read.sum + dram__bytes_write.sum); None where no
+# capture of the current kernels exists.  zipf-256-131k: captured on its first
+# 16 streams (1.227 GB per call) and scaled by the 8x stream count, which is
+# exact in expectation because the streams are independent.
+PROFILED_DRAM_BYTES = {"zipf-256-131k": 9.81e9}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -387,7 +395,8 @@ def main():
     achieved = ab[dom] / (mean_op[dom] / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": f"rosa_{dom}", "achieved": round(achieved, 2), "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 5),
-                "traffic": None, "algorithmic_bytes": ab[dom], "ms": round(mean_op[dom], 4),
+                "traffic": (PROFILED_DRAM_BYTES.get(wl["name"]) if dom == "match" else None),
+                "algorithmic_bytes": ab[dom], "ms": round(mean_op[dom], 4),
                 "ops_ms": {o: round(v, 4) for o, v in mean_op.items()}}
 
     e2e = None
