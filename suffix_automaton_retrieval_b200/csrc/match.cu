@@ -100,7 +100,10 @@ struct Workspace {
     int32_t *minpos1, *emin1, *ein1, *minpos2, *emin2, *ein2;
     int32_t *hard;           // ranks of queries left for the warp-cooperative phase
     int32_t *wq;             // output slots of queries waiting for a wavelet lookup
-    int32_t *hardb;          // ranks of queries whose interval runs past their window
+    int32_t *hardb;          // ranks of queries whose interval runs past their window (long L)
+    int32_t *hardw;          // same, short L: waiting for a shared per-tile bound
+    int32_t *btask;          // (tile, side, L) bound tasks
+    int32_t *btab;           // their results
     int32_t *kcount;         // keys before each rank (q != k)
     int *ktile;              // keys per 2048-rank tile
     uint32_t *wvals[2];      // wavelet level sequences
@@ -145,6 +148,10 @@ Workspace carve(const Geometry &G, void *base) {
     W.hard = (int32_t *)take(N * 4);
     W.wq = (int32_t *)take((size_t)G.S * G.T * 4);
     W.hardb = (int32_t *)take((size_t)G.S * G.T * 4);
+    W.hardw = (int32_t *)take((size_t)G.S * G.T * 4);
+    const size_t ntiles_resolve = (size_t)G.S * ceil_div(G.n, 1024);
+    W.btask = (int32_t *)take(ntiles_resolve * 128 * 4);
+    W.btab = (int32_t *)take(ntiles_resolve * 128 * 4);
     W.kcount = (int32_t *)take(N * 4);
     W.ktile = (int *)take((size_t)G.S * G.ntps * 4);
     W.wvals[0] = (uint32_t *)take((size_t)G.S * G.T * 4);
@@ -961,6 +968,7 @@ constexpr int kNeedWarp = -1;          // qL codes
 constexpr int kNeedHard = -2;
 
 constexpr int kWarpScanMax = 256;      // widest interval a warp scans in shared memory
+constexpr int kBoundShared = 64;       // match lengths whose out-of-window bounds are shared per tile
 
 struct WinSmem {
     int kp[kRWin];
@@ -971,6 +979,7 @@ struct WinSmem {
     int16_t bq[kRTile];
     int16_t dlo[kRTile];     // phase D: interval bounds of queries a warp finishes
     int16_t dhi[kRTile];     // (their query indices reuse bq)
+    unsigned long long need[2];   // lengths L < 64 whose interval leaves the window below / above
     int nq, nb, nd;
     uint8_t sp[kSpLevels][kRWin];
 };
@@ -1055,7 +1064,8 @@ __device__ void window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
 __global__ void __launch_bounds__(kRThreads)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
-                    int *hard_count, int32_t *__restrict__ hardb, int *hardb_count, int32_t *__restrict__ wq,
+                    int *hard_count, int32_t *__restrict__ hardb, int *hardb_count, int32_t *__restrict__ hardw,
+                    int *hardw_count, int32_t *__restrict__ btask, int *btask_count, int32_t *__restrict__ wq,
                     int *wq_count) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     WinSmem &w = *reinterpret_cast<WinSmem *>(smem_raw);
@@ -1064,7 +1074,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const int64_t seg = (int64_t)s * G.n;
     const int w0 = tt * kRTile - kRHalo;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; w.nd = 0; }
+    if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; w.nd = 0; w.need[0] = 0; w.need[1] = 0; }
     for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
         const int r = w0 + i;
         int p = INT_MAX, l = -1;
@@ -1173,12 +1183,19 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         if (L > 0) {
             window_bounds(w, at_start, jl, L, lo, hi);
             if (lo < 0 || hi < 0) {
-                // L is known; only the interval's far end lies outside the window
+                // L is known; only the interval's far end lies outside the window.  That
+                // end depends on (tile, side, L) alone, so short L share one scan.
                 const int64_t o = (int64_t)s * G.T + t;
                 len[o] = L;
                 end_idx[o] = lo < 0 ? -1 : w0 + lo;
                 sym[o] = hi < 0 ? -1 : w0 + hi;
-                hardb[atomicAdd(hardb_count, 1)] = (int32_t)(seg + w0 + jl);
+                if (L < kBoundShared) {
+                    if (lo < 0) atomicOr(&w.need[0], 1ull << L);
+                    if (hi < 0) atomicOr(&w.need[1], 1ull << L);
+                    hardw[atomicAdd(hardw_count, 1)] = (int32_t)(seg + w0 + jl);
+                } else {
+                    hardb[atomicAdd(hardb_count, 1)] = (int32_t)(seg + w0 + jl);
+                }
                 continue;
             }
         }
@@ -1220,6 +1237,12 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
         if (lane == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
+    }
+    // one bound task per (side, L) this tile needs beyond its window
+    if (threadIdx.x < 2 * kBoundShared) {
+        const int side = threadIdx.x / kBoundShared, L = threadIdx.x % kBoundShared;
+        if ((w.need[side] >> L) & 1ull)
+            btask[atomicAdd(btask_count, 1)] = (int32_t)(((int64_t)blockIdx.x << 7) | (side << 6) | L);
     }
 }
 
@@ -1411,6 +1434,53 @@ __global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, int32_t *__rest
     }
 }
 
+// One warp per (tile, side, L): the interval bound beyond the tile's window.
+__global__ void bound_task_kernel(Geometry G, ResolveArgs A, const int32_t *__restrict__ btask,
+                                  const int *__restrict__ btask_count, int32_t *__restrict__ btab) {
+    const int nt = *btask_count;
+    const int lane = threadIdx.x & 31;
+    const int ntr = ceil_div(G.n, kRTile);
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t e = wid; e < nt; e += nw) {
+        const int code = btask[e];
+        const int tile = code >> 7, side = (code >> 6) & 1, L = code & 63;
+        const int s = tile / ntr, tt = tile - s * ntr;
+        const int w0 = tt * kRTile - kRHalo;
+        const StreamView v = make_view(G, s, A);
+        const int r = side ? warp_scan<BOUND>(v, w0 + kRWin - 1, +1, 0, L, lane)
+                           : warp_scan<BOUND>(v, w0, -1, 0, L, lane);
+        if (lane == 0) btab[(int64_t)tile * 2 * kBoundShared + side * kBoundShared + L] = r;
+    }
+}
+
+// Queries waiting for a shared bound: fill the open side(s) from the table
+// and park the query for the wavelet lookup.
+__global__ void bound_finish_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
+                                    const int32_t *__restrict__ len, int32_t *__restrict__ sym,
+                                    const int32_t *__restrict__ hardw, const int *__restrict__ hardw_count,
+                                    const int32_t *__restrict__ btab, int32_t *__restrict__ wq, int *wq_count) {
+    const int nh = *hardw_count;
+    const int ntr = ceil_div(G.n, kRTile);
+    for (int64_t h = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; h < nh; h += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t gi = hardw[h];
+        const int s = (int)(gi / G.n);
+        const int j = (int)(gi - (int64_t)s * G.n);
+        const uint32_t x = A.sa[gi];
+        const int t = G.same ? (int)x : (int)x - G.T;
+        const int64_t o = (int64_t)s * G.T + t;
+        const int L = len[o];
+        const int64_t tb = ((int64_t)s * ntr + j / kRTile) * 2 * kBoundShared;
+        int lo = end_idx[o], hi = sym[o];
+        if (lo < 0) lo = btab[tb + L];
+        if (hi < 0) hi = btab[tb + kBoundShared + L];
+        const StreamView v = make_view(G, s, A);
+        end_idx[o] = kc(v, lo);
+        sym[o] = kc(v, hi + 1);
+        wq[atomicAdd(wq_count, 1)] = (int32_t)o;
+    }
+}
+
 // Largest admissible key position inside each parked query's key range.
 __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                                      int32_t *__restrict__ end_idx, int32_t *__restrict__ sym,
@@ -1455,8 +1525,8 @@ int match_launch_count(int S, int T, int K, bool same) {
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
-    // + wavelet (key count when q != k, compaction, one per level) + 4 resolve
-    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 4;
+    // + wavelet (key count when q != k, compaction, one per level) + 6 resolve
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 6;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1529,11 +1599,17 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
     int *hardb_count = W.counts + 7;
+    int *hardw_count = W.counts + 8;
+    int *btask_count = W.counts + 9;
     resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
-        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.hardb, hardb_count, W.wq, wq_count);
+        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.hardb, hardb_count, W.hardw, hardw_count, W.btask,
+        btask_count, W.wq, wq_count);
     resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
     resolve_bounds_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardb, hardb_count, W.wq,
                                                         wq_count);
+    bound_task_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, W.btask, btask_count, W.btab);
+    bound_finish_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardw, hardw_count, W.btab, W.wq,
+                                                      wq_count);
     wavelet_query_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
     return cudaGetLastError();
 }
