@@ -70,9 +70,10 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     G.N = (int64_t)S * G.n;
     G.bps = bits_for(K - 1);
     if (G.bps < 1) G.bps = 1;
-    // D0 symbols of bps bits plus the available length (0..D0+1) must fit 64 bits
-    int d = 64 / G.bps;
-    while (d > 1 && d * G.bps + bits_for(d + 1) > 64) --d;
+    // D0 symbols of bps bits plus the available length (0..D0+1) in at most 56
+    // bits: seven 8-bit radix passes; deeper ties go to prefix doubling
+    int d = 56 / G.bps;
+    while (d > 1 && d * G.bps + bits_for(d + 1) > 56) --d;
     G.D0 = d;
     G.abits = bits_for(d + 1);
     G.keybits = d * G.bps + G.abits;
