@@ -964,7 +964,7 @@ __device__ __forceinline__ int warp_prefix_min(int x, int lane) {
 // Queries are resolved in three uniform phases (see resolve_tile_kernel).
 constexpr int kSpLevels = 11;          // lifting reaches 2^11 - 1 ranks: a whole side of the window
 constexpr int kProbe = 16;             // ranks a lane probes on each side before its warp helps
-constexpr int kLaneScan = 256;         // ranks a lane scans on each side for a query the probes left open
+constexpr int kWarpSteps = 24;         // 32-rank steps of a warp-cooperative scan (768 ranks)
 constexpr int kNeedWarp = -1;          // qL codes
 constexpr int kNeedHard = -2;
 
@@ -995,6 +995,34 @@ __device__ __forceinline__ void defer_wavelet(const Geometry &G, int s, int t, i
     end_idx[o] = klo;
     sym[o] = khi;
     wq[atomicAdd(wq_count, 1)] = (int32_t)o;
+}
+
+// Warp-cooperative nearest admissible key in direction dir, 32 ranks per
+// step: the LCP with it when that exceeds lim, 0 when the running LCP falls
+// to lim first, kNeedHard when the answer lies beyond the window or the steps.
+__device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int lim, int lane) {
+    int carry = INT_MAX;
+    for (int step = 0; step < kWarpSteps; ++step) {
+        const int r = jl + dir * (1 + step * 32 + lane);
+        int e;
+        bool valid;
+        if (dir < 0) {
+            e = r >= -1 ? w.lc[r + 1] : kNeedHard;
+            valid = r >= 0 && w.kp[r] <= X;
+        } else {
+            e = r <= kRWin ? w.lc[r] : kNeedHard;
+            valid = r < kRWin && w.kp[r] <= X;
+        }
+        const int pm = min(carry, warp_prefix_min(e, lane));
+        const unsigned sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
+        const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid && pm > lim);
+        const int fs = sm ? __ffs(sm) - 1 : 32;
+        const int fv = vm ? __ffs(vm) - 1 : 32;
+        if (fv < fs) return __shfl_sync(ROSA_FULL_MASK, pm, fv);
+        if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
+        carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
+    }
+    return kNeedHard;
 }
 
 // Interval of local ranks around jl whose LCP with jl is >= L.  A side that
@@ -1046,7 +1074,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const int s = blockIdx.x / ntr, tt = blockIdx.x - s * ntr;
     const int64_t seg = (int64_t)s * G.n;
     const int w0 = tt * kRTile - kRHalo;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; w.nd = 0; w.need[0] = 0; w.need[1] = 0; }
     for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
         const int r = w0 + i;
@@ -1090,7 +1118,6 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     }
     __syncthreads();
     const int nq = w.nq;
-    const bool at_start_b = w0 <= 0;
     // Phase A
     for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
         const int jl = w.qj[qi];
@@ -1126,37 +1153,19 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         w.qL[qi] = L;
     }
     __syncthreads();
-    // Phase B: one lane per query the probes left open, scanning up to
-    // kLaneScan ranks each way in shared memory (ranks beyond: hard list)
+    // Phase B
     const int nb = w.nb;
-    for (int bi = threadIdx.x; bi < nb; bi += kRThreads) {
+    for (int bi = warp; bi < nb; bi += kRThreads / 32) {
         const int qi = w.bq[bi];
         const int jl = w.qj[qi];
         const int X = w.qt[qi] - G.g;
-        int Ll = kNeedHard;
-        {
-            int m = INT_MAX;
-            const int stop = max(-1, jl - 1 - kLaneScan);
-            for (int r = jl - 1; r > stop; --r) {
-                m = min(m, w.lc[r + 1]);
-                if (m <= 0) { Ll = 0; break; }
-                if (w.kp[r] <= X) { Ll = m; break; }
-            }
-            // reached the window start inside the stream: the stream start edge decides
-            if (Ll == kNeedHard && stop < 0 && at_start_b && w.lc[0] <= 0) Ll = 0;
-        }
-        int L = kNeedHard;
+        const int Ll = warp_nearest_smem(w, jl, X, -1, 0, lane);
+        int L = Ll;
         if (Ll != kNeedHard) {
-            int m = INT_MAX, Lr = kNeedHard;
-            const int stop = min(kRWin + 1, jl + 1 + kLaneScan);
-            for (int r = jl + 1; r < stop; ++r) {
-                m = min(m, w.lc[r]);             // lc[kRWin] is the edge past the window
-                if (m <= Ll) { Lr = 0; break; }
-                if (r < kRWin && w.kp[r] <= X) { Lr = m; break; }
-            }
-            if (Lr != kNeedHard) L = max(Ll, Lr);
+            const int Lr = warp_nearest_smem(w, jl, X, +1, Ll, lane);
+            L = Lr == kNeedHard ? kNeedHard : max(Ll, Lr);
         }
-        w.qL[qi] = L;
+        if (lane == 0) w.qL[qi] = L;
     }
     __syncthreads();
     // Phase C
@@ -1215,18 +1224,20 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
     }
     __syncthreads();
-    // Phase D: mid-size intervals, one lane each
+    // Phase D: mid-size intervals, one warp each, 32 ranks per step
     const int nd = w.nd;
-    for (int di = threadIdx.x; di < nd; di += kRThreads) {
+    for (int di = warp; di < nd; di += kRThreads / 32) {
         const int qi = w.bq[di];
         const int lo = w.dlo[di], hi = w.dhi[di];
         const int X = w.qt[qi] - G.g;
         int best = -1;
-        for (int r = lo; r <= hi; ++r) {
+        for (int r = lo + lane; r <= hi; r += 32) {
             const int c = w.kp[r];
             if (c <= X) best = max(best, c);
         }
-        write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
+        if (lane == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
     }
     // one bound task per (side, L) this tile needs beyond its window
     if (threadIdx.x < 2 * kBoundShared) {
