@@ -890,7 +890,7 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
 //     queries per warp in parallel.
 // ---------------------------------------------------------------------------
 constexpr int kRTile = 1024;
-constexpr int kRHalo = 1024;
+constexpr int kRHalo = 512;
 constexpr int kRWin = kRTile + 2 * kRHalo;
 constexpr int kRThreads = 512;
 
@@ -1062,7 +1062,7 @@ __device__ void window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
 //            sparse table, then i* by a 16-rank probe or, for wider
 //            intervals, a deferred wavelet lookup.
 // Queries whose answer needs ranks outside the window go to the hard list.
-__global__ void __launch_bounds__(kRThreads)
+__global__ void __launch_bounds__(kRThreads, 4)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
                     int *hard_count, int32_t *__restrict__ hardb, int *hardb_count, int32_t *__restrict__ hardw,
@@ -1090,10 +1090,28 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         w.lc[i] = l;
     }
     __syncthreads();
+    // sparse table levels, four byte entries per step with byte-wise SIMD minima
     for (int k = 1; k < kSpLevels; ++k) {
         const int h = 1 << (k - 1);
-        for (int i = threadIdx.x; i < kRWin; i += kRThreads)
-            w.sp[k][i] = (i + 2 * h - 1 < kRWin) ? min(w.sp[k - 1][i], w.sp[k - 1][i + h]) : 0;
+        const uint32_t *prev = reinterpret_cast<const uint32_t *>(w.sp[k - 1]);
+        uint32_t *cur = reinterpret_cast<uint32_t *>(w.sp[k]);
+        for (int q4 = threadIdx.x; q4 < kRWin / 4; q4 += kRThreads) {
+            const int i = q4 * 4;
+            const uint32_t a = prev[q4];
+            uint32_t b;
+            if ((h & 3) == 0) {
+                b = (i + h < kRWin) ? prev[q4 + (h >> 2)] : 0u;
+            } else {   // h = 1 or 2: bytes i+h .. i+h+3 straddle two words
+                const uint32_t lo = prev[q4];
+                const uint32_t hi = (q4 + 1 < kRWin / 4) ? prev[q4 + 1] : 0u;
+                b = __byte_perm(lo, hi, h == 1 ? 0x4321 : 0x5432);
+            }
+            uint32_t m = __vminu4(a, b);
+            // entries whose range runs past the window stay 0 (never read)
+            const int valid = kRWin - (2 * h - 1) - i;   // entries i .. i+valid-1 are in range
+            if (valid < 4) m = valid <= 0 ? 0u : (m & (0xffffffffu >> (8 * (4 - valid))));
+            cur[q4] = m;
+        }
         __syncthreads();
     }
     // compact the tile's query items so that every lane has one to answer
