@@ -57,7 +57,7 @@ int bits_for(int v) {   // number of bits to hold values 0..v
 struct Geometry {
     int S, T, K, g, n;
     bool same;
-    int bps, D0, abits, keybits;
+    int bps, D0, abits, idbits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
     int wbits, ntw, nw;      // wavelet matrix: levels, 2048-element tiles and 64-bit words per stream
@@ -70,13 +70,17 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     G.N = (int64_t)S * G.n;
     G.bps = bits_for(K - 1);
     if (G.bps < 1) G.bps = 1;
-    // D0 symbols of bps bits plus the available length (0..D0+1) in at most 56
-    // bits: seven 8-bit radix passes; deeper ties go to prefix doubling
-    int d = 56 / G.bps;
-    while (d > 1 && d * G.bps + bits_for(d + 1) > 56) --d;
+    // 64-bit sort key: [D0 symbols | available length 0..D0+1 | item id].  The
+    // symbols and length take at most 48 bits (six 8-bit radix passes) and at
+    // most what the item id leaves; deeper ties go to prefix doubling.
+    G.idbits = bits_for(G.n > 0 ? G.n - 1 : 0);
+    if (G.idbits < 1) G.idbits = 1;
+    const int budget = min(48, 64 - G.idbits);
+    int d = budget / G.bps;
+    while (d > 1 && d * G.bps + bits_for(d + 1) > budget) --d;
     G.D0 = d;
     G.abits = bits_for(d + 1);
-    G.keybits = d * G.bps + G.abits;
+    G.keybits = G.idbits + d * G.bps + G.abits;
     G.ntps = ceil_div(G.n, kRadixTile);
     G.nb1 = ceil_div(G.n, kL1);
     G.nb2 = ceil_div(G.n, kL2);
@@ -92,7 +96,7 @@ struct Workspace {
     uint32_t *status;
     int *counts;             // [2 buffers][2 kinds]
     uint64_t *keys[2];
-    uint32_t *vals[2];
+    uint32_t *sa;            // item ids in sorted order (low bits of the sorted keys)
     int32_t *rank;
     int32_t *lcp;
     uint32_t *k2;
@@ -132,8 +136,7 @@ Workspace carve(const Geometry &G, void *base) {
     W.counts = (int *)take(4 * sizeof(int));
     W.keys[0] = (uint64_t *)take(N * 8);
     W.keys[1] = (uint64_t *)take(N * 8);
-    W.vals[0] = (uint32_t *)take(N * 4);
-    W.vals[1] = (uint32_t *)take(N * 4);
+    W.sa = (uint32_t *)take(N * 4);
     W.rank = (int32_t *)take(N * 4);
     W.lcp = (int32_t *)take(N * 4);
     W.k2 = (uint32_t *)take(N * 4);
@@ -166,12 +169,12 @@ Workspace carve(const Geometry &G, void *base) {
 
 // ---------------------------------------------------------------------------
 // 1a. Round-0 keys: first D0 symbols of the reversed prefix, most significant
-//     first, zero-padded past the start, then min(p+1, D0+1) in the low bits so
-//     that a string that ends sorts before its extensions.
+//     first, zero-padded past the start, then min(p+1, D0+1) so that a string
+//     that ends sorts before its extensions, then the item id in the low bits
+//     (carried through the sort, never sorted on).
 // ---------------------------------------------------------------------------
 __global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
-                             uint64_t *__restrict__ keys, uint32_t *__restrict__ vals,
-                             uint32_t *__restrict__ status) {
+                             uint64_t *__restrict__ keys, uint32_t *__restrict__ status) {
     const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (gi >= G.N) return;
     const int s = (int)(gi / G.n);
@@ -188,8 +191,7 @@ __global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__res
         chars = (chars << G.bps) | (c & symmask);
     }
     if ((uint32_t)a[p] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
-    keys[gi] = (chars << G.abits) | (uint64_t)avail;
-    vals[gi] = (uint32_t)x;
+    keys[gi] = (((chars << G.abits) | (uint64_t)avail) << G.idbits) | (uint64_t)x;
 }
 
 // ---------------------------------------------------------------------------
@@ -234,11 +236,9 @@ radix_scan_kernel(uint32_t *__restrict__ hist, int ntps) {
 // tile; ranks come from warp-private digit counters, so the whole tile needs
 // only three block barriers.
 __global__ void __launch_bounds__(kRadixThreads, 4)
-radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restrict__ vin,
-                     uint64_t *__restrict__ kout, uint32_t *__restrict__ vout, Geometry G, int shift,
+radix_scatter_kernel(const uint64_t *__restrict__ kin, uint64_t *__restrict__ kout, Geometry G, int shift,
                      const uint32_t *__restrict__ hist) {
     __shared__ uint64_t sk[kRadixTile];
-    __shared__ uint32_t sv[kRadixTile];
     __shared__ uint32_t wcnt[kRadixWarps][kRadixBins];   // per-warp digit counts, then per-warp offsets
     __shared__ uint32_t tstart[kRadixBins];
     __shared__ uint32_t gofs[kRadixBins];
@@ -257,7 +257,6 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
     __syncthreads();
 
     uint64_t key[kRadixIPT];
-    uint32_t val[kRadixIPT];
     unsigned peer[kRadixIPT];
     const int wbase = warp * kWarpItems;
     const unsigned lt = lanemask_lt();
@@ -268,7 +267,6 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
         const int i = wbase + u * 32 + lane;
         const bool ok = i < lim;
         key[u] = ok ? kin[base + i] : 0ull;
-        val[u] = ok ? vin[base + i] : 0u;
         const unsigned d = (unsigned)(key[u] >> shift) & (kRadixBins - 1);
         unsigned pm = __ballot_sync(ROSA_FULL_MASK, ok);
 #pragma unroll
@@ -307,7 +305,6 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
         if (ok) {
             const uint32_t pos = wcnt[warp][d] + before;
             sk[pos] = key[u];
-            sv[pos] = val[u];
         }
         __syncwarp();
         if (ok && before == 0) wcnt[warp][d] += __popc(peer[u]);
@@ -319,7 +316,6 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, const uint32_t *__restric
         const int d = (int)((kk >> shift) & (kRadixBins - 1));
         const int64_t dst = seg + gofs[d] + (j - tstart[d]);
         kout[dst] = kk;
-        vout[dst] = sv[j];
     }
 }
 
@@ -339,20 +335,23 @@ __device__ __forceinline__ void push_group(int2 *small, int2 *large, int *counts
     }
 }
 
-__global__ void groups0_kernel(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ sa, Geometry G,
+__global__ void groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geometry G,
                                int32_t *__restrict__ rank, int2 *small, int2 *large, int *counts_next) {
     const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (gi >= G.N) return;
     const int s = (int)(gi / G.n);
     const int j = (int)(gi - (int64_t)s * G.n);
     const int64_t seg = (int64_t)s * G.n;
-    const uint64_t kk = keys[gi];
-    if (j > 0 && keys[gi - 1] == kk) return;   // not a group head
+    const uint64_t idmask = (1ull << G.idbits) - 1ull;
+    const uint64_t full = keys[gi];
+    const uint64_t kk = full >> G.idbits;
+    sa[gi] = (uint32_t)(full & idmask);
+    if (j > 0 && (keys[gi - 1] >> G.idbits) == kk) return;   // not a group head
     int e = j + 1;
-    while (e < G.n && keys[seg + e] == kk) ++e;
-    for (int m = j; m < e; ++m) rank[seg + sa[seg + m]] = j;
+    while (e < G.n && (keys[seg + e] >> G.idbits) == kk) ++e;
+    for (int m = j; m < e; ++m) rank[seg + (keys[seg + m] & idmask)] = j;
     const int size = e - j;
-    if (size > 1 && item_pos(sa[gi], G.T) + 1 > G.D0) push_group(small, large, counts_next, gi, size);
+    if (size > 1 && item_pos((uint32_t)(full & idmask), G.T) + 1 > G.D0) push_group(small, large, counts_next, gi, size);
 }
 
 // ---------------------------------------------------------------------------
@@ -519,7 +518,7 @@ __global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restr
     const int s = (int)(gi / G.n);
     const int j = (int)(gi - (int64_t)s * G.n);
     if (j == 0) { lcp[gi] = 0; return; }
-    const uint64_t k1 = keys[gi - 1], kk2 = keys[gi];
+    const uint64_t k1 = keys[gi - 1] >> G.idbits, kk2 = keys[gi] >> G.idbits;
     const uint64_t amask = (1ull << G.abits) - 1ull;
     const int a1 = (int)(k1 & amask), a2 = (int)(kk2 & amask);
     if (k1 != kk2) {
@@ -1542,7 +1541,7 @@ int match_launch_count(int S, int T, int K, bool same) {
     const Geometry G = make_geometry(S, T, K, 1, same);
     int rounds = 0;
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
-    const int passes = ceil_div(G.keybits, kRadixBits);
+    const int passes = ceil_div(G.keybits - G.idbits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
     // + wavelet (key count when q != k, compaction, one per level) + 6 resolve
     return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 6;
@@ -1566,20 +1565,19 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     const uint8_t *vs = v ? v : k;
 
     // 1a. keys
-    keys0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, W.keys[0], W.vals[0], W.status);
-    // 1b. radix sort over keybits, 8 bits per pass
+    keys0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, W.keys[0], W.status);
+    // 1b. radix sort over the key bits above the item id, 8 bits per pass
     int cur = 0;
     const unsigned tiles = (unsigned)(G.S * G.ntps);
-    for (int shift = 0; shift < G.keybits; shift += kRadixBits) {
+    for (int shift = G.idbits; shift < G.keybits; shift += kRadixBits) {
         radix_hist_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], G, shift, W.hist);
         radix_scan_kernel<<<(unsigned)G.S, kRadixBins, 0, st>>>(W.hist, G.ntps);
-        radix_scatter_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], W.vals[cur], W.keys[cur ^ 1],
-                                                              W.vals[cur ^ 1], G, shift, W.hist);
+        radix_scatter_kernel<<<tiles, kRadixThreads, 0, st>>>(W.keys[cur], W.keys[cur ^ 1], G, shift, W.hist);
         cur ^= 1;
     }
     uint64_t *keys = W.keys[cur];
     uint64_t *scratch = W.keys[cur ^ 1];
-    uint32_t *sa = W.vals[cur];
+    uint32_t *sa = W.sa;
     // 1c. round-0 groups (lists buffer 0)
     groups0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(keys, sa, G, W.rank, W.lists[0][0], W.lists[0][1],
                                                        W.counts);
