@@ -808,33 +808,23 @@ wavelet_level_kernel(Geometry G, int lv, const uint32_t *__restrict__ in, uint32
     // base of each digit's next slot for this warp (advanced after every round)
     int base0 = start[0] + before[0] + wpre[0], base1 = start[1] + before[1] + wpre[1];
     int base2 = start[2] + before[2] + wpre[2], base3 = start[3] + before[3] + wpre[3];
-    // next-level counts: lane k owns (digit k>>3, destination tile k>>2&1, next digit k&3)
-    const int kd = lane >> 3, ks = (lane >> 2) & 1, kn = lane & 3;
-    int kcnt = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const unsigned lo = blo[warp * 8 + u], hi = bhi[warp * 8 + u];
         const int i = warp * 256 + u * 32 + lane;
         const unsigned okm = __ballot_sync(ROSA_FULL_MASK, i < lim);
         const unsigned m0 = okm & ~lo & ~hi, m1 = lo & ~hi, m2 = ~lo & hi, m3 = lo & hi;
-        const int d = (int)((v[u] >> b) & 3u);
-        const int pos = sel4(base0, base1, base2, base3, d) + __popc(sel4u(m0, m1, m2, m3, d) & lt);
-        if (i < lim) dst[pos] = v[u];
-        if (lv + 1 < nlev) {
-            const bool ok = i < lim;
-            const int r0 = sel4(rt0[0], rt0[1], rt0[2], rt0[3], d);
-            const unsigned nd = (v[u] >> (b - 2)) & 3u;
-            const unsigned sb = __ballot_sync(ROSA_FULL_MASK, ok && pos / kWTile > r0);
-            const unsigned nl = __ballot_sync(ROSA_FULL_MASK, ok && (nd & 1u));
-            const unsigned nh = __ballot_sync(ROSA_FULL_MASK, ok && (nd & 2u));
-            const unsigned md = sel4u(m0, m1, m2, m3, kd);
-            const unsigned ms = ks ? sb : ~sb;
-            const unsigned mn = ((kn & 1) ? nl : ~nl) & ((kn & 2) ? nh : ~nh);
-            kcnt += __popc(md & ms & mn);
+        if (i < lim) {
+            const int d = (int)((v[u] >> b) & 3u);
+            const int pos = sel4(base0, base1, base2, base3, d) + __popc(sel4u(m0, m1, m2, m3, d) & lt);
+            dst[pos] = v[u];
+            if (lv + 1 < nlev) {
+                const int r0 = sel4(rt0[0], rt0[1], rt0[2], rt0[3], d);
+                atomicAdd(&nxt[d][pos / kWTile - r0][(v[u] >> (b - 2)) & 3u], 1);
+            }
         }
         base0 += __popc(m0); base1 += __popc(m1); base2 += __popc(m2); base3 += __popc(m3);
     }
-    if (lv + 1 < nlev && kcnt) atomicAdd(&nxt[kd][ks][kn], kcnt);
     // rank directory: 32 words of 64 positions
     if (threadIdx.x < 32) {
         const int k = threadIdx.x;
