@@ -60,7 +60,7 @@ struct Geometry {
     int bps, D0, abits, idbits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
-    int wbits, wlev, ntw, nw;   // wavelet matrix: value bits, base-4 levels, 2048-element tiles, 64-position words
+    int wbits, ntw, nw;      // wavelet matrix: levels, 2048-element tiles and 64-bit words per stream
 };
 
 Geometry make_geometry(int S, int T, int K, int g, bool same) {
@@ -87,7 +87,6 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     int wb = 0;
     while ((1 << wb) < T) ++wb;   // key positions 0..T-1
     G.wbits = wb < 1 ? 1 : wb;
-    G.wlev = (G.wbits + 1) / 2;
     G.ntw = ceil_div(T, 2048);
     G.nw = (T >> 6) + 1;
     return G;
@@ -161,9 +160,9 @@ Workspace carve(const Geometry &G, void *base) {
     W.ktile = (int *)take((size_t)G.S * G.ntps * 4);
     W.wvals[0] = (uint32_t *)take((size_t)G.S * G.T * 4);
     W.wvals[1] = (uint32_t *)take((size_t)G.S * G.T * 4);
-    W.wcnt = (int *)take((size_t)G.wlev * G.S * G.ntw * 4 * 4);
-    W.words = take((size_t)G.S * G.wlev * G.nw * 32);
-    W.wz = (int *)take((size_t)G.S * G.wlev * 4 * 4);
+    W.wcnt = (int *)take((size_t)G.wbits * G.S * G.ntw * 4);
+    W.words = take((size_t)G.S * G.wbits * G.nw * 16);
+    W.wz = (int *)take((size_t)G.S * G.wbits * 4);
     W.bytes = off;
     return W;
 }
@@ -632,16 +631,16 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
 
 // ---------------------------------------------------------------------------
 // 3b. Wavelet matrix over the key positions in rank order, for the query
-//     "largest key position <= X among ranks [lo, hi]" in O(log T).  Base 4:
-//     each level stably partitions the sequence by one 2-bit digit (most
-//     significant first) and stores, per 64 positions, the digit's two bit
-//     planes and the counts of digits 1, 2, 3 before them.
+//     "largest key position <= X among ranks [lo, hi]" in O(log T).  One
+//     stable partition by bit per level, most significant bit first; each
+//     level stores its bits with the count of ones before every 64-bit word.
 // ---------------------------------------------------------------------------
 constexpr int kWTile = 2048;
 
-struct __align__(32) WWord {
-    uint32_t c1, c2, c3, pad;      // digits 1, 2, 3 before this word, in this level's sequence
-    unsigned long long lo, hi;     // digit bit planes of the word's 64 positions
+struct __align__(16) WWord {
+    uint32_t cum;
+    uint32_t pad;
+    unsigned long long bits;
 };
 
 // Keys per 2048-rank tile of the sorted order (q != k only).
@@ -665,26 +664,26 @@ key_tile_count_kernel(Geometry G, const uint32_t *__restrict__ sa, int *__restri
 }
 
 // Level-0 sequence (key positions in rank order), the exclusive key count
-// before every rank (q != k), and the level-0 digit counts per wavelet tile.
+// before every rank (q != k), and the level-0 ones per wavelet tile.
 __global__ void __launch_bounds__(256)
-wavelet_compact_kernel(Geometry G, const uint32_t *__restrict__ sa, const int *__restrict__ ktile,
+wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, const int *__restrict__ ktile,
                        int32_t *__restrict__ kcount, uint32_t *__restrict__ a0, int *__restrict__ wcnt0) {
     __shared__ int wk[8];
     __shared__ int pre_s;
-    __shared__ int dc[2][4];      // this tile's keys touch at most two wavelet tiles
     const int s = blockIdx.x / G.ntps, tt = blockIdx.x - s * G.ntps;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
     const int lim = min(kRadixTile, G.n - tt * kRadixTile);
     const int ntw = ceil_div(G.T, kWTile);
-    const int b0 = 2 * (G.wlev - 1);
     if (threadIdx.x == 0) {
         int p = 0;
         if (G.same) p = tt * kRadixTile;
         else for (int i = 0; i < tt; ++i) p += ktile[(int64_t)s * G.ntps + i];
         pre_s = p;
     }
-    if (threadIdx.x < 8) dc[threadIdx.x >> 2][threadIdx.x & 3] = 0;
+    // this tile's keys take consecutive key indices, so they touch at most two wavelet tiles
+    __shared__ int ones[2];
+    if (threadIdx.x < 2) ones[threadIdx.x] = 0;
     __syncthreads();
     int run = pre_s;
     const int t0 = run / kWTile;
@@ -705,242 +704,173 @@ wavelet_compact_kernel(Geometry G, const uint32_t *__restrict__ sa, const int *_
         if (ok && !G.same) kcount[base + i] = kidx;
         if (key) {
             a0[(int64_t)s * G.T + kidx] = x;
-            atomicAdd(&dc[kidx / kWTile - t0][(x >> b0) & 3u], 1);
+            if ((x >> (nbits - 1)) & 1u) atomicAdd(&ones[kidx / kWTile - t0], 1);
         }
         run += rtot;
         __syncthreads();
     }
-    if (threadIdx.x < 8) {
-        const int side = threadIdx.x >> 2, d = threadIdx.x & 3;
-        const int c = dc[side][d];
-        if (c) atomicAdd(&wcnt0[(((int64_t)s * ntw) + t0 + side) * 4 + d], c);
-    }
+    if (threadIdx.x < 2 && ones[threadIdx.x]) atomicAdd(&wcnt0[(int64_t)s * ntw + t0 + threadIdx.x], ones[threadIdx.x]);
 }
 
-__device__ __forceinline__ int sel4(int a0, int a1, int a2, int a3, int d) {
-    return d == 0 ? a0 : (d == 1 ? a1 : (d == 2 ? a2 : a3));
-}
-__device__ __forceinline__ unsigned sel4u(unsigned a0, unsigned a1, unsigned a2, unsigned a3, int d) {
-    return d == 0 ? a0 : (d == 1 ? a1 : (d == 2 ? a2 : a3));
-}
-
-// One level: stable 4-way partition of a 2048-element tile by its digit.
-// Warp w owns elements [256w, 256w + 256); digit offsets come from the
-// stream's per-tile counts, the warps' counts and ballot ranks.
-__global__ void __launch_bounds__(256, 4)
-wavelet_level_kernel(Geometry G, int lv, const uint32_t *__restrict__ in, uint32_t *__restrict__ out,
+__global__ void __launch_bounds__(256)
+wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__ in, uint32_t *__restrict__ out,
                      int *__restrict__ wcnt, WWord *__restrict__ words, int *__restrict__ wz) {
-    __shared__ uint32_t blo[kWTile / 32], bhi[kWTile / 32];
-    __shared__ int wdc[8][4];
-    __shared__ int red[8][8];
-    __shared__ int nxt[4][2][4];  // digit run, destination tile offset, next digit
-    const int nlev = G.wlev;
+    // warp w owns elements [256w, 256w + 256) of the tile: its ones count
+    // gives the warp's offsets, so the tile needs only two block barriers
+    __shared__ uint32_t ballots[kWTile / 32];
+    __shared__ int wones[8];
+    __shared__ int red_a[8], red_t[8];
+    __shared__ int nxt[4];
     const int ntw = ceil_div(G.T, kWTile), nw = (G.T >> 6) + 1;
     const int s = blockIdx.x / ntw, tt = blockIdx.x - s * ntw;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = 2 * (nlev - 1 - lv);
-    const int *cnt = wcnt + ((int64_t)lv * G.S + s) * ntw * 4;
-    // per digit: count in earlier tiles (before) and in the whole stream (total)
-    int bf[4] = {0, 0, 0, 0}, tot[4] = {0, 0, 0, 0};
+    const int b = nbits - 1 - lv;
+    const int *cnt = wcnt + ((int64_t)lv * G.S + s) * ntw;
+    int a = 0, tot = 0;
     for (int i = threadIdx.x; i < ntw; i += 256) {
-#pragma unroll
-        for (int d = 0; d < 4; ++d) {
-            const int c = cnt[i * 4 + d];
-            tot[d] += c;
-            if (i < tt) bf[d] += c;
-        }
+        const int c = cnt[i];
+        tot += c;
+        if (i < tt) a += c;
     }
 #pragma unroll
-    for (int d = 0; d < 4; ++d) {
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            bf[d] += __shfl_xor_sync(ROSA_FULL_MASK, bf[d], o);
-            tot[d] += __shfl_xor_sync(ROSA_FULL_MASK, tot[d], o);
-        }
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int d = 0; d < 4; ++d) { red[warp][d] = bf[d]; red[warp][4 + d] = tot[d]; }
+    for (int o = 16; o >= 1; o >>= 1) {
+        a += __shfl_xor_sync(ROSA_FULL_MASK, a, o);
+        tot += __shfl_xor_sync(ROSA_FULL_MASK, tot, o);
     }
     const int lim = min(kWTile, G.T - tt * kWTile);
     const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
     uint32_t v[8];
-    int wc0 = 0, wc1 = 0, wc2 = 0, wc3 = 0;
+    unsigned bal[8];
+    int mine = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const int i = warp * 256 + u * 32 + lane;
         const bool ok = i < lim;
         v[u] = ok ? src[i] : 0u;
-        const unsigned d = (v[u] >> b) & 3u;
-        const unsigned okm = __ballot_sync(ROSA_FULL_MASK, ok);
-        const unsigned lo = __ballot_sync(ROSA_FULL_MASK, ok && (d & 1u));
-        const unsigned hi = __ballot_sync(ROSA_FULL_MASK, ok && (d & 2u));
-        wc0 += __popc(okm & ~lo & ~hi);
-        wc1 += __popc(lo & ~hi);
-        wc2 += __popc(~lo & hi);
-        wc3 += __popc(lo & hi);
-        if (lane == 0) { blo[warp * 8 + u] = lo; bhi[warp * 8 + u] = hi; }
+        bal[u] = __ballot_sync(ROSA_FULL_MASK, ok && ((v[u] >> b) & 1u));
+        mine += __popc(bal[u]);
     }
-    if (lane == 0) { wdc[warp][0] = wc0; wdc[warp][1] = wc1; wdc[warp][2] = wc2; wdc[warp][3] = wc3; }
-    if (threadIdx.x < 32) nxt[threadIdx.x >> 3][(threadIdx.x >> 2) & 1][threadIdx.x & 3] = 0;
+    if (lane == 0) {
+        red_a[warp] = a;
+        red_t[warp] = tot;
+        wones[warp] = mine;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ballots[warp * 8 + u] = bal[u];
+    }
+    if (threadIdx.x < 4) nxt[threadIdx.x] = 0;
     __syncthreads();
-    int before[4], total[4], start[4], wpre[4], tdc[4];
+    int ones_before = 0, total_ones = 0, wpre = 0;
 #pragma unroll
-    for (int d = 0; d < 4; ++d) {
-        before[d] = 0; total[d] = 0; wpre[d] = 0; tdc[d] = 0;
-        for (int w2 = 0; w2 < 8; ++w2) {
-            before[d] += red[w2][d];
-            total[d] += red[w2][4 + d];
-            if (w2 < warp) wpre[d] += wdc[w2][d];
-            tdc[d] += wdc[w2][d];
-        }
+    for (int w2 = 0; w2 < 8; ++w2) {
+        ones_before += red_a[w2];
+        total_ones += red_t[w2];
+        if (w2 < warp) wpre += wones[w2];
     }
-    start[0] = 0;
-    start[1] = total[0];
-    start[2] = total[0] + total[1];
-    start[3] = total[0] + total[1] + total[2];
-    // first destination tile of each digit's run from this tile
-    int rt0[4];
-#pragma unroll
-    for (int d = 0; d < 4; ++d) rt0[d] = (start[d] + before[d]) / kWTile;
+    const int Z = G.T - total_ones;
+    const int zeros_before = tt * kWTile - ones_before;
+    // zeros of this tile land in one contiguous range and ones in another, so
+    // the next level's per-tile counts touch at most four tiles
+    const int zr0 = zeros_before / kWTile, or0 = (Z + ones_before) / kWTile;
     uint32_t *dst = out + (int64_t)s * G.T;
-    const unsigned lt = lanemask_lt();
-    // base of each digit's next slot for this warp (advanced after every round)
-    int base0 = start[0] + before[0] + wpre[0], base1 = start[1] + before[1] + wpre[1];
-    int base2 = start[2] + before[2] + wpre[2], base3 = start[3] + before[3] + wpre[3];
+    int run = wpre;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const unsigned lo = blo[warp * 8 + u], hi = bhi[warp * 8 + u];
         const int i = warp * 256 + u * 32 + lane;
-        const unsigned okm = __ballot_sync(ROSA_FULL_MASK, i < lim);
-        const unsigned m0 = okm & ~lo & ~hi, m1 = lo & ~hi, m2 = ~lo & hi, m3 = lo & hi;
+        const int bit = (bal[u] >> lane) & 1;
+        const int lo1 = run + __popc(bal[u] & lanemask_lt());
         if (i < lim) {
-            const int d = (int)((v[u] >> b) & 3u);
-            const int pos = sel4(base0, base1, base2, base3, d) + __popc(sel4u(m0, m1, m2, m3, d) & lt);
-            dst[pos] = v[u];
-            if (lv + 1 < nlev) {
-                const int r0 = sel4(rt0[0], rt0[1], rt0[2], rt0[3], d);
-                atomicAdd(&nxt[d][pos / kWTile - r0][(v[u] >> (b - 2)) & 3u], 1);
+            const int d = bit ? Z + ones_before + lo1 : zeros_before + (i - lo1);
+            dst[d] = v[u];
+            if (lv + 1 < nbits && ((v[u] >> (b - 1)) & 1u)) {
+                const int dt = d / kWTile;
+                atomicAdd(&nxt[bit ? 2 + (dt - or0) : (dt - zr0)], 1);
             }
         }
-        base0 += __popc(m0); base1 += __popc(m1); base2 += __popc(m2); base3 += __popc(m3);
+        run += __popc(bal[u]);
     }
-    // rank directory: 32 words of 64 positions
     if (threadIdx.x < 32) {
         const int k = threadIdx.x;
-        const unsigned long long wl = (unsigned long long)blo[2 * k] | ((unsigned long long)blo[2 * k + 1] << 32);
-        const unsigned long long wh = (unsigned long long)bhi[2 * k] | ((unsigned long long)bhi[2 * k + 1] << 32);
-        int c1 = __popcll(wl & ~wh), c2 = __popcll(~wl & wh), c3 = __popcll(wl & wh);
-        int i1 = c1, i2 = c2, i3 = c3;
+        const unsigned long long bits =
+            (unsigned long long)ballots[2 * k] | ((unsigned long long)ballots[2 * k + 1] << 32);
+        const int pc = __popcll(bits);
+        int incl = pc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y1 = __shfl_up_sync(ROSA_FULL_MASK, i1, o);
-            const int y2 = __shfl_up_sync(ROSA_FULL_MASK, i2, o);
-            const int y3 = __shfl_up_sync(ROSA_FULL_MASK, i3, o);
-            if (lane >= o) { i1 += y1; i2 += y2; i3 += y3; }
+            const int y = __shfl_up_sync(ROSA_FULL_MASK, incl, o);
+            if (lane >= o) incl += y;
         }
         if (k * 64 < lim) {
             WWord wd;
-            wd.c1 = (uint32_t)(before[1] + i1 - c1);
-            wd.c2 = (uint32_t)(before[2] + i2 - c2);
-            wd.c3 = (uint32_t)(before[3] + i3 - c3);
+            wd.cum = (uint32_t)(ones_before + incl - pc);
             wd.pad = 0;
-            wd.lo = wl;
-            wd.hi = wh;
-            words[((int64_t)s * nlev + lv) * nw + tt * 32 + k] = wd;
+            wd.bits = bits;
+            words[((int64_t)s * nbits + lv) * nw + tt * 32 + k] = wd;
         }
     }
     __syncthreads();
-    if (lv + 1 < nlev && threadIdx.x < 32) {
-        const int d = threadIdx.x >> 3, side = (threadIdx.x >> 2) & 1, nd = threadIdx.x & 3;
-        const int c = nxt[d][side][nd];
-        const int r0 = sel4(rt0[0], rt0[1], rt0[2], rt0[3], d);
-        if (c) atomicAdd(&wcnt[(((int64_t)(lv + 1) * G.S + s) * ntw + r0 + side) * 4 + nd], c);
+    if (lv + 1 < nbits && threadIdx.x < 4) {
+        const int c = nxt[threadIdx.x];
+        const int dt = threadIdx.x < 2 ? zr0 + threadIdx.x : or0 + threadIdx.x - 2;
+        if (c) atomicAdd(&wcnt[((int64_t)(lv + 1) * G.S + s) * ntw + dt], c);
     }
     if (threadIdx.x == 0) {
         if (tt == ntw - 1 && (G.T & 63) == 0) {
             WWord wd;
-            wd.c1 = (uint32_t)total[1];
-            wd.c2 = (uint32_t)total[2];
-            wd.c3 = (uint32_t)total[3];
+            wd.cum = (uint32_t)total_ones;
             wd.pad = 0;
-            wd.lo = 0ull;
-            wd.hi = 0ull;
-            words[((int64_t)s * nlev + lv) * nw + (G.T >> 6)] = wd;
+            wd.bits = 0ull;
+            words[((int64_t)s * nbits + lv) * nw + (G.T >> 6)] = wd;
         }
-        if (tt == 0) {
-#pragma unroll
-            for (int d = 0; d < 4; ++d) wz[((int64_t)s * nlev + lv) * 4 + d] = start[d];
-        }
+        if (tt == 0) wz[(int64_t)s * nbits + lv] = Z;
     }
-    (void)tdc;
 }
 
-// Counts of digits 0..3 before position i of a level's sequence.
-__device__ __forceinline__ void wrank4(const WWord *W, int i, int r[4]) {
-    const WWord *w = W + (i >> 6);
-    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(w));
-    const uint4 c = __ldg(reinterpret_cast<const uint4 *>(w) + 1);
+__device__ __forceinline__ int wrank1(const WWord *W, int i) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(W + (i >> 6)));
+    const unsigned long long bits = ((unsigned long long)raw.w << 32) | raw.z;
     const unsigned long long mask = (i & 63) ? ((1ull << (i & 63)) - 1ull) : 0ull;
-    const unsigned long long lo = (((unsigned long long)c.y << 32) | c.x) & mask;
-    const unsigned long long hi = (((unsigned long long)c.w << 32) | c.z) & mask;
-    r[1] = (int)a.x + __popcll(lo & ~hi);
-    r[2] = (int)a.y + __popcll(~lo & hi);
-    r[3] = (int)a.z + __popcll(lo & hi);
-    r[0] = i - r[1] - r[2] - r[3];
+    return (int)raw.x + __popcll(bits & mask);
 }
 
 // Largest value <= X in positions [l, r) of the level-0 sequence, or -1.
-// C holds, per level, where each digit's elements start in the next level.
-__device__ int wavelet_max_le(const WWord *W, const int *C, int nlev, int nw, int l, int r, int X) {
+__device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, int l, int r, int X) {
     if (l >= r || X < 0) return -1;
-    const int top = (1 << (2 * nlev)) - 1;
+    const int top = (1 << nbits) - 1;
     if (X > top) X = top;
-    int alt_lv = -1, alt_d = 0, alt_l = 0, alt_r = 0;
+    int alt_lv = -1, alt_l = 0, alt_r = 0;
     bool alive = true;
-    for (int lv = 0; lv < nlev; ++lv) {
-        const int b = 2 * (nlev - 1 - lv);
-        const int x = (X >> b) & 3;
-        int rl[4], rr[4];
-        wrank4(W + (int64_t)lv * nw, l, rl);
-        wrank4(W + (int64_t)lv * nw, r, rr);
-        bool got = false;
-#pragma unroll
-        for (int d = 3; d >= 0; --d) {
-            if (!got && d < x && rr[d] > rl[d]) {
-                got = true;
-                alt_lv = lv; alt_d = d; alt_l = C[lv * 4 + d] + rl[d]; alt_r = C[lv * 4 + d] + rr[d];
-            }
+    for (int lv = 0; lv < nbits; ++lv) {
+        const int b = nbits - 1 - lv;
+        const WWord *Wl = W + (int64_t)lv * nw;
+        const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
+        const int zl = l - ol, zr = r - orr;
+        if ((X >> b) & 1) {
+            if (zr > zl) { alt_lv = lv; alt_l = zl; alt_r = zr; }
+            l = Z[lv] + ol;
+            r = Z[lv] + orr;
+        } else {
+            l = zl;
+            r = zr;
         }
-        const int cx = C[lv * 4 + x];
-        l = cx + sel4(rl[0], rl[1], rl[2], rl[3], x);
-        r = cx + sel4(rr[0], rr[1], rr[2], rr[3], x);
         if (l >= r) { alive = false; break; }
     }
     if (alive) return X;
     if (alt_lv < 0) return -1;
-    const int ba = 2 * (nlev - 1 - alt_lv);
-    int val = ((X >> (ba + 2)) << (ba + 2)) | (alt_d << ba);
+    int val = (X >> (nbits - alt_lv)) << (nbits - alt_lv);
     l = alt_l;
     r = alt_r;
-    for (int lv = alt_lv + 1; lv < nlev; ++lv) {
-        const int b = 2 * (nlev - 1 - lv);
-        int rl[4], rr[4];
-        wrank4(W + (int64_t)lv * nw, l, rl);
-        wrank4(W + (int64_t)lv * nw, r, rr);
-        bool got = false;
-        int nl = l, nr = r;
-#pragma unroll
-        for (int d = 3; d >= 0; --d) {
-            if (!got && rr[d] > rl[d]) {
-                got = true;
-                val |= d << b;
-                nl = C[lv * 4 + d] + rl[d];
-                nr = C[lv * 4 + d] + rr[d];
-            }
+    for (int lv = alt_lv + 1; lv < nbits; ++lv) {
+        const int b = nbits - 1 - lv;
+        const WWord *Wl = W + (int64_t)lv * nw;
+        const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
+        if (orr > ol) {
+            val |= 1 << b;
+            l = Z[lv] + ol;
+            r = Z[lv] + orr;
+        } else {
+            l -= ol;
+            r -= orr;
         }
-        l = nl;
-        r = nr;
     }
     return val;
 }
@@ -970,7 +900,7 @@ struct StreamView {
     const int32_t *kcount;
     const WWord *W;
     const int *Z;
-    int n, T, nb1, nb2, nlev, nw;
+    int n, T, nb1, nb2, nbits, nw;
     bool same;
 };
 
@@ -987,7 +917,7 @@ struct ResolveArgs {
     const int32_t *lcp, *mp1, *em1, *ein1, *mp2, *em2, *ein2, *kcount;
     const WWord *words;
     const int *wz;
-    int nlev;
+    int nbits;
 };
 
 __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const ResolveArgs &A) {
@@ -996,8 +926,8 @@ __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const 
     return StreamView{A.sa + seg, A.lcp + seg, A.mp1 + (int64_t)s * G.nb1, A.em1 + (int64_t)s * G.nb1,
                       A.ein1 + (int64_t)s * G.nb1, A.mp2 + (int64_t)s * G.nb2, A.em2 + (int64_t)s * G.nb2,
                       A.ein2 + (int64_t)s * G.nb2, A.kcount ? A.kcount + seg : nullptr,
-                      A.words + (int64_t)s * A.nlev * nw, A.wz + (int64_t)s * A.nlev * 4, G.n, G.T, G.nb1, G.nb2,
-                      A.nlev, nw, G.same};
+                      A.words + (int64_t)s * A.nbits * nw, A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, G.nb2,
+                      A.nbits, nw, G.same};
 }
 
 __device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *vsym, int s, int t, int L, int ib,
@@ -1580,8 +1510,8 @@ __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *_
         const int s = (int)(o / G.T);
         const int t = (int)(o - (int64_t)s * G.T);
         const int klo = end_idx[o], khi = sym[o];
-        const WWord *W = A.words + (int64_t)s * A.nlev * nw;
-        const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nlev * 4, A.nlev, nw, klo, khi, t - G.g);
+        const WWord *W = A.words + (int64_t)s * A.nbits * nw;
+        const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nbits, A.nbits, nw, klo, khi, t - G.g);
         end_idx[o] = ib;
         sym[o] = ib >= 0 ? (int32_t)vsym[(int64_t)s * G.T + ib + 1] : -1;
     }
@@ -1614,7 +1544,7 @@ int match_launch_count(int S, int T, int K, bool same) {
     const int passes = ceil_div(G.keybits - G.idbits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
     // + wavelet (key count when q != k, compaction, one per level) + 6 resolve
-    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wlev + 6;
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 6;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1671,17 +1601,18 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
                                                            W.minpos2, W.emin2, W.ein2);
     // 3b. wavelet matrix over key positions in rank order
-    if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wlev * G.S * G.ntw * 4 * 4, st)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wbits * G.S * G.ntw * 4, st)) != cudaSuccess) return err;
     if (!G.same) key_tile_count_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile);
-    wavelet_compact_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile, W.kcount, W.wvals[0], W.wcnt);
+    wavelet_compact_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, G.wbits, sa, W.ktile, W.kcount, W.wvals[0],
+                                                                      W.wcnt);
     WWord *words = static_cast<WWord *>(W.words);
-    for (int lv = 0; lv < G.wlev; ++lv)
-        wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, lv, W.wvals[lv & 1], W.wvals[(lv + 1) & 1],
-                                                                       W.wcnt, words, W.wz);
+    for (int lv = 0; lv < G.wbits; ++lv)
+        wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, G.wbits, lv, W.wvals[lv & 1],
+                                                                       W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
     // 3c. resolve: thread per query, then warp per query for the long scans
     if ((err = tile_smem_optin()) != cudaSuccess) return err;
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.same ? nullptr : W.kcount,
-                  words, W.wz, G.wlev};
+                  words, W.wz, G.wbits};
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
     int *hardb_count = W.counts + 7;
