@@ -133,7 +133,7 @@ Workspace carve(const Geometry &G, void *base) {
     const size_t N = (size_t)G.N;
     const size_t list_cap = N / 2 + 1;
     W.status = (uint32_t *)take(256);
-    W.counts = (int *)take(4 * sizeof(int));
+    W.counts = (int *)take(64 * sizeof(int));   // list, hard-query and tie counters (cleared with status)
     W.keys[0] = (uint64_t *)take(N * 8);
     W.keys[1] = (uint64_t *)take(N * 8);
     W.sa = (uint32_t *)take(N * 4);
@@ -321,37 +321,169 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, uint64_t *__restrict__ ko
 
 // ---------------------------------------------------------------------------
 // 1c. Groups after round 0: rank = position of the group head; groups of more
-//     than one incomplete string (p + 1 > D0) go to the unresolved lists.
+//     than one incomplete string (p + 1 > D0) go to the unresolved lists
+//     (small: up to kSmallGroup members, large: more).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ? (int)x : (int)x - T; }
 
-__device__ __forceinline__ void push_group(int2 *small, int2 *large, int *counts_next, int64_t start, int size) {
-    if (size <= kSmallGroup) {
-        const int i = atomicAdd(&counts_next[0], 1);
-        small[i] = make_int2((int)start, size);
-    } else {
-        const int i = atomicAdd(&counts_next[1], 1);
-        large[i] = make_int2((int)start, size);
-    }
-}
+// One CTA per 2048-item tile of a stream's round-0 order; thread t owns
+// items [8t, 8t+8).  The tile passes through shared memory (9 words per
+// thread, conflict-free) so that global loads and stores stay coalesced.
+// Group heads (key differs from the previous item) come from a block-wide
+// max-scan; a group running in from the previous tile is found by a warp
+// search.  The adjacent LCP is written here wherever it cannot change later:
+// across different round-0 keys (it depends on the keys only) and inside
+// groups of identical complete strings.  Positions inside unresolved groups
+// are listed (-1 in lcp); their LCP is taken after doubling.
+constexpr int kG0Stride = 9;
+__device__ __forceinline__ int g0_slot(int i) { return (i >> 3) * kG0Stride + (i & 7); }
 
-__global__ void groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geometry G,
-                               int32_t *__restrict__ rank, int2 *small, int2 *large, int *counts_next) {
-    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (gi >= G.N) return;
-    const int s = (int)(gi / G.n);
-    const int j = (int)(gi - (int64_t)s * G.n);
+__global__ void __launch_bounds__(256)
+groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geometry G, int32_t *__restrict__ rank,
+               int32_t *__restrict__ lcp, int2 *small, int2 *large, int *counts_next, int32_t *__restrict__ ties,
+               int *tie_count) {
+    __shared__ uint64_t sk[256 * kG0Stride];
+    __shared__ int32_t so[256 * kG0Stride];
+    __shared__ int wmax[8];
+    __shared__ uint32_t scan_ws[9];
+    __shared__ int list_base[3];
+    __shared__ int look;
+    const int s = blockIdx.x / G.ntps, tt = blockIdx.x - s * G.ntps;
     const int64_t seg = (int64_t)s * G.n;
+    const int j0 = tt * kRadixTile;
+    const int lim = min(kRadixTile, G.n - j0);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint64_t idmask = (1ull << G.idbits) - 1ull;
-    const uint64_t full = keys[gi];
-    const uint64_t kk = full >> G.idbits;
-    sa[gi] = (uint32_t)(full & idmask);
-    if (j > 0 && (keys[gi - 1] >> G.idbits) == kk) return;   // not a group head
-    int e = j + 1;
-    while (e < G.n && (keys[seg + e] >> G.idbits) == kk) ++e;
-    for (int m = j; m < e; ++m) rank[seg + (keys[seg + m] & idmask)] = j;
-    const int size = e - j;
-    if (size > 1 && item_pos((uint32_t)(full & idmask), G.T) + 1 > G.D0) push_group(small, large, counts_next, gi, size);
+    const uint64_t amask = (1ull << G.abits) - 1ull;
+    const int base = threadIdx.x * 8;
+    for (int i = threadIdx.x; i < lim; i += 256) sk[g0_slot(i)] = keys[seg + j0 + i];
+    if (warp == 0) {
+        // Head of the group that runs into this tile from the previous one.
+        // Keys are sorted, so the group is the run of keys equal to keys[j0]:
+        // its head is a lower bound, found 32 positions per step.
+        int h = -1;
+        if (j0 > 0 && lim > 0) {
+            const uint64_t kk = keys[seg + j0] >> G.idbits;
+            // backward probes j0-1 .. j0-32 first: most runs are short
+            const int p0 = j0 - 1 - lane;
+            const unsigned ne = ~__ballot_sync(ROSA_FULL_MASK, p0 >= 0 && (keys[seg + p0] >> G.idbits) == kk);
+            int lo, hi;                            // keys[hi] == kk; the head lies in [lo, hi]
+            if (ne) lo = hi = j0 - (__ffs(ne) - 1);
+            else { lo = 0; hi = j0 - 32; }
+            while (lo < hi) {
+                const int64_t span = hi - lo;
+                const int p = lo + (int)(span * lane / 32);
+                const unsigned b = __ballot_sync(ROSA_FULL_MASK, (keys[seg + p] >> G.idbits) == kk);
+                if (b & 1u) { hi = lo; break; }
+                const int f = b ? __ffs(b) - 1 : 32;   // first probe inside the run
+                const int nlo = lo + (int)(span * (f - 1) / 32) + 1;
+                if (f < 32) hi = lo + (int)(span * f / 32);
+                lo = nlo;
+            }
+            if (hi < j0) h = hi;
+        }
+        look = h;
+    }
+    __syncthreads();
+    uint64_t kv[8];
+    uint32_t id[8];
+    int hp = -1;
+    unsigned headbits = 0;
+    uint64_t prev = ~0ull;
+    if (base < lim && j0 + base > 0) prev = (base > 0 ? sk[g0_slot(base - 1)] : keys[seg + j0 - 1]) >> G.idbits;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int jl = base + e, j = j0 + jl;
+        const bool ok = jl < lim;
+        const uint64_t full = ok ? sk[g0_slot(jl)] : 0ull;
+        const uint64_t k = full >> G.idbits;
+        kv[e] = k;
+        id[e] = (uint32_t)(full & idmask);
+        if (ok) {
+            const bool head = (j == 0) || k != prev;
+            if (head) { hp = j; headbits |= 1u << e; }
+            int l = -1;   // -1: decided after doubling
+            const int a2 = (int)(k & amask);
+            if (j == 0) {
+                l = 0;
+            } else if (head) {
+                const int a1 = (int)(prev & amask);
+                const uint64_t x = (prev >> G.abits) ^ (k >> G.abits);
+                int diff = G.D0;
+                if (x) diff = (__clzll((long long)x) - (64 - G.D0 * G.bps)) / G.bps;
+                l = min(diff, min(min(a1, G.D0), min(a2, G.D0)));
+            } else if (a2 <= G.D0) {
+                l = a2;   // identical complete strings
+            }
+            so[g0_slot(jl)] = l;
+            prev = k;
+        }
+    }
+    // first key after this thread's chunk, for end-of-group tests
+    uint64_t nk = ~0ull;
+    if (base + 8 < lim) nk = sk[g0_slot(base + 8)] >> G.idbits;
+    else if (base + 8 == lim && j0 + lim < G.n) nk = keys[seg + j0 + lim] >> G.idbits;
+    // exclusive max-scan of the threads' last head positions
+    int incl = hp;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(ROSA_FULL_MASK, incl, o);
+        if (lane >= o) incl = max(incl, y);
+    }
+    if (lane == 31) wmax[warp] = incl;
+    __syncthreads();
+    for (int i = threadIdx.x; i < lim; i += 256) lcp[seg + j0 + i] = so[g0_slot(i)];
+    int carry = look;
+    for (int w2 = 0; w2 < warp; ++w2) carry = max(carry, wmax[w2]);
+    const int excl = __shfl_up_sync(ROSA_FULL_MASK, incl, 1);
+    if (lane > 0) carry = max(carry, excl);
+    __syncthreads();   // so[] is reused for the item ids
+    // Pass 1: ranks, and which items end a group to refine or are ties.
+    unsigned tiebits = 0, smallbits = 0, largebits = 0;
+    int h = carry;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int jl = base + e, j = j0 + jl;
+        const bool head = (headbits >> e) & 1u;
+        if (head) h = j;
+        if (jl < lim) {
+            so[g0_slot(jl)] = (int32_t)id[e];
+            rank[seg + id[e]] = h;
+            const uint64_t next = e < 7 ? (jl + 1 < lim ? kv[e + 1] : ~0ull) : nk;
+            const bool last = j + 1 >= G.n || next != kv[e];
+            const bool incomplete = (int)(kv[e] & amask) > G.D0;
+            if (last && j > h && incomplete) {
+                if (j - h + 1 <= kSmallGroup) smallbits |= 1u << e;
+                else largebits |= 1u << e;
+            }
+            if (!head && incomplete) tiebits |= 1u << e;
+        }
+    }
+    // Pass 2: one atomic per list per CTA.  Counts share a word: ties <= 2048
+    // (12 bits), group ends <= 1024 (11 bits: a refined group has two members
+    // in the tile), ends of groups over 32 members <= 63 (9 bits).
+    const uint32_t packed = __popc(tiebits) | (__popc(smallbits) << 12) | (__popc(largebits) << 23);
+    uint32_t total;
+    const uint32_t ex = block_exclusive_scan<256>(packed, scan_ws, &total);
+    if (threadIdx.x == 0) {
+        const uint32_t nt = total & 4095u, ns = (total >> 12) & 2047u, nl = total >> 23;
+        list_base[0] = nt ? atomicAdd(tie_count, (int)nt) : 0;
+        list_base[1] = ns ? atomicAdd(&counts_next[0], (int)ns) : 0;
+        list_base[2] = nl ? atomicAdd(&counts_next[1], (int)nl) : 0;
+    }
+    __syncthreads();
+    int it = list_base[0] + (int)(ex & 4095u), is = list_base[1] + (int)((ex >> 12) & 2047u),
+        il = list_base[2] + (int)(ex >> 23);
+    h = carry;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int j = j0 + base + e;
+        if ((headbits >> e) & 1u) h = j;
+        if ((tiebits >> e) & 1u) ties[it++] = (int32_t)(seg + j);
+        if ((smallbits >> e) & 1u) small[is++] = make_int2((int)(seg + h), j - h + 1);
+        if ((largebits >> e) & 1u) large[il++] = make_int2((int)(seg + h), j - h + 1);
+    }
+    for (int i = threadIdx.x; i < lim; i += 256) sa[seg + j0 + i] = (uint32_t)so[g0_slot(i)];
 }
 
 // ---------------------------------------------------------------------------
@@ -447,30 +579,52 @@ dbl_sort_large_kernel(const int2 *__restrict__ large, const int *__restrict__ co
 }
 
 // Split sorted groups at k2 changes.  New group id = local head position;
-// new groups of more than one incomplete string (p + 1 > 2h) go on.
+// new groups of more than one incomplete string (p + 1 > 2h) go on.  List
+// appends take one atomic per warp (per list), not one per group.
 __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
                                    const int *__restrict__ counts, Geometry G, int64_t h2,
                                    const uint32_t *__restrict__ sa, const uint32_t *__restrict__ k2,
                                    int32_t *__restrict__ rank, int2 *nsmall, int2 *nlarge, int *counts_next) {
     const int ns = counts[0], nl = counts[1];
+    const int lane = threadIdx.x & 31;
     const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t nth = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t gidx = tid; gidx < ns; gidx += nth) {
-        const int2 gr = small[gidx];
+    // Small groups, one per thread; the loop runs warp-uniformly.  A group of
+    // at most 32 only splits into small groups.
+    for (int64_t gb = tid - lane; gb < ns; gb += nth) {
+        const int64_t gidx = gb + lane;
+        const int2 gr = gidx < ns ? small[gidx] : make_int2(0, 0);
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
         const int jstart = (int)(gr.x - seg);
-        int head = 0;
+        int head = 0, npush = 0;
         for (int m = 0; m < gr.y; ++m) {
             const uint32_t kk = k2[gr.x + m];
             if (m > 0 && kk != k2[gr.x + m - 1]) head = m;
             const uint32_t x = sa[gr.x + m];
             rank[seg + x] = jstart + head;
             const bool last = (m == gr.y - 1) || (k2[gr.x + m + 1] != kk);
-            if (last && m > head && (int64_t)item_pos(x, G.T) + 1 > h2)
-                push_group(nsmall, nlarge, counts_next, gr.x + head, m - head + 1);
+            if (last && m > head && (int64_t)item_pos(x, G.T) + 1 > h2) ++npush;
+        }
+        int incl = npush;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(ROSA_FULL_MASK, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int wbase = 0;
+        if (lane == 31 && incl) wbase = atomicAdd(&counts_next[0], incl);
+        int slot = __shfl_sync(ROSA_FULL_MASK, wbase, 31) + incl - npush;
+        if (npush) {
+            head = 0;
+            for (int m = 0; m < gr.y; ++m) {
+                const uint32_t kk = k2[gr.x + m];
+                if (m > 0 && kk != k2[gr.x + m - 1]) head = m;
+                const bool last = (m == gr.y - 1) || (k2[gr.x + m + 1] != kk);
+                if (last && m > head && (int64_t)item_pos(sa[gr.x + m], G.T) + 1 > h2)
+                    nsmall[slot++] = make_int2(gr.x + head, m - head + 1);
+            }
         }
     }
-    const int lane = threadIdx.x & 31;
     for (int64_t gidx = tid >> 5; gidx < nl; gidx += nth >> 5) {
         const int2 gr = large[gidx];
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
@@ -488,15 +642,28 @@ __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *_
                 if (lane >= o) hp = max(hp, y);
             }
             const int gid = max(hp, carry);
+            bool push = false;
+            int size = 0;
             if (ok) {
                 const uint32_t x = sa[gr.x + m];
                 rank[seg + x] = gid;
                 const bool last = (m == gr.y - 1) || (k2[gr.x + m + 1] != kk);
-                if (last) {
-                    const int size = jstart + m - gid + 1;
-                    if (size > 1 && (int64_t)item_pos(x, G.T) + 1 > h2)
-                        push_group(nsmall, nlarge, counts_next, seg + gid, size);
-                }
+                size = jstart + m - gid + 1;
+                push = last && size > 1 && (int64_t)item_pos(x, G.T) + 1 > h2;
+            }
+            const unsigned ms = __ballot_sync(ROSA_FULL_MASK, push && size <= kSmallGroup);
+            const unsigned ml = __ballot_sync(ROSA_FULL_MASK, push && size > kSmallGroup);
+            int bs = 0, bl = 0;
+            if (lane == 0) {
+                if (ms) bs = atomicAdd(&counts_next[0], __popc(ms));
+                if (ml) bl = atomicAdd(&counts_next[1], __popc(ml));
+            }
+            bs = __shfl_sync(ROSA_FULL_MASK, bs, 0);
+            bl = __shfl_sync(ROSA_FULL_MASK, bl, 0);
+            if (push) {
+                const int2 ng = make_int2((int)(seg + gid), size);
+                if (size <= kSmallGroup) nsmall[bs + __popc(ms & lanemask_lt())] = ng;
+                else nlarge[bl + __popc(ml & lanemask_lt())] = ng;
             }
             carry = __shfl_sync(ROSA_FULL_MASK, gid, 31);
         }
@@ -504,41 +671,33 @@ __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *_
 }
 
 // ---------------------------------------------------------------------------
-// 2. Adjacent LCP of the final order.  Ties never leave a round-0 key group,
-//    so keys[] (sorted in round 0) still holds the key of the item at each
-//    rank.
+// 2. Adjacent LCP of the final order.  groups0 already wrote every position
+//    whose neighbours differ in their round-0 keys; the rest lie inside tied
+//    groups, whose members share the first D0 symbols.
 // ---------------------------------------------------------------------------
 constexpr int kLcpSerial = 24;         // symbols past D0 one thread compares before handing off
 
-__global__ void lcp_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
-                           const uint64_t *__restrict__ keys, const uint32_t *__restrict__ sa,
-                           int32_t *__restrict__ lcp, int32_t *__restrict__ long_list, int *long_count) {
-    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (gi >= G.N) return;
-    const int s = (int)(gi / G.n);
-    const int j = (int)(gi - (int64_t)s * G.n);
-    if (j == 0) { lcp[gi] = 0; return; }
-    const uint64_t k1 = keys[gi - 1] >> G.idbits, kk2 = keys[gi] >> G.idbits;
-    const uint64_t amask = (1ull << G.abits) - 1ull;
-    const int a1 = (int)(k1 & amask), a2 = (int)(kk2 & amask);
-    if (k1 != kk2) {
-        const uint64_t x = (k1 >> G.abits) ^ (kk2 >> G.abits);
-        int diff = G.D0;
-        if (x) diff = (__clzll((long long)x) - (64 - G.D0 * G.bps)) / G.bps;
-        lcp[gi] = min(diff, min(min(a1, G.D0), min(a2, G.D0)));
-        return;
+// Positions listed by groups0 (inside unresolved round-0 groups): their
+// neighbours share the first D0 symbols; compare onward in the final order.
+__global__ void lcp_ties_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
+                                const uint32_t *__restrict__ sa, int32_t *__restrict__ lcp,
+                                const int32_t *__restrict__ ties, const int *__restrict__ tie_count,
+                                int32_t *__restrict__ long_list, int *long_count) {
+    const int nt = *tie_count;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nt; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t gi = ties[e];
+        const int s = (int)(gi / G.n);
+        const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
+        const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
+        const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
+        const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
+        int m = G.D0;
+        const int lim = min(p1, p2) + 1;
+        const int stop = min(lim, G.D0 + kLcpSerial);
+        while (m < stop && s1[p1 - m] == s2[p2 - m]) ++m;
+        lcp[gi] = m;
+        if (m == stop && m < lim) long_list[atomicAdd(long_count, 1)] = (int32_t)gi;   // still equal: a warp finishes it
     }
-    if (a1 <= G.D0) { lcp[gi] = a1; return; }   // identical complete strings
-    const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
-    const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
-    const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
-    const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
-    int m = G.D0;
-    const int lim = min(p1, p2) + 1;
-    const int stop = min(lim, G.D0 + kLcpSerial);
-    while (m < stop && s1[p1 - m] == s2[p2 - m]) ++m;
-    lcp[gi] = m;
-    if (m == stop && m < lim) long_list[atomicAdd(long_count, 1)] = (int32_t)gi;   // still equal: a warp finishes it
 }
 
 // Long common prefixes (repeats): one warp per pair, 32 symbols per step.
@@ -1579,8 +1738,8 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     uint64_t *scratch = W.keys[cur ^ 1];
     uint32_t *sa = W.sa;
     // 1c. round-0 groups (lists buffer 0)
-    groups0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(keys, sa, G, W.rank, W.lists[0][0], W.lists[0][1],
-                                                       W.counts);
+    groups0_kernel<<<tiles, 256, 0, st>>>(keys, sa, G, W.rank, W.lcp, W.lists[0][0], W.lists[0][1], W.counts,
+                                          W.kcount, W.counts + 10);
     // 1d. doubling rounds while some string is longer than the sorted depth
     int lb = 0;
     const unsigned wgrid = kNumSMs * 8;   // 8 CTAs of 8 warps per SM, grid-stride over groups
@@ -1595,7 +1754,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
         lb ^= 1;
     }
     // 2. LCP
-    lcp_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, keys, sa, W.lcp, W.hard, W.counts + 6);
+    lcp_ties_kernel<<<kNumSMs * 16, 256, 0, st>>>(q, k, G, sa, W.lcp, W.kcount, W.counts + 10, W.hard, W.counts + 6);
     lcp_long_kernel<<<kNumSMs * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
     // 3a. summaries
     summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
