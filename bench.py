@@ -227,6 +227,16 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def wait_first(self, busy, limit_s: float = 3.0):
+        """Run `busy` (GPU work of the timed kind) until the first sample is
+        written, so that a short timed region still has samples under load."""
+        t0 = time.perf_counter()
+        while self.proc and time.perf_counter() - t0 < limit_s:
+            busy()
+            torch.cuda.synchronize()
+            if os.path.getsize(self.path) > 0:
+                break
+
     def stop(self):
         if not self.proc:
             return None
@@ -359,10 +369,11 @@ def main():
     per_step = []
     op_ms = {o: [] for o in wl["ops"]}
     sampler = ClockSampler(local)
+    sampler.start()
+    sampler.wait_first(runner.step)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.start()
     t_wall = time.perf_counter()
     for _ in range(args.steps):
         flush.zero_()

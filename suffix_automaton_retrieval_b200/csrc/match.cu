@@ -57,7 +57,7 @@ int bits_for(int v) {   // number of bits to hold values 0..v
 struct Geometry {
     int S, T, K, g, n;
     bool same;
-    int bps, D0, abits, idbits, keybits;
+    int bps, D0, idbits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
     int wbits, ntw, nw;      // wavelet matrix: levels, 2048-element tiles and 64-bit words per stream
@@ -70,17 +70,16 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     G.N = (int64_t)S * G.n;
     G.bps = bits_for(K - 1);
     if (G.bps < 1) G.bps = 1;
-    // 64-bit sort key: [D0 symbols | available length 0..D0+1 | item id].  The
-    // symbols and length take at most 48 bits (six 8-bit radix passes) and at
-    // most what the item id leaves; deeper ties go to prefix doubling.
+    // 64-bit sort key: [D0 symbols | item id].  The symbols take at most 40
+    // bits (five 8-bit radix passes) and at most what the item id leaves;
+    // deeper ties go to prefix doubling.  Strings shorter than D0 (the first
+    // D0 positions of a stream) are told apart by their initial place in the
+    // array, which the stable sort keeps among equal symbols.
     G.idbits = bits_for(G.n > 0 ? G.n - 1 : 0);
     if (G.idbits < 1) G.idbits = 1;
-    const int budget = min(48, 64 - G.idbits);
-    int d = budget / G.bps;
-    while (d > 1 && d * G.bps + bits_for(d + 1) > budget) --d;
-    G.D0 = d;
-    G.abits = bits_for(d + 1);
-    G.keybits = G.idbits + d * G.bps + G.abits;
+    const int budget = min(40, 64 - G.idbits);
+    G.D0 = max(1, budget / G.bps);
+    G.keybits = G.idbits + G.D0 * G.bps;
     G.ntps = ceil_div(G.n, kRadixTile);
     G.nb1 = ceil_div(G.n, kL1);
     G.nb2 = ceil_div(G.n, kL2);
@@ -191,7 +190,15 @@ __global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__res
         chars = (chars << G.bps) | (c & symmask);
     }
     if ((uint32_t)a[p] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
-    keys[gi] = (((chars << G.abits) | (uint64_t)avail) << G.idbits) | (uint64_t)x;
+    // Initial place: the short strings first, by length, a key before the
+    // query of the same length; then the rest in item order.  Equal symbols
+    // then sort as (length, item id), the order of the full comparison.
+    int pos = x;
+    if (!G.same) {
+        const int m = min(G.D0, G.T);
+        pos = p < m ? 2 * p + (x >= G.T) : (x < G.T ? m + p : x);
+    }
+    keys[(int64_t)s * G.n + pos] = (chars << G.idbits) | (uint64_t)x;
 }
 
 // ---------------------------------------------------------------------------
@@ -338,6 +345,14 @@ __device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ?
 constexpr int kG0Stride = 9;
 __device__ __forceinline__ int g0_slot(int i) { return (i >> 3) * kG0Stride + (i & 7); }
 
+// Round-0 group key: [D0 symbols | available length 0..D0+1], the length
+// taken from the item id.  Sorted keys are ascending in it.
+constexpr int kAvailBits = 6;   // D0 + 1 <= 41
+__device__ __forceinline__ uint64_t g0_key(uint64_t full, const Geometry &G) {
+    const int p = item_pos((uint32_t)(full & ((1ull << G.idbits) - 1ull)), G.T);
+    return ((full >> G.idbits) << kAvailBits) | (uint64_t)min(p + 1, G.D0 + 1);
+}
+
 __global__ void __launch_bounds__(256)
 groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geometry G, int32_t *__restrict__ rank,
                int32_t *__restrict__ lcp, int2 *small, int2 *large, int *counts_next, int32_t *__restrict__ ties,
@@ -354,7 +369,7 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
     const int lim = min(kRadixTile, G.n - j0);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint64_t idmask = (1ull << G.idbits) - 1ull;
-    const uint64_t amask = (1ull << G.abits) - 1ull;
+    const uint64_t amask = (1ull << kAvailBits) - 1ull;
     const int base = threadIdx.x * 8;
     for (int i = threadIdx.x; i < lim; i += 256) sk[g0_slot(i)] = keys[seg + j0 + i];
     if (warp == 0) {
@@ -363,17 +378,17 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
         // its head is a lower bound, found 32 positions per step.
         int h = -1;
         if (j0 > 0 && lim > 0) {
-            const uint64_t kk = keys[seg + j0] >> G.idbits;
+            const uint64_t kk = g0_key(keys[seg + j0], G);
             // backward probes j0-1 .. j0-32 first: most runs are short
             const int p0 = j0 - 1 - lane;
-            const unsigned ne = ~__ballot_sync(ROSA_FULL_MASK, p0 >= 0 && (keys[seg + p0] >> G.idbits) == kk);
+            const unsigned ne = ~__ballot_sync(ROSA_FULL_MASK, p0 >= 0 && g0_key(keys[seg + p0], G) == kk);
             int lo, hi;                            // keys[hi] == kk; the head lies in [lo, hi]
             if (ne) lo = hi = j0 - (__ffs(ne) - 1);
             else { lo = 0; hi = j0 - 32; }
             while (lo < hi) {
                 const int64_t span = hi - lo;
                 const int p = lo + (int)(span * lane / 32);
-                const unsigned b = __ballot_sync(ROSA_FULL_MASK, (keys[seg + p] >> G.idbits) == kk);
+                const unsigned b = __ballot_sync(ROSA_FULL_MASK, g0_key(keys[seg + p], G) == kk);
                 if (b & 1u) { hi = lo; break; }
                 const int f = b ? __ffs(b) - 1 : 32;   // first probe inside the run
                 const int nlo = lo + (int)(span * (f - 1) / 32) + 1;
@@ -390,13 +405,13 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
     int hp = -1;
     unsigned headbits = 0;
     uint64_t prev = ~0ull;
-    if (base < lim && j0 + base > 0) prev = (base > 0 ? sk[g0_slot(base - 1)] : keys[seg + j0 - 1]) >> G.idbits;
+    if (base < lim && j0 + base > 0) prev = g0_key(base > 0 ? sk[g0_slot(base - 1)] : keys[seg + j0 - 1], G);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         const int jl = base + e, j = j0 + jl;
         const bool ok = jl < lim;
         const uint64_t full = ok ? sk[g0_slot(jl)] : 0ull;
-        const uint64_t k = full >> G.idbits;
+        const uint64_t k = g0_key(full, G);
         kv[e] = k;
         id[e] = (uint32_t)(full & idmask);
         if (ok) {
@@ -408,7 +423,7 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
                 l = 0;
             } else if (head) {
                 const int a1 = (int)(prev & amask);
-                const uint64_t x = (prev >> G.abits) ^ (k >> G.abits);
+                const uint64_t x = (prev >> kAvailBits) ^ (k >> kAvailBits);
                 int diff = G.D0;
                 if (x) diff = (__clzll((long long)x) - (64 - G.D0 * G.bps)) / G.bps;
                 l = min(diff, min(min(a1, G.D0), min(a2, G.D0)));
@@ -421,8 +436,8 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
     }
     // first key after this thread's chunk, for end-of-group tests
     uint64_t nk = ~0ull;
-    if (base + 8 < lim) nk = sk[g0_slot(base + 8)] >> G.idbits;
-    else if (base + 8 == lim && j0 + lim < G.n) nk = keys[seg + j0 + lim] >> G.idbits;
+    if (base + 8 < lim) nk = g0_key(sk[g0_slot(base + 8)], G);
+    else if (base + 8 == lim && j0 + lim < G.n) nk = g0_key(keys[seg + j0 + lim], G);
     // exclusive max-scan of the threads' last head positions
     int incl = hp;
 #pragma unroll
