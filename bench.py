@@ -228,12 +228,12 @@ class ClockSampler:
             self.proc = None
 
     def wait_first(self, busy, limit_s: float = 3.0):
-        """Run `busy` (GPU work of the timed kind) until the first sample is
-        written, so that a short timed region still has samples under load."""
+        """Run `busy` (GPU work of the timed kind, synchronised) until the
+        first sample is written, so that a short timed region still has
+        samples under load."""
         t0 = time.perf_counter()
         while self.proc and time.perf_counter() - t0 < limit_s:
             busy()
-            torch.cuda.synchronize()
             if os.path.getsize(self.path) > 0:
                 break
 
@@ -370,7 +370,7 @@ def main():
     op_ms = {o: [] for o in wl["ops"]}
     sampler = ClockSampler(local)
     sampler.start()
-    sampler.wait_first(runner.step)
+    sampler.wait_first(lambda: (runner.step(), torch.cuda.synchronize()))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
