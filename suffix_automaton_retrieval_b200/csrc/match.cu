@@ -267,13 +267,17 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, uint64_t *__restrict__ ko
     unsigned peer[kRadixIPT];
     const int wbase = warp * kWarpItems;
     const unsigned lt = lanemask_lt();
+    // loads first: eight independent loads in flight per thread
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {
+        const int i = wbase + u * 32 + lane;
+        key[u] = i < lim ? kin[base + i] : 0ull;
+    }
     // pass 1: lanes holding the same digit (8 ballots, one per digit bit);
     // each digit's lowest lane adds the group size to the warp's counter
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
-        const int i = wbase + u * 32 + lane;
-        const bool ok = i < lim;
-        key[u] = ok ? kin[base + i] : 0ull;
+        const bool ok = wbase + u * 32 + lane < lim;
         const unsigned d = (unsigned)(key[u] >> shift) & (kRadixBins - 1);
         unsigned pm = __ballot_sync(ROSA_FULL_MASK, ok);
 #pragma unroll
