@@ -865,10 +865,18 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
     __syncthreads();
     int run = pre_s;
     const int t0 = run / kWTile;
+    int c0 = 0, c1 = 0;   // level-0 ones landing in wavelet tiles t0 and t0 + 1
+    uint32_t xs[kRadixIPT];
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {   // loads first: the loop below has barriers
+        const int i = u * 256 + threadIdx.x;
+        xs[u] = i < lim ? sa[base + i] : 0u;
+    }
+#pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
         const int i = u * 256 + threadIdx.x;
         const bool ok = i < lim;
-        const uint32_t x = ok ? sa[base + i] : 0u;
+        const uint32_t x = xs[u];
         const bool key = ok && (G.same || (int)x < G.T);
         const unsigned bal = __ballot_sync(ROSA_FULL_MASK, key);
         if (lane == 0) wk[warp] = __popc(bal);
@@ -882,11 +890,24 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
         if (ok && !G.same) kcount[base + i] = kidx;
         if (key) {
             a0[(int64_t)s * G.T + kidx] = x;
-            if ((x >> (nbits - 1)) & 1u) atomicAdd(&ones[kidx / kWTile - t0], 1);
+            if ((x >> (nbits - 1)) & 1u) {
+                if (kidx / kWTile == t0) ++c0;
+                else ++c1;
+            }
         }
         run += rtot;
         __syncthreads();
     }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        c0 += __shfl_xor_sync(ROSA_FULL_MASK, c0, o);
+        c1 += __shfl_xor_sync(ROSA_FULL_MASK, c1, o);
+    }
+    if (lane == 0) {
+        if (c0) atomicAdd(&ones[0], c0);
+        if (c1) atomicAdd(&ones[1], c1);
+    }
+    __syncthreads();
     if (threadIdx.x < 2 && ones[threadIdx.x]) atomicAdd(&wcnt0[(int64_t)s * ntw + t0 + threadIdx.x], ones[threadIdx.x]);
 }
 
