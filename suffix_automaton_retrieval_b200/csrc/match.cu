@@ -47,6 +47,7 @@ constexpr int kSmemSortCap = 4096;     // larger groups up to this size sort in 
 constexpr int kLargeThreads = 512;
 constexpr int kL1 = 32;                // summary block sizes (ranks)
 constexpr int kL2 = 1024;
+constexpr int kWLeafBits = 5;         // a wavelet leaf holds at most 32 values
 
 int bits_for(int v) {   // number of bits to hold values 0..v
     int b = 0;
@@ -60,7 +61,8 @@ struct Geometry {
     int bps, D0, idbits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
-    int wbits, ntw, nw;      // wavelet matrix: levels, 2048-element tiles and 64-bit words per stream
+    int wbits, ntw, nw;      // wavelet matrix: bits of a key position, 2048-element tiles, 64-bit words per stream
+    int wlev;                // levels built: the rest (kWLeafBits) is scanned in the leaf
 };
 
 Geometry make_geometry(int S, int T, int K, int g, bool same) {
@@ -86,6 +88,7 @@ Geometry make_geometry(int S, int T, int K, int g, bool same) {
     int wb = 0;
     while ((1 << wb) < T) ++wb;   // key positions 0..T-1
     G.wbits = wb < 1 ? 1 : wb;
+    G.wlev = G.wbits > kWLeafBits ? G.wbits - kWLeafBits : 0;
     G.ntw = ceil_div(T, 2048);
     G.nw = (T >> 6) + 1;
     return G;
@@ -166,37 +169,55 @@ Workspace carve(const Geometry &G, void *base) {
     return W;
 }
 
+// Position of item x in its string (keys 0..T-1, then queries).
+__device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ? (int)x : (int)x - T; }
+// Stream of a global item index (item counts stay below 2^31).
+__device__ __forceinline__ int stream_of(int64_t gi, int n) { return (int)((uint32_t)gi / (uint32_t)n); }
+
 // ---------------------------------------------------------------------------
 // 1a. Round-0 keys: first D0 symbols of the reversed prefix, most significant
-//     first, zero-padded past the start, then min(p+1, D0+1) so that a string
-//     that ends sorts before its extensions, then the item id in the low bits
+//     first, zero-padded past the start, then the item id in the low bits
 //     (carried through the sort, never sorted on).
 // ---------------------------------------------------------------------------
-__global__ void keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
-                             uint64_t *__restrict__ keys, uint32_t *__restrict__ status) {
-    const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (gi >= G.N) return;
-    const int s = (int)(gi / G.n);
-    const int x = (int)(gi - (int64_t)s * G.n);
-    const uint8_t *a;
-    int p;
-    if (x < G.T) { a = k + (int64_t)s * G.T; p = x; }
-    else         { a = q + (int64_t)s * G.T; p = x - G.T; }
+// One CTA per 256 positions of one string (a stream's keys or queries): the
+// positions and the D0 - 1 symbols before them are staged in shared memory.
+constexpr int kKeysTile = 256;
+constexpr int kMaxD0 = 40;
+
+__global__ void __launch_bounds__(kKeysTile)
+keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
+             uint64_t *__restrict__ keys, uint32_t *__restrict__ status) {
+    __shared__ uint8_t sb[kMaxD0 + kKeysTile];
+    const int ntile = ceil_div(G.T, kKeysTile);
+    const int sp = blockIdx.x / ntile, tile = blockIdx.x - sp * ntile;
+    const int s = G.same ? sp : sp >> 1;
+    const bool isq = !G.same && (sp & 1);
+    const uint8_t *a = (isq ? q : k) + (int64_t)s * G.T;
+    const int p0 = tile * kKeysTile;
+    for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysTile) {
+        const int p = p0 - kMaxD0 + i;
+        sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;
+    }
+    __syncthreads();
+    const int p = p0 + threadIdx.x;
+    if (p >= G.T) return;
     const uint32_t symmask = (1u << G.bps) - 1u;
     const int avail = min(p + 1, G.D0 + 1);
+    const uint8_t *e = sb + kMaxD0 + threadIdx.x;   // e[-m] = symbol at p - m
     uint64_t chars = 0;
     for (int m = 0; m < G.D0; ++m) {
-        uint32_t c = (m < avail) ? (uint32_t)a[p - m] : 0u;
+        const uint32_t c = (m < avail) ? (uint32_t)e[-m] : 0u;
         chars = (chars << G.bps) | (c & symmask);
     }
-    if ((uint32_t)a[p] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
+    if ((uint32_t)e[0] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
     // Initial place: the short strings first, by length, a key before the
     // query of the same length; then the rest in item order.  Equal symbols
     // then sort as (length, item id), the order of the full comparison.
+    const int x = isq ? G.T + p : p;
     int pos = x;
     if (!G.same) {
         const int m = min(G.D0, G.T);
-        pos = p < m ? 2 * p + (x >= G.T) : (x < G.T ? m + p : x);
+        pos = p < m ? 2 * p + (int)isq : (isq ? x : m + p);
     }
     keys[(int64_t)s * G.n + pos] = (chars << G.idbits) | (uint64_t)x;
 }
@@ -335,7 +356,6 @@ radix_scatter_kernel(const uint64_t *__restrict__ kin, uint64_t *__restrict__ ko
 //     than one incomplete string (p + 1 > D0) go to the unresolved lists
 //     (small: up to kSmallGroup members, large: more).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ? (int)x : (int)x - T; }
 
 // One CTA per 2048-item tile of a stream's round-0 order; thread t owns
 // items [8t, 8t+8).  The tile passes through shared memory (9 words per
@@ -705,7 +725,7 @@ __global__ void lcp_ties_kernel(const uint8_t *__restrict__ q, const uint8_t *__
     const int nt = *tie_count;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nt; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t gi = ties[e];
-        const int s = (int)(gi / G.n);
+        const int s = stream_of(gi, G.n);
         const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
         const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
         const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
@@ -719,7 +739,22 @@ __global__ void lcp_ties_kernel(const uint8_t *__restrict__ q, const uint8_t *__
     }
 }
 
-// Long common prefixes (repeats): one warp per pair, 32 symbols per step.
+// Four symbols of a stream ending at byte address `e` (the symbol at e in the
+// top byte, e-3 in the low byte), from aligned words that lie inside
+// [lo, hi); returns false (nothing read) where they would not.
+__device__ __forceinline__ bool load4_back(const uint8_t *e, const uint8_t *lo, const uint8_t *hi, uint32_t &v) {
+    const uintptr_t a = (uintptr_t)(e - 3);
+    const uintptr_t w = a & ~(uintptr_t)3;
+    const int sh = (int)(a & 3);
+    if (w < (uintptr_t)lo || w + (sh ? 8 : 4) > (uintptr_t)hi) return false;
+    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(w);
+    const uint32_t w1 = sh ? *reinterpret_cast<const uint32_t *>(w + 4) : 0u;
+    v = __funnelshift_r(w0, w1, 8 * sh);
+    return true;
+}
+
+// Long common prefixes (repeats): one warp per pair, 4 symbols per lane and
+// 128 per step, compared as words.
 __global__ void lcp_long_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
                                 const uint32_t *__restrict__ sa, int32_t *__restrict__ lcp,
                                 const int32_t *__restrict__ long_list, const int *__restrict__ long_count) {
@@ -727,24 +762,37 @@ __global__ void lcp_long_kernel(const uint8_t *__restrict__ q, const uint8_t *__
     const int lane = threadIdx.x & 31;
     const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t total = (int64_t)G.S * G.T;
     for (int64_t e = wid; e < nl; e += nw) {
         const int64_t gi = long_list[e];
-        const int s = (int)(gi / G.n);
+        const int s = stream_of(gi, G.n);
         const uint32_t x1 = sa[gi - 1], x2 = sa[gi];
-        const uint8_t *s1 = ((int)x1 < G.T ? k : q) + (int64_t)s * G.T;
-        const uint8_t *s2 = ((int)x2 < G.T ? k : q) + (int64_t)s * G.T;
+        const uint8_t *b1 = (int)x1 < G.T ? k : q, *b2 = (int)x2 < G.T ? k : q;
+        const uint8_t *s1 = b1 + (int64_t)s * G.T, *s2 = b2 + (int64_t)s * G.T;
         const int p1 = item_pos(x1, G.T), p2 = item_pos(x2, G.T);
         const int lim = min(p1, p2) + 1;
         int m = lcp[gi];
         for (;;) {
-            const int i = m + lane;
-            const bool diff = i >= lim || s1[p1 - i] != s2[p2 - i];
-            const unsigned dm = __ballot_sync(ROSA_FULL_MASK, diff);
+            const int i0 = m + 4 * lane;   // this lane compares symbols i0 .. i0+3 back from the ends
+            int off = 4;                   // first differing symbol within the four (4: none)
+            uint32_t v1, v2;
+            if (i0 + 3 < lim && load4_back(s1 + p1 - i0, b1, b1 + total, v1) &&
+                load4_back(s2 + p2 - i0, b2, b2 + total, v2)) {
+                const uint32_t x = v1 ^ v2;
+                if (x) off = __clz(x) >> 3;
+            } else {
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j;
+                    if (i >= lim || s1[p1 - i] != s2[p2 - i]) { off = j; break; }
+                }
+            }
+            const unsigned dm = __ballot_sync(ROSA_FULL_MASK, off < 4);
             if (dm) {
-                m += __ffs(dm) - 1;
+                const int f = __ffs(dm) - 1;
+                m += 4 * f + __shfl_sync(ROSA_FULL_MASK, off, f);
                 break;
             }
-            m += 32;
+            m += 128;
         }
         if (lane == 0) lcp[gi] = m;
     }
@@ -759,38 +807,52 @@ __device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
     return (same || (int)x < T) ? (int)x : INT_MAX;
 }
 
-__global__ void __launch_bounds__(kL2)
+// One CTA of 256 threads per 1024 ranks; thread t loads ranks t + 256u
+// (u < 4) up front, so that each warp's u-th group is one 32-rank block.
+__global__ void __launch_bounds__(256)
 summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__restrict__ lcp,
                int32_t *__restrict__ minpos1, int32_t *__restrict__ emin1, int32_t *__restrict__ ein1,
                int32_t *__restrict__ minpos2, int32_t *__restrict__ emin2, int32_t *__restrict__ ein2) {
-    __shared__ int wpos[32], wemin[32], wfirst[32];
+    constexpr int kPer = kL2 / 256;
+    __shared__ int wpos[kL2 / kL1], wemin[kL2 / kL1], wfirst[kL2 / kL1];
+    __shared__ int edge_in;   // LCP edge entering the 1024 ranks
     const int s = blockIdx.x / G.nb2, B2 = blockIdx.x - s * G.nb2;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int j = B2 * kL2 + threadIdx.x;
-    const int64_t gi = (int64_t)s * G.n + j;
-    int pos = INT_MAX, l = INT_MAX;
-    if (j < G.n) {
-        pos = key_pos_or_inf(sa[gi], G.T, G.same);
-        l = lcp[gi];
-    }
-    const int first = __shfl_sync(ROSA_FULL_MASK, l, 0);
-    int mp = pos, me = lane == 0 ? INT_MAX : l;
+    const int64_t seg = (int64_t)s * G.n;
+    int pos[kPer], l[kPer];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        mp = min(mp, __shfl_xor_sync(ROSA_FULL_MASK, mp, o));
-        me = min(me, __shfl_xor_sync(ROSA_FULL_MASK, me, o));
-    }
-    const int b1 = B2 * (kL2 / kL1) + warp;
-    if (lane == 0) {
-        if (b1 < G.nb1) {
-            minpos1[(int64_t)s * G.nb1 + b1] = mp;
-            emin1[(int64_t)s * G.nb1 + b1] = me;
-            ein1[(int64_t)s * G.nb1 + b1] = first;
+    for (int u = 0; u < kPer; ++u) {
+        const int j = B2 * kL2 + u * 256 + threadIdx.x;
+        pos[u] = INT_MAX;
+        l[u] = INT_MAX;
+        if (j < G.n) {
+            pos[u] = key_pos_or_inf(sa[seg + j], G.T, G.same);
+            l[u] = lcp[seg + j];
         }
-        wpos[warp] = mp;
-        wemin[warp] = me;
-        wfirst[warp] = warp == 0 ? INT_MAX : first;
     }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int first = __shfl_sync(ROSA_FULL_MASK, l[u], 0);
+        int mp = pos[u], me = lane == 0 ? INT_MAX : l[u];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            mp = min(mp, __shfl_xor_sync(ROSA_FULL_MASK, mp, o));
+            me = min(me, __shfl_xor_sync(ROSA_FULL_MASK, me, o));
+        }
+        const int blk = u * 8 + warp;   // 32-rank block within the 1024
+        const int b1 = B2 * (kL2 / kL1) + blk;
+        if (lane == 0) {
+            if (b1 < G.nb1) {
+                minpos1[(int64_t)s * G.nb1 + b1] = mp;
+                emin1[(int64_t)s * G.nb1 + b1] = me;
+                ein1[(int64_t)s * G.nb1 + b1] = first;
+            }
+            wpos[blk] = mp;
+            wemin[blk] = me;
+            wfirst[blk] = blk == 0 ? INT_MAX : first;
+        }
+    }
+    if (threadIdx.x == 0) edge_in = l[0];
     __syncthreads();
     if (warp == 0) {
         int p2 = wpos[lane], e2 = min(wemin[lane], wfirst[lane]);
@@ -802,7 +864,7 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
         if (lane == 0) {
             minpos2[(int64_t)s * G.nb2 + B2] = p2;
             emin2[(int64_t)s * G.nb2 + B2] = e2;
-            ein2[(int64_t)s * G.nb2 + B2] = first;
+            ein2[(int64_t)s * G.nb2 + B2] = edge_in;
         }
     }
 }
@@ -980,7 +1042,7 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         if (i < lim) {
             const int d = bit ? Z + ones_before + lo1 : zeros_before + (i - lo1);
             dst[d] = v[u];
-            if (lv + 1 < nbits && ((v[u] >> (b - 1)) & 1u)) {
+            if (lv + 1 < G.wlev && ((v[u] >> (b - 1)) & 1u)) {
                 const int dt = d / kWTile;
                 atomicAdd(&nxt[bit ? 2 + (dt - or0) : (dt - zr0)], 1);
             }
@@ -1007,7 +1069,7 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         }
     }
     __syncthreads();
-    if (lv + 1 < nbits && threadIdx.x < 4) {
+    if (lv + 1 < G.wlev && threadIdx.x < 4) {
         const int c = nxt[threadIdx.x];
         const int dt = threadIdx.x < 2 ? zr0 + threadIdx.x : or0 + threadIdx.x - 2;
         if (c) atomicAdd(&wcnt[((int64_t)(lv + 1) * G.S + s) * ntw + dt], c);
@@ -1032,13 +1094,17 @@ __device__ __forceinline__ int wrank1(const WWord *W, int i) {
 }
 
 // Largest value <= X in positions [l, r) of the level-0 sequence, or -1.
-__device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, int l, int r, int X) {
+// Only the top nlev bits have levels: a range that shares them holds at most
+// 2^(nbits - nlev) values (key positions are distinct), which are read from
+// the level-nlev sequence `leaf`.
+__device__ int wavelet_max_le(const WWord *W, const int *Z, const uint32_t *leaf, int nbits, int nlev, int nw, int l,
+                              int r, int X) {
     if (l >= r || X < 0) return -1;
     const int top = (1 << nbits) - 1;
     if (X > top) X = top;
     int alt_lv = -1, alt_l = 0, alt_r = 0;
     bool alive = true;
-    for (int lv = 0; lv < nbits; ++lv) {
+    for (int lv = 0; lv < nlev; ++lv) {
         const int b = nbits - 1 - lv;
         const WWord *Wl = W + (int64_t)lv * nw;
         const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
@@ -1053,17 +1119,23 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
         }
         if (l >= r) { alive = false; break; }
     }
-    if (alive) return X;
+    if (alive) {   // values with X's top nlev bits
+        int best = -1;
+        for (int i = l; i < r; ++i) {
+            const int v = (int)leaf[i];
+            if (v <= X && v > best) best = v;
+        }
+        if (best >= 0) return best;
+    }
     if (alt_lv < 0) return -1;
-    int val = (X >> (nbits - alt_lv)) << (nbits - alt_lv);
+    // deepest level where X has a one and the zero side is not empty: every
+    // value there is below X; follow ones where possible, then take the leaf's max
     l = alt_l;
     r = alt_r;
-    for (int lv = alt_lv + 1; lv < nbits; ++lv) {
-        const int b = nbits - 1 - lv;
+    for (int lv = alt_lv + 1; lv < nlev; ++lv) {
         const WWord *Wl = W + (int64_t)lv * nw;
         const int ol = wrank1(Wl, l), orr = wrank1(Wl, r);
         if (orr > ol) {
-            val |= 1 << b;
             l = Z[lv] + ol;
             r = Z[lv] + orr;
         } else {
@@ -1071,7 +1143,9 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, int nbits, int nw, i
             r -= orr;
         }
     }
-    return val;
+    int best = -1;
+    for (int i = l; i < r; ++i) best = max(best, (int)leaf[i]);
+    return best;
 }
 
 // ---------------------------------------------------------------------------
@@ -1116,7 +1190,8 @@ struct ResolveArgs {
     const int32_t *lcp, *mp1, *em1, *ein1, *mp2, *em2, *ein2, *kcount;
     const WWord *words;
     const int *wz;
-    int nbits;
+    const uint32_t *leaf;    // wavelet level-nlev sequence
+    int nbits, nlev;
 };
 
 __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const ResolveArgs &A) {
@@ -1596,7 +1671,7 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restri
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t h = wid; h < nh; h += nw) {
         const int64_t gi = hard[h];
-        const int s = (int)(gi / G.n);
+        const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
         const int t = G.same ? (int)x : (int)x - G.T;
@@ -1631,7 +1706,7 @@ __global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, int32_t *__rest
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t h = wid; h < nh; h += nw) {
         const int64_t gi = hardb[h];
-        const int s = (int)(gi / G.n);
+        const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
         const int t = G.same ? (int)x : (int)x - G.T;
@@ -1681,7 +1756,7 @@ __global__ void bound_finish_kernel(Geometry G, ResolveArgs A, int32_t *__restri
     const int ntr = ceil_div(G.n, kRTile);
     for (int64_t h = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; h < nh; h += (int64_t)gridDim.x * blockDim.x) {
         const int64_t gi = hardw[h];
-        const int s = (int)(gi / G.n);
+        const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
         const int t = G.same ? (int)x : (int)x - G.T;
@@ -1706,11 +1781,12 @@ __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *_
     const int nw = (G.T >> 6) + 1;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t o = wq[i];
-        const int s = (int)(o / G.T);
+        const int s = stream_of(o, G.T);
         const int t = (int)(o - (int64_t)s * G.T);
         const int klo = end_idx[o], khi = sym[o];
         const WWord *W = A.words + (int64_t)s * A.nbits * nw;
-        const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nbits, A.nbits, nw, klo, khi, t - G.g);
+        const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nbits, A.leaf + (int64_t)s * G.T, A.nbits, A.nlev, nw,
+                                      klo, khi, t - G.g);
         end_idx[o] = ib;
         sym[o] = ib >= 0 ? (int32_t)vsym[(int64_t)s * G.T + ib + 1] : -1;
     }
@@ -1743,7 +1819,7 @@ int match_launch_count(int S, int T, int K, bool same) {
     const int passes = ceil_div(G.keybits - G.idbits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
     // + wavelet (key count when q != k, compaction, one per level) + 6 resolve
-    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wbits + 6;
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wlev + 6;
 }
 
 size_t match_workspace_bytes(int S, int T, int K, bool same) {
@@ -1764,7 +1840,8 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     const uint8_t *vs = v ? v : k;
 
     // 1a. keys
-    keys0_kernel<<<grid_for(G.N, 256), 256, 0, st>>>(q, k, G, W.keys[0], W.status);
+    keys0_kernel<<<(unsigned)((int64_t)G.S * (G.same ? 1 : 2) * ceil_div(T, kKeysTile)), kKeysTile, 0, st>>>(
+        q, k, G, W.keys[0], W.status);
     // 1b. radix sort over the key bits above the item id, 8 bits per pass
     int cur = 0;
     const unsigned tiles = (unsigned)(G.S * G.ntps);
@@ -1797,7 +1874,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     lcp_ties_kernel<<<kNumSMs * 16, 256, 0, st>>>(q, k, G, sa, W.lcp, W.kcount, W.counts + 10, W.hard, W.counts + 6);
     lcp_long_kernel<<<kNumSMs * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
     // 3a. summaries
-    summary_kernel<<<(unsigned)(G.S * G.nb2), kL2, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
+    summary_kernel<<<(unsigned)(G.S * G.nb2), 256, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
                                                            W.minpos2, W.emin2, W.ein2);
     // 3b. wavelet matrix over key positions in rank order
     if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wbits * G.S * G.ntw * 4, st)) != cudaSuccess) return err;
@@ -1805,13 +1882,13 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     wavelet_compact_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, G.wbits, sa, W.ktile, W.kcount, W.wvals[0],
                                                                       W.wcnt);
     WWord *words = static_cast<WWord *>(W.words);
-    for (int lv = 0; lv < G.wbits; ++lv)
+    for (int lv = 0; lv < G.wlev; ++lv)
         wavelet_level_kernel<<<(unsigned)(G.S * G.ntw), 256, 0, st>>>(G, G.wbits, lv, W.wvals[lv & 1],
                                                                        W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
     // 3c. resolve: thread per query, then warp per query for the long scans
     if ((err = tile_smem_optin()) != cudaSuccess) return err;
     ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.same ? nullptr : W.kcount,
-                  words, W.wz, G.wbits};
+                  words, W.wz, W.wvals[G.wlev & 1], G.wbits, G.wlev};
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
     int *hardb_count = W.counts + 7;
