@@ -179,12 +179,14 @@ __device__ __forceinline__ int stream_of(int64_t gi, int n) { return (int)((uint
 //     first, zero-padded past the start, then the item id in the low bits
 //     (carried through the sort, never sorted on).
 // ---------------------------------------------------------------------------
-// One CTA per 256 positions of one string (a stream's keys or queries): the
-// positions and the D0 - 1 symbols before them are staged in shared memory.
-constexpr int kKeysTile = 256;
+// One CTA per 2048 positions of one string (a stream's keys or queries), 8
+// per thread: the positions and the D0 - 1 symbols before them are staged in
+// shared memory.
+constexpr int kKeysThreads = 256;
+constexpr int kKeysTile = 2048;
 constexpr int kMaxD0 = 40;
 
-__global__ void __launch_bounds__(kKeysTile)
+__global__ void __launch_bounds__(kKeysThreads)
 keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
              uint64_t *__restrict__ keys, uint32_t *__restrict__ status) {
     __shared__ uint8_t sb[kMaxD0 + kKeysTile];
@@ -194,32 +196,36 @@ keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geome
     const bool isq = !G.same && (sp & 1);
     const uint8_t *a = (isq ? q : k) + (int64_t)s * G.T;
     const int p0 = tile * kKeysTile;
-    for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysTile) {
+    for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysThreads) {
         const int p = p0 - kMaxD0 + i;
         sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;
     }
     __syncthreads();
-    const int p = p0 + threadIdx.x;
-    if (p >= G.T) return;
     const uint32_t symmask = (1u << G.bps) - 1u;
-    const int avail = min(p + 1, G.D0 + 1);
-    const uint8_t *e = sb + kMaxD0 + threadIdx.x;   // e[-m] = symbol at p - m
-    uint64_t chars = 0;
-    for (int m = 0; m < G.D0; ++m) {
-        const uint32_t c = (m < avail) ? (uint32_t)e[-m] : 0u;
-        chars = (chars << G.bps) | (c & symmask);
+    const int m0 = min(G.D0, G.T);
+    uint64_t *out = keys + (int64_t)s * G.n;
+    bool bad = false;
+    for (int u = 0; u < kKeysTile / kKeysThreads; ++u) {
+        const int j = u * kKeysThreads + threadIdx.x;
+        const int p = p0 + j;
+        if (p >= G.T) break;
+        const int avail = min(p + 1, G.D0 + 1);
+        const uint8_t *e = sb + kMaxD0 + j;   // e[-m] = symbol at p - m
+        uint64_t chars = 0;
+        for (int m = 0; m < G.D0; ++m) {
+            const uint32_t c = (m < avail) ? (uint32_t)e[-m] : 0u;
+            chars = (chars << G.bps) | (c & symmask);
+        }
+        bad |= (uint32_t)e[0] >= (uint32_t)G.K;
+        // Initial place: the short strings first, by length, a key before the
+        // query of the same length; then the rest in item order.  Equal symbols
+        // then sort as (length, item id), the order of the full comparison.
+        const int x = isq ? G.T + p : p;
+        int pos = x;
+        if (!G.same) pos = p < m0 ? 2 * p + (int)isq : (isq ? x : m0 + p);
+        out[pos] = (chars << G.idbits) | (uint64_t)x;
     }
-    if ((uint32_t)e[0] >= (uint32_t)G.K) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
-    // Initial place: the short strings first, by length, a key before the
-    // query of the same length; then the rest in item order.  Equal symbols
-    // then sort as (length, item id), the order of the full comparison.
-    const int x = isq ? G.T + p : p;
-    int pos = x;
-    if (!G.same) {
-        const int m = min(G.D0, G.T);
-        pos = p < m ? 2 * p + (int)isq : (isq ? x : m + p);
-    }
-    keys[(int64_t)s * G.n + pos] = (chars << G.idbits) | (uint64_t)x;
+    if (bad) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
 }
 
 // ---------------------------------------------------------------------------
@@ -238,8 +244,15 @@ radix_hist_kernel(const uint64_t *__restrict__ keys, Geometry G, int shift, uint
     __syncthreads();
     const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
     const int lim = min(kRadixTile, G.n - tt * kRadixTile);
-    for (int i = threadIdx.x; i < lim; i += kRadixThreads)
-        atomicAdd(&cnt[(keys[base + i] >> shift) & (kRadixBins - 1)], 1u);
+    uint64_t key[kRadixIPT];
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {   // loads first: eight in flight per thread
+        const int i = u * kRadixThreads + threadIdx.x;
+        key[u] = i < lim ? keys[base + i] : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u)
+        if (u * kRadixThreads + (int)threadIdx.x < lim) atomicAdd(&cnt[(key[u] >> shift) & (kRadixBins - 1)], 1u);
     __syncthreads();
     hist[((int64_t)s * G.ntps + tt) * kRadixBins + threadIdx.x] = cnt[threadIdx.x];
 }
@@ -1792,7 +1805,6 @@ __global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *_
     }
 }
 
-inline unsigned grid_for(int64_t n, int threads) { return (unsigned)ceil_div64(n, threads); }
 
 // The resolve tile needs more than 48 KB of shared memory; opt in once per
 // device (a host-side attribute, so later calls, captured or not, skip it).
@@ -1840,7 +1852,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     const uint8_t *vs = v ? v : k;
 
     // 1a. keys
-    keys0_kernel<<<(unsigned)((int64_t)G.S * (G.same ? 1 : 2) * ceil_div(T, kKeysTile)), kKeysTile, 0, st>>>(
+    keys0_kernel<<<(unsigned)((int64_t)G.S * (G.same ? 1 : 2) * ceil_div(T, kKeysTile)), kKeysThreads, 0, st>>>(
         q, k, G, W.keys[0], W.status);
     // 1b. radix sort over the key bits above the item id, 8 bits per pass
     int cur = 0;
