@@ -560,9 +560,10 @@ __global__ void dbl_keys_sort_kernel(const int2 *__restrict__ small, const int2 
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
         uint32_t *gs = sa + gr.x;
         uint32_t *gk = k2 + gr.x;
-        for (int m = 0; m < gr.y; ++m) {
-            const uint32_t x = gs[m];
-            const uint32_t kk = (uint32_t)rank[seg + x - h];
+        // keys first: the members' rank loads are independent of each other
+        for (int m = 0; m < gr.y; ++m) gk[m] = (uint32_t)rank[seg + gs[m] - h];
+        for (int m = 1; m < gr.y; ++m) {   // insertion sort of (key, id) pairs
+            const uint32_t x = gs[m], kk = gk[m];
             const uint64_t key = pair_key(kk, x);
             int i = m - 1;
             while (i >= 0 && pair_key(gk[i], gs[i]) > key) {
@@ -1362,18 +1363,31 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const int w0 = tt * kRTile - kRHalo;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) { w.nq = 0; w.nb = 0; w.nd = 0; w.need[0] = 0; w.need[1] = 0; }
-    for (int i = threadIdx.x; i <= kRWin; i += kRThreads) {
-        const int r = w0 + i;
-        int p = INT_MAX, l = -1;
-        if (r >= 0 && r < G.n) {
-            if (i < kRWin) p = key_pos_or_inf(A.sa[seg + r], G.T, G.same);
-            l = A.lcp[seg + r];
+    {
+        // loads first: the window's ranks and edges, five of each per thread
+        constexpr int kStage = (kRWin + 1 + kRThreads - 1) / kRThreads;
+        uint32_t xs[kStage];
+        int ls[kStage];
+#pragma unroll
+        for (int u = 0; u < kStage; ++u) {
+            const int i = u * kRThreads + threadIdx.x;
+            const int r = w0 + i;
+            const bool in = i <= kRWin && r >= 0 && r < G.n;
+            xs[u] = (in && i < kRWin) ? A.sa[seg + r] : 0u;
+            ls[u] = in ? A.lcp[seg + r] : -1;
         }
-        if (i < kRWin) {
-            w.kp[i] = p;
-            w.sp[0][i] = (uint8_t)(l < 0 ? 0 : (l > 255 ? 255 : l));
+#pragma unroll
+        for (int u = 0; u < kStage; ++u) {
+            const int i = u * kRThreads + threadIdx.x;
+            if (i > kRWin) break;
+            const int r = w0 + i;
+            const int l = ls[u];
+            if (i < kRWin) {
+                w.kp[i] = (r >= 0 && r < G.n) ? key_pos_or_inf(xs[u], G.T, G.same) : INT_MAX;
+                w.sp[0][i] = (uint8_t)(l < 0 ? 0 : (l > 255 ? 255 : l));
+            }
+            w.lc[i] = l;
         }
-        w.lc[i] = l;
     }
     __syncthreads();
     // sparse table levels, four byte entries per step with byte-wise SIMD minima
