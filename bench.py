@@ -281,10 +281,8 @@ def reduce_over_ranks(local_ms: float, local_units: float, device=None):
 
 # DRAM bytes (read + write) of one rosa_match call, from an ncu capture of the
 # same kernels (dram__bytes_read.sum + dram__bytes_write.sum); None where no
-# capture of the current kernels exists.  zipf-256-131k: captured on its first
-# 16 streams (1.227 GB per call) and scaled by the 8x stream count, which is
-# exact in expectation because the streams are independent.
-PROFILED_DRAM_BYTES = {"zipf-256-131k": 9.81e9}
+# capture of the current kernels exists.
+PROFILED_DRAM_BYTES = {}
 
 
 def load_peaks():
