@@ -1255,7 +1255,7 @@ constexpr int kWarpSteps = 24;         // 32-rank steps of a warp-cooperative sc
 constexpr int kNeedWarp = -1;          // qL codes
 constexpr int kNeedHard = -2;
 
-constexpr int kWarpScanMax = 256;      // widest interval a warp scans in shared memory
+constexpr int kWarpScanMax = 128;      // widest interval a warp scans in shared memory
 constexpr int kBoundShared = 64;       // match lengths whose out-of-window bounds are shared per tile
 
 struct WinSmem {
