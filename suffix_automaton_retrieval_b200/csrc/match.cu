@@ -179,9 +179,11 @@ __device__ __forceinline__ int stream_of(int64_t gi, int n) { return (int)((uint
 //     first, zero-padded past the start, then the item id in the low bits
 //     (carried through the sort, never sorted on).
 // ---------------------------------------------------------------------------
-// One CTA per 2048 positions of one string (a stream's keys or queries), 8
-// per thread: the positions and the D0 - 1 symbols before them are staged in
-// shared memory.
+// One CTA per 2048 positions of one string (a stream's keys or queries).
+// The positions and the D0 - 1 symbols before them are staged in shared
+// memory; thread t builds the keys of positions 8t .. 8t+7, each from the
+// previous one by one shift (the oldest symbol drops out at the bottom), and
+// the keys leave through shared memory in coalesced stores.
 constexpr int kKeysThreads = 256;
 constexpr int kKeysTile = 2048;
 constexpr int kMaxD0 = 40;
@@ -190,42 +192,47 @@ __global__ void __launch_bounds__(kKeysThreads)
 keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
              uint64_t *__restrict__ keys, uint32_t *__restrict__ status) {
     __shared__ uint8_t sb[kMaxD0 + kKeysTile];
+    __shared__ uint64_t sk[kKeysThreads * 9];   // 9 words per thread: conflict-free
     const int ntile = ceil_div(G.T, kKeysTile);
     const int sp = blockIdx.x / ntile, tile = blockIdx.x - sp * ntile;
     const int s = G.same ? sp : sp >> 1;
     const bool isq = !G.same && (sp & 1);
     const uint8_t *a = (isq ? q : k) + (int64_t)s * G.T;
     const int p0 = tile * kKeysTile;
+    const int lim = min(kKeysTile, G.T - p0);
     for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysThreads) {
         const int p = p0 - kMaxD0 + i;
-        sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;
+        sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;   // zeros before the start pad short strings
     }
     __syncthreads();
     const uint32_t symmask = (1u << G.bps) - 1u;
-    const int m0 = min(G.D0, G.T);
-    uint64_t *out = keys + (int64_t)s * G.n;
+    const int top = (G.D0 - 1) * G.bps;
+    const int j0 = threadIdx.x * 8;
     bool bad = false;
-    for (int u = 0; u < kKeysTile / kKeysThreads; ++u) {
-        const int j = u * kKeysThreads + threadIdx.x;
-        const int p = p0 + j;
-        if (p >= G.T) break;
-        const int avail = min(p + 1, G.D0 + 1);
-        const uint8_t *e = sb + kMaxD0 + j;   // e[-m] = symbol at p - m
+    if (j0 < lim) {
+        const uint8_t *e = sb + kMaxD0 + j0;      // e[-m] = symbol at p0 + j0 - m
         uint64_t chars = 0;
-        for (int m = 0; m < G.D0; ++m) {
-            const uint32_t c = (m < avail) ? (uint32_t)e[-m] : 0u;
-            chars = (chars << G.bps) | (c & symmask);
+        for (int m = 0; m < G.D0; ++m) chars = (chars << G.bps) | ((uint32_t)e[-m] & symmask);
+        for (int u = 0; u < 8 && j0 + u < lim; ++u) {
+            if (u > 0) chars = (chars >> G.bps) | ((uint64_t)((uint32_t)e[u] & symmask) << top);
+            bad |= (uint32_t)e[u] >= (uint32_t)G.K;
+            const int x = (isq ? G.T : 0) + p0 + j0 + u;
+            sk[threadIdx.x * 9 + u] = (chars << G.idbits) | (uint64_t)x;
         }
-        bad |= (uint32_t)e[0] >= (uint32_t)G.K;
-        // Initial place: the short strings first, by length, a key before the
-        // query of the same length; then the rest in item order.  Equal symbols
-        // then sort as (length, item id), the order of the full comparison.
-        const int x = isq ? G.T + p : p;
-        int pos = x;
-        if (!G.same) pos = p < m0 ? 2 * p + (int)isq : (isq ? x : m0 + p);
-        out[pos] = (chars << G.idbits) | (uint64_t)x;
     }
     if (bad) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
+    __syncthreads();
+    // Initial place: the short strings first, by length, a key before the
+    // query of the same length; then the rest in item order.  Equal symbols
+    // then sort as (length, item id), the order of the full comparison.
+    uint64_t *out = keys + (int64_t)s * G.n;
+    const int m0 = min(G.D0, G.T);
+    for (int i = threadIdx.x; i < lim; i += kKeysThreads) {
+        const int p = p0 + i;
+        int pos = p;
+        if (!G.same) pos = p < m0 ? 2 * p + (int)isq : (isq ? G.T + p : m0 + p);
+        out[pos] = sk[(i >> 3) * 9 + (i & 7)];
+    }
 }
 
 // ---------------------------------------------------------------------------
