@@ -280,9 +280,10 @@ def reduce_over_ranks(local_ms: float, local_units: float, device=None):
 
 
 # DRAM bytes (read + write) of one rosa_match call, from an ncu capture of the
-# same kernels (dram__bytes_read.sum + dram__bytes_write.sum); None where no
-# capture of the current kernels exists.
-PROFILED_DRAM_BYTES = {}
+# same kernels (dram__bytes_read.sum + dram__bytes_write.sum, summed over the
+# call's launches); None where no capture of the current kernels exists.
+# zipf-256-131k: captured at full size (one pass per launch).
+PROFILED_DRAM_BYTES = {"zipf-256-131k": 9.835e9}
 
 
 def load_peaks():
