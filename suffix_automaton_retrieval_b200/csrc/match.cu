@@ -1171,16 +1171,16 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, const uint32_t *leaf
 
 // ---------------------------------------------------------------------------
 // 3c. Per-query resolution.
-//     Phase 1 (resolve_tile_kernel): a CTA stages 1024 ranks plus 1024 on
-//     each side (key position, LCP edge) in shared memory and resolves the
-//     tile's queries there.  The nearest admissible key on each side gives L;
-//     the interval scan then continues from that key, so every rank is
-//     visited about once.  Queries whose scans would leave the staged window
-//     or exceed a visit budget go to a list.
-//     Phase 2 (resolve_hard_kernel): one warp per listed query scans global
-//     memory 32 ranks or 32 blocks per step for L and the interval bounds;
-//     the most recent admissible end comes from the wavelet matrix, 32
-//     queries per warp in parallel.
+//     resolve_tile_kernel: a CTA stages 1024 ranks plus 512 on each side (key
+//     position, LCP edge) in shared memory and resolves the tile's queries
+//     there: the nearest admissible key on each side gives L, binary lifting
+//     on a sparse table gives the interval of ranks sharing L symbols, and a
+//     scan of that interval gives i* when it spans at most 128 ranks.
+//     Wider intervals are parked for wavelet_query_kernel.  Queries whose
+//     nearest key lies outside the window go to resolve_hard_kernel (one warp
+//     per query over global memory, 32 ranks or 32 blocks per step); interval
+//     ends outside the window are found by resolve_bounds_kernel, or once per
+//     (tile, side, L) for short L by bound_task/bound_finish_kernel.
 // ---------------------------------------------------------------------------
 constexpr int kRTile = 1024;
 constexpr int kRHalo = 512;
@@ -1347,15 +1347,16 @@ __device__ void window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
     }
 }
 
-// One CTA per 1024 ranks of a stream, with 1024 ranks of context on each side.
+// One CTA per 1024 ranks of a stream, with 512 ranks of context on each side.
 //   Phase A: each lane probes 16 ranks on each side of its query for the
 //            nearest admissible key (fixed trip count, no divergence).
 //   Phase B: queries the probes could not settle get a warp each, scanning
 //            32 ranks per step in shared memory.
 //   Phase C: each lane finds its interval bounds by binary lifting on the
-//            sparse table, then i* by a 16-rank probe or, for wider
-//            intervals, a deferred wavelet lookup.
-// Queries whose answer needs ranks outside the window go to the hard list.
+//            sparse table, then i* by a 16-rank probe; intervals of up to
+//            kWarpScanMax ranks go to phase D, wider ones to the wavelet.
+//   Phase D: one warp per listed interval, 32 ranks per step.
+// Queries whose answer needs ranks outside the window go to the hard lists.
 __global__ void __launch_bounds__(kRThreads, 4)
 resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
                     int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
