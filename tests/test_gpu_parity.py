@@ -91,6 +91,38 @@ def test_match_degenerate_streams(rosa):
             _assert_same(_gpu_match(rosa, q, k, None, K, g), oracle.match_sam(q, k, g=g), f"K={K} g={g}")
 
 
+@pytest.mark.parametrize("T", [20, 32, 33, 64, 65, 128, 129, 256, 257, 1024, 1025])
+def test_match_wide_intervals_near_powers_of_two(rosa, T):
+    """Low-entropy streams, where many matches share a short suffix with hundreds of ranks, so
+    their most recent admissible end comes from the wavelet matrix; T around powers of two moves
+    the number of wavelet levels (none up to T = 32, the last five bits are always a leaf scan)."""
+    rng = np.random.default_rng(300 + T)
+    S = 6
+    streams = [
+        (np.zeros((S, T), np.uint8), 1),
+        ((rng.random((S, T)) < 0.1).astype(np.uint8), 2),
+        (((np.arange(T)[None, :] + rng.integers(0, 3, (S, 1))) % 3).astype(np.uint8), 3),
+    ]
+    for q, K in streams:
+        k_ind = (rng.random((S, T)) < 0.1).astype(np.uint8) if K > 1 else np.zeros((S, T), np.uint8)
+        for k in (q, q.copy(), k_ind):
+            for g in (1, 2):
+                want = oracle.match_brute(q, k, g=g)
+                _assert_same(_gpu_match(rosa, q, k, None, K, g), want, f"T={T} K={K} g={g} k_is_q={k is q}")
+
+
+def test_match_many_short_streams(rosa):
+    """Many streams of a few positions: grids sized by the stream count (over 65535 streams too)."""
+    rng = np.random.default_rng(77)
+    for S, T, K in [(70000, 2, 256), (20000, 3, 2), (5000, 17, 4), (3000, 40, 256)]:
+        q = rng.integers(0, K, (S, T)).astype(np.uint8)
+        k = rng.integers(0, K, (S, T)).astype(np.uint8)
+        for kk in (q, k):
+            for g in (1, 2):
+                _assert_same(_gpu_match(rosa, q, kk, None, K, g), oracle.match_brute(q, kk, g=g),
+                             f"S={S} T={T} K={K} g={g}")
+
+
 def test_match_recipes_reduced(rosa):
     """The five input recipes at sizes the oracle finishes in seconds."""
     ws = [
