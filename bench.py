@@ -66,7 +66,7 @@ def build_workload(cfg: int, device, seed_offset: int = 0):
 
     wl = {"cfg": cfg}
     if cfg == 3:
-        c = W.CONFIGS[3]
+        c = W.spec("qwen-proj-64")
         T, width, ch, M, d, rho = c["T"], c["width"], c["channels"], c["M"], c["d"], c["rho"]
         H, Wq, Wk = W.qwen_projection_inputs(T=T, width=width, channels=ch, device=device,
                                              seed_h=3 + 1000 * seed_offset)
@@ -79,7 +79,7 @@ def build_workload(cfg: int, device, seed_offset: int = 0):
         wl["V"] = W.value_rows(1, T, R * rho, seed=c["seed_v"] + 1000 * seed_offset, device=device)
         wl["ops"] = ["discretize", "match", "gather"]
         return wl
-    c = W.CONFIGS[cfg]
+    c = W.WORKLOADS[cfg]
     if seed_offset:
         # other ranks draw the same recipe with shifted seeds
         gen = {1: lambda: W.binary_iid(seed=1 + 1000 * seed_offset),
@@ -522,7 +522,7 @@ def run_reference(args, rank, world):
         print(json.dumps({"impl": "reference", "unavailable":
                           "qwen-proj-64 needs the GPU projection set-up; reference arm runs on symbol workloads"}))
         return 0
-    sw = W.CONFIGS[cfg]["make"]()
+    sw = W.WORKLOADS[cfg]["make"]()
     cores = os.cpu_count() or 1
     n = args.cpu_sample_streams or min(sw.S, cores)
     # size the per-step sample so the whole run stays within a few minutes

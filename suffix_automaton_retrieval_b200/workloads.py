@@ -194,7 +194,7 @@ def value_rows(B: int, T: int, width: int, seed: int, device="cpu"):
 # registry of the five full-size workloads
 # --------------------------------------------------------------------------
 
-CONFIGS = {
+WORKLOADS = {
     1: dict(name="binary-4k", kind="symbols", make=lambda: binary_iid()),
     2: dict(name="planted-16", kind="symbols", make=lambda: planted_copies()),
     3: dict(name="qwen-proj-64", kind="hidden", T=32768, width=2048, channels=64, M=1,
@@ -202,3 +202,11 @@ CONFIGS = {
     4: dict(name="zipf-256-131k", kind="symbols", make=lambda: zipf_planted()),
     5: dict(name="markov-4-train", kind="symbols", make=lambda: markov(), d=64, rho=64, seed_v=53),
 }
+
+
+def spec(name: str) -> dict:
+    """The registry entry of the workload called ``name``."""
+    for v in WORKLOADS.values():
+        if v["name"] == name:
+            return v
+    raise KeyError(name)

@@ -89,7 +89,7 @@ def test_full_zipf_256_131k(rosa):
 
 
 def test_full_markov_4_train_with_gather(rosa):
-    c = workloads.CONFIGS[5]
+    c = workloads.spec("markov-4-train")
     w = workloads.markov()
     got, streams = _symbol_case(rosa, w, 12)
     V = workloads.value_rows(w.B, w.T, w.R * c["rho"], seed=c["seed_v"], device=DEV)
@@ -106,7 +106,7 @@ def test_full_markov_4_train_with_gather(rosa):
 
 
 def test_full_qwen_proj_64_path(rosa):
-    c = workloads.CONFIGS[3]
+    c = workloads.spec("qwen-proj-64")
     T, width, ch, M, d, rho = c["T"], c["width"], c["channels"], c["M"], c["d"], c["rho"]
     H, Wq, Wk = workloads.qwen_projection_inputs(T=T, width=width, channels=ch, device=DEV)
     qv, kv = (H @ Wq).contiguous(), (H @ Wk).contiguous()
