@@ -1,0 +1,100 @@
+"""Host-side logic of bench.py that needs no GPU: the algorithmic-byte
+counts behind the roofline, the clock sampler's parsing and throttle
+detection, and the reference arm (the CPU oracle) with its JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+from tests.conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+class _Vec:
+    def __init__(self, shape):
+        self.shape = shape
+
+
+def test_algorithmic_bytes_per_op():
+    # zipf-256-131k: q and k (1 B each) and three int32 outputs per position
+    wl = {"S": 128, "T": 131072, "same": False, "ops": ["match"]}
+    assert bench.algorithmic_bytes(wl) == {"match": 128 * 131072 * 14}
+    # self-retrieval reads one symbol stream
+    wl = {"S": 128, "T": 16384, "same": True, "ops": ["match"]}
+    assert bench.algorithmic_bytes(wl)["match"] == 128 * 16384 * 13
+    # markov-4-train: the gather reads end_idx and a d-wide bf16 row, writes the row
+    wl = {"S": 2048, "T": 8192, "same": False, "ops": ["match", "gather"], "B": 8, "R": 256, "d": 64}
+    assert bench.algorithmic_bytes(wl)["gather"] == 8 * 8192 * 256 * (4 + 2 * 64 * 2)
+    # qwen-proj-64: two bf16 [1, T, 64] tensors read, two u8 [1, 64, T] symbol tensors written
+    wl = {"S": 64, "T": 32768, "same": False, "ops": ["discretize", "match", "gather"], "B": 1, "R": 64,
+          "d": 128, "M": 1, "qvec": _Vec((1, 32768, 64))}
+    assert bench.algorithmic_bytes(wl)["discretize"] == 2 * (32768 * 64 * 2 + 64 * 32768)
+
+
+def _sampler_with(tmp_path, lines):
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "clocks.csv")
+    with open(s.path, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    s.proc = subprocess.Popen([sys.executable, "-c", "pass"])
+    return s
+
+
+def test_clock_sampler_reports_median_and_reasons(tmp_path):
+    row = "0, {mhz} MHz, 1965 MHz, 800.00 W, 0x0, Not Active, Not Active, Not Active, {cap}"
+    s = _sampler_with(tmp_path, [row.format(mhz=1965, cap="Not Active"), row.format(mhz=1800, cap="Active"),
+                                 row.format(mhz=1950, cap="Not Active"), "garbage line"])
+    c = s.stop()
+    assert c["sm_mhz"] == 1950 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_flags_thermal_slowdown(tmp_path):
+    row = "0, 1500 MHz, 1965 MHz, 900.00 W, 0x0, Not Active, Active, Not Active, Not Active"
+    c = _sampler_with(tmp_path, [row]).stop()
+    assert c["reasons"] == ["hw_thermal_slowdown"]
+
+
+def test_clock_sampler_without_samples(tmp_path):
+    assert _sampler_with(tmp_path, []).stop() is None
+
+
+def _run_bench(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
+                          timeout=600, cwd=ROOT, env=env)
+
+
+def test_reference_arm_prints_one_oracle_line():
+    out = _run_bench(["--impl", "reference", "--config", "1", "--steps", "2", "--warmup", "1"])
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "positions/s" and d["value"] > 0
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "binary-4k"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_nothing():
+    out = _run_bench(["--impl", "reference", "--config", "1", "--steps", "1", "--warmup", "0"],
+                     {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("cfg", [1])
+def test_cpu_baseline_reports_all_cores_and_one_core(cfg):
+    from suffix_automaton_retrieval_b200 import workloads as W
+    sw = W.binary_iid(T=4096, S=3)
+    wl = {"cfg": cfg, "q_host": sw.q, "k_host": sw.k, "S": sw.S, "T": sw.T, "same": sw.same_qk, "g": sw.g}
+    c = bench.cpu_oracle_baseline(wl, target_seconds=(0.01, 0.1))
+    assert c["kind"] == "oracle" and c["value"] > 0 and c["cores"] >= 1
+    assert c["single_core"]["cores"] == 1 and c["single_core"]["value"] > 0
