@@ -451,11 +451,17 @@ def main():
 
 def end_to_end(wl, device, steps):
     """Same metric through the public API with host buffers: pinned host
-    inputs copied in, the step, outputs copied back, every step."""
+    inputs copied in, the step, outputs copied back, every step.
+
+    Steps alternate between two CUDA streams, each with its own device
+    buffers and workspace, as a caller overlapping transfers would run them:
+    one step's copies overlap the neighbouring steps' kernels.  The same
+    steps on one stream (no overlap) are timed and reported beside it, and
+    the two buffer sets' results must agree."""
     import torch
     rosa = __import__("suffix_automaton_retrieval_b200.binding", fromlist=["x"])
     S, T = wl["S"], wl["T"]
-    stream = torch.cuda.current_stream(device)
+    main = torch.cuda.current_stream(device)
     if "discretize" in wl["ops"]:
         hin = [wl["qvec"].cpu().pin_memory(), wl["kvec"].cpu().pin_memory(), wl["V"].cpu().pin_memory()]
     elif "gather" in wl["ops"]:
@@ -465,16 +471,23 @@ def end_to_end(wl, device, steps):
         hin = [torch.from_numpy(wl["q_host"]).pin_memory()]
         if not wl["same"]:
             hin.append(torch.from_numpy(wl["k_host"]).pin_memory())
-    din = [torch.empty_like(h, device=device) for h in hin]
-    ws = rosa.alloc_workspace(S, T, wl["K"], device)
-    outs = tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))
-    if "gather" in wl["ops"]:
-        gout = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
-        hout = [torch.empty(gout.shape, dtype=gout.dtype).pin_memory()]
-    else:
-        hout = [torch.empty((S, T), dtype=torch.int32).pin_memory() for _ in range(3)]
 
-    def one():
+    def make_set():
+        b = {"din": [torch.empty_like(h, device=device) for h in hin],
+             "ws": rosa.alloc_workspace(S, T, wl["K"], device),
+             "outs": tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))}
+        if "gather" in wl["ops"]:
+            b["gout"] = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
+            b["hout"] = [torch.empty(b["gout"].shape, dtype=b["gout"].dtype).pin_memory()]
+        else:
+            b["hout"] = [torch.empty((S, T), dtype=torch.int32).pin_memory() for _ in range(3)]
+        return b
+
+    sets = [make_set()]
+    side = []
+
+    def one(b):
+        din, hout = b["din"], b["hout"]
         for h, d in zip(hin, din):
             d.copy_(h, non_blocking=True)
         if "discretize" in wl["ops"]:
@@ -484,29 +497,58 @@ def end_to_end(wl, device, steps):
         else:
             q = din[0]
             k = None if wl["same"] else din[1]
-        e, l, s = rosa.match(q, k, K=wl["K"], g=wl["g"], out=outs, workspace=ws)
+        e, l, s = rosa.match(q, k, K=wl["K"], g=wl["g"], out=b["outs"], workspace=b["ws"])
         if "gather" in wl["ops"]:
-            rosa.gather(din[-1], e, wl["R"], wl["d"], wl["rho"], out=gout)
-            hout[0].copy_(gout, non_blocking=True)
+            rosa.gather(din[-1], e, wl["R"], wl["d"], wl["rho"], out=b["gout"])
+            hout[0].copy_(b["gout"], non_blocking=True)
         else:
             for h, d in zip(hout, (e, l, s)):
                 h.copy_(d, non_blocking=True)
 
-    for _ in range(2):
-        one()
+    def timed(overlap):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        if overlap:
+            for st in side:
+                st.wait_event(e0)
+            for i in range(steps):
+                with torch.cuda.stream(side[i % 2]):
+                    one(sets[i % 2])
+            for st in side:
+                main.wait_stream(st)
+        else:
+            for _ in range(steps):
+                one(sets[0])
+        e1.record(main)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    for _ in range(2):   # warm-up
+        one(sets[0])
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    seq_ms = timed(False)
+    overlap_ok = False
+    try:   # the overlapped form; on any failure the one-stream figure stands
+        sets.append(make_set())
+        side.extend([torch.cuda.Stream(device), torch.cuda.Stream(device)])
+        for i in range(2):
+            with torch.cuda.stream(side[i]):
+                one(sets[i])
+        torch.cuda.synchronize()
+        pipe_ms = timed(True)
+        overlap_ok = all(torch.equal(a, b) for a, b in zip(sets[0]["hout"], sets[1]["hout"]))
+    except Exception as ex:  # noqa: BLE001 - reported, not fatal
+        print(f"bench: overlapped end-to-end run failed ({ex!r}); reporting the one-stream figure",
+              file=sys.stderr)
+    ms = pipe_ms if overlap_ok else seq_ms
     h2d = sum(h.numel() * h.element_size() for h in hin)
-    d2h = sum(h.numel() * h.element_size() for h in hout)
+    d2h = sum(h.numel() * h.element_size() for h in sets[0]["hout"])
     return {"value": S * T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
+            "overlap": ("two CUDA streams, alternate buffer sets: a step's copies overlap the neighbouring "
+                        "steps' kernels" if overlap_ok else "none (one stream)"),
+            "sequential_ms_per_step": seq_ms / steps}
 
 
 def run_reference(args, rank, world):

@@ -1,6 +1,8 @@
 """Host-side logic of bench.py that needs no GPU: the algorithmic-byte
 counts behind the roofline, the clock sampler's parsing and throttle
-detection, and the reference arm (the CPU oracle) with its JSON line."""
+detection, the reference arm (the CPU oracle) with its JSON line, and the
+control flow of the end-to-end measurement (with CPU stand-ins for the CUDA
+stream API and the binding)."""
 import json
 import os
 import subprocess
@@ -98,3 +100,87 @@ def test_cpu_baseline_reports_all_cores_and_one_core(cfg):
     c = bench.cpu_oracle_baseline(wl, target_seconds=(0.01, 0.1))
     assert c["kind"] == "oracle" and c["value"] > 0 and c["cores"] >= 1
     assert c["single_core"]["cores"] == 1 and c["single_core"]["value"] > 0
+
+
+# ---------------------------------------------------------------- end-to-end control flow
+
+class _FakeEvent:
+    def __init__(self, enable_timing=False):
+        self.t = None
+
+    def record(self, stream=None):
+        import time
+        self.t = time.perf_counter()
+
+    def elapsed_time(self, other):
+        return (other.t - self.t) * 1e3
+
+
+class _FakeStream:
+    def __init__(self, device=None):
+        self.waits = []
+
+    def wait_event(self, e):
+        self.waits.append(e)
+
+    def wait_stream(self, s):
+        self.waits.append(s)
+
+
+def _fake_cuda(monkeypatch, match_fails_on_workspace=None):
+    """CPU stand-ins for the CUDA stream/event API and for the binding, so
+    that the end-to-end driver's control flow runs without a GPU."""
+    import contextlib
+    import types
+    import torch
+    main = _FakeStream()
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: main)
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "Stream", _FakeStream)
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    fake = types.ModuleType("suffix_automaton_retrieval_b200.binding")
+    made = []
+
+    def alloc_workspace(S, T, K, device):
+        made.append(torch.empty(16, dtype=torch.uint8))
+        return made[-1]
+
+    def match(q, k=None, v=None, *, K, g, out, workspace):
+        i = match_fails_on_workspace
+        if i is not None and len(made) > i and workspace is made[i]:
+            raise RuntimeError("injected failure")
+        kk = q if k is None else k
+        out[0].copy_(q.int() * 7 + kk.int())
+        out[1].copy_(q.int() + g)
+        out[2].copy_(kk.int() - K)
+        return out
+
+    fake.alloc_workspace, fake.match = alloc_workspace, match
+    monkeypatch.setitem(sys.modules, "suffix_automaton_retrieval_b200.binding", fake)
+    return main
+
+
+def _symbol_wl():
+    import numpy as np
+    rng = np.random.default_rng(5)
+    return {"S": 3, "T": 40, "K": 4, "g": 2, "same": False, "ops": ["match"],
+            "q_host": rng.integers(0, 4, (3, 40)).astype(np.uint8),
+            "k_host": rng.integers(0, 4, (3, 40)).astype(np.uint8)}
+
+
+def test_end_to_end_overlapped_form(monkeypatch):
+    _fake_cuda(monkeypatch)
+    e = bench.end_to_end(_symbol_wl(), "cpu", 5)
+    assert e["overlap"].startswith("two CUDA streams")
+    assert e["h2d_bytes_per_step"] == 2 * 3 * 40 and e["d2h_bytes_per_step"] == 3 * 3 * 40 * 4
+    assert e["value"] > 0 and e["ms_per_step"] > 0 and e["sequential_ms_per_step"] > 0
+
+
+def test_end_to_end_falls_back_to_one_stream(monkeypatch, capsys):
+    _fake_cuda(monkeypatch, match_fails_on_workspace=1)   # the second buffer set fails
+    e = bench.end_to_end(_symbol_wl(), "cpu", 3)
+    assert e["overlap"] == "none (one stream)"
+    assert e["ms_per_step"] == e["sequential_ms_per_step"]
+    assert "overlapped end-to-end run failed" in capsys.readouterr().err
