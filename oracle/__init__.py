@@ -15,6 +15,10 @@ Enhancing Windowed Attention with Global Recall" (arXiv 2602.02499):
 * ``match_sam`` -- the online suffix automaton of section 2.2 run in lockstep
   with the query stream (appendix B.3: tau = endpos + 1).
 * ``gather`` -- appendix C.4 read-out at tau with the Eq. (17) mask.
+* ``match_cf_brute`` / ``match_cf_sam`` -- the per-bit counterfactual
+  destinations of section 3.5: every query bit forced to 0 and to 1, one
+  retrieval step each from the same historical state (definition and
+  automaton forms).
 """
 from __future__ import annotations
 
@@ -53,7 +57,10 @@ def _load():
         lib.oracle_match_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
         lib.oracle_gather.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, i32p,
                                       c_int, c_int, c_int, c_int, u16p]
-        for f in (lib.oracle_discretize, lib.oracle_match_brute, lib.oracle_match_sam, lib.oracle_gather):
+        lib.oracle_match_cf_brute.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p]
+        lib.oracle_match_cf_sam.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p, c_int]
+        for f in (lib.oracle_discretize, lib.oracle_match_brute, lib.oracle_match_sam, lib.oracle_gather,
+                  lib.oracle_match_cf_brute, lib.oracle_match_cf_sam):
             f.restype = c_int
         _lib = lib
     return _lib
@@ -116,6 +123,40 @@ def match_brute(q, k, v=None, g: int = 2):
 def match_sam(q, k, v=None, g: int = 2, threads: int | None = None):
     """Online suffix-automaton matcher over host threads.  Returns (end_idx, len, sym)."""
     return _match("sam", q, k, v, g, threads)
+
+
+def _match_cf(fn: str, q, k, M, g, threads=None):
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    k = np.ascontiguousarray(k, dtype=np.uint8)
+    if q.ndim == 1:
+        q, k = q[None], k[None]
+    S, T = q.shape
+    if k.shape != (S, T):
+        raise ValueError("q and k must have the same shape [S, T]")
+    if M < 1 or M > 8 or (q.size and int(q.max()) >= (1 << M)):
+        raise ValueError("need 1 <= M <= 8 and query symbols below 2^M")
+    end = np.empty((S, T, M, 2), np.int32)
+    ln = np.empty((S, T, M, 2), np.int32)
+    lib = _load()
+    args = [_ptr(q, ctypes.c_uint8), _ptr(k, ctypes.c_uint8), S, T, M, g,
+            _ptr(end, ctypes.c_int32), _ptr(ln, ctypes.c_int32)]
+    if fn == "sam":
+        args.append(threads if threads else (os.cpu_count() or 1))
+        _check(lib.oracle_match_cf_sam(*args), "match_cf_sam")
+    else:
+        _check(lib.oracle_match_cf_brute(*args), "match_cf_brute")
+    return end, ln
+
+
+def match_cf_brute(q, k, M: int, g: int = 2):
+    """Counterfactual destinations by the definition.  Returns (end_idx, len),
+    each ``[S, T, M, 2]``: position t with query bit j forced to beta."""
+    return _match_cf("brute", q, k, M, g)
+
+
+def match_cf_sam(q, k, M: int, g: int = 2, threads: int | None = None):
+    """Counterfactual destinations with the suffix automaton (same layout)."""
+    return _match_cf("sam", q, k, M, g, threads)
 
 
 def gather(V_bits: np.ndarray, end_idx: np.ndarray, R: int, d: int, rho: int) -> np.ndarray:

@@ -18,6 +18,9 @@
  *                                  O(1) transitions and suffix-link jumps
  *   appendix B.3                   tau_t = endpos(s_t) + 1 when it exists, else -1
  *   appendix C.4, Eq. (17)         read-out of the value at tau, mask I[tau >= 0]
+ *   section 3.5                    counterfactual branches: each query bit forced
+ *                                  to 0 and to 1, one retrieval step each from
+ *                                  the same historical state
  *
  * Readings taken where the pages are garbled or silent (Eq. 16 itself is lost
  * in the page text):
@@ -350,6 +353,160 @@ int oracle_match_sam(const uint8_t *q, const uint8_t *k, const uint8_t *v,
     /* streams of threads that failed to start are done here */
     for (int i = started + 1; i < nthreads; ++i) {
         sam_worker(&jobs[i]);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    free(th);
+    free(jobs);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-bit counterfactual destinations (section 3.5: each query bit is a     */
+/* decision switch; the branches "force the bit to 0" and "force it to 1"    */
+/* each take one retrieval step from the same historical state).             */
+/*                                                                           */
+/* For position t, bit j < M and beta in {0, 1}, the branch symbol is        */
+/* c = (q[t] with bit j set to beta).  The history q[0..t-1] and the keys    */
+/* are unchanged, so the branch's longest admissible match and most recent   */
+/* end follow from D(t-1, .) alone:                                          */
+/*   D'(t, i) = k[i] == c ? 1 + D(t-1, i-1) : 0,  L' = max_{i <= t-g} D',     */
+/*   i*' = largest such i with D'(t, i) = L' when L' > 0, else -1.           */
+/* Outputs end_cf, len_cf: [S, T, M, 2] int32, index beta last.              */
+/* ------------------------------------------------------------------------ */
+
+static int cf_brute_stream(const uint8_t *q, const uint8_t *k, int T, int M, int g,
+                           int32_t *end_cf, int32_t *len_cf)
+{
+    int32_t *prev = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));   /* D(t-1, .) */
+    int32_t *cur = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));
+    if (!prev || !cur) { free(prev); free(cur); return ORACLE_ERR_NOMEM; }
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < M; ++j)
+            for (int beta = 0; beta < 2; ++beta) {
+                unsigned c = ((unsigned)q[t] & ~(1u << j)) | ((unsigned)beta << j);
+                int best = 0, best_i = -1;
+                for (int i = 0; i <= t - g; ++i) {
+                    if (k[i] != c) continue;
+                    int d = 1 + ((t > 0 && i > 0) ? prev[i - 1] : 0);
+                    if (d >= best) { best = d; best_i = i; }   /* later i wins ties */
+                }
+                size_t o = (((size_t)t * M) + j) * 2 + beta;
+                end_cf[o] = best_i;
+                len_cf[o] = best;
+            }
+        /* advance D with the actual query symbol */
+        for (int i = 0; i < T; ++i)
+            cur[i] = (q[t] == k[i]) ? 1 + ((t > 0 && i > 0) ? prev[i - 1] : 0) : 0;
+        int32_t *tmp = prev; prev = cur; cur = tmp;
+    }
+    free(prev);
+    free(cur);
+    return ORACLE_OK;
+}
+
+int oracle_match_cf_brute(const uint8_t *q, const uint8_t *k, int S, int T, int M, int g,
+                          int32_t *end_cf, int32_t *len_cf)
+{
+    if (S < 0 || T < 0 || M < 1 || M > 8 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    for (int s = 0; s < S; ++s) {
+        size_t o = (size_t)s * T;
+        size_t oc = o * (size_t)M * 2;
+        int rc = cf_brute_stream(q + o, k + o, T, M, g, end_cf + oc, len_cf + oc);
+        if (rc) return rc;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The same with the suffix automaton: at each t, after inserting k[t-g],
+ * every branch symbol is tried from the matching state (state, L) that the
+ * actual step starts from, by the same transition rule, without moving it;
+ * then the actual symbol q[t] advances the state as in sam_stream.
+ */
+static int cf_sam_stream(const uint8_t *q, const uint8_t *k, int T, int M, int g,
+                         int32_t *end_cf, int32_t *len_cf)
+{
+    sam_t a;
+    int rc = sam_init(&a, T);
+    if (rc) { sam_free(&a); return rc; }
+    int st = 0, L = 0;
+    for (int t = 0; t < T; ++t) {
+        int p = t - g;
+        if (p >= 0) {
+            rc = sam_extend(&a, k[p], p);
+            if (rc) { sam_free(&a); return rc; }
+        }
+        for (int j = 0; j < M; ++j)
+            for (int beta = 0; beta < 2; ++beta) {
+                uint8_t c = (uint8_t)(((unsigned)q[t] & ~(1u << j)) | ((unsigned)beta << j));
+                int s2 = st, L2 = L;
+                while (s2 != 0 && sam_get(&a, s2, c) < 0) {
+                    s2 = a.link[s2];
+                    L2 = a.len[s2];
+                }
+                int nx = sam_get(&a, s2, c);
+                if (nx >= 0) { s2 = nx; L2 += 1; } else { s2 = 0; L2 = 0; }
+                size_t o = (((size_t)t * M) + j) * 2 + beta;
+                end_cf[o] = L2 > 0 ? a.last_end[s2] : -1;
+                len_cf[o] = L2;
+            }
+        uint8_t c = q[t];
+        while (st != 0 && sam_get(&a, st, c) < 0) {
+            st = a.link[st];
+            L = a.len[st];
+        }
+        int nx = sam_get(&a, st, c);
+        if (nx >= 0) { st = nx; L += 1; } else { st = 0; L = 0; }
+    }
+    sam_free(&a);
+    return ORACLE_OK;
+}
+
+typedef struct {
+    const uint8_t *q, *k;
+    int S, T, M, g, nthreads, tid;
+    int32_t *end_cf, *len_cf;
+    int rc;
+} cf_job_t;
+
+static void *cf_worker(void *arg)
+{
+    cf_job_t *j = (cf_job_t *)arg;
+    j->rc = ORACLE_OK;
+    for (int s = j->tid; s < j->S; s += j->nthreads) {
+        size_t o = (size_t)s * j->T;
+        size_t oc = o * (size_t)j->M * 2;
+        int rc = cf_sam_stream(j->q + o, j->k + o, j->T, j->M, j->g, j->end_cf + oc, j->len_cf + oc);
+        if (rc) { j->rc = rc; break; }
+    }
+    return NULL;
+}
+
+int oracle_match_cf_sam(const uint8_t *q, const uint8_t *k, int S, int T, int M, int g,
+                        int32_t *end_cf, int32_t *len_cf, int nthreads)
+{
+    if (S < 0 || T < 0 || M < 1 || M > 8 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > S) nthreads = S > 0 ? S : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    cf_job_t *jobs = (cf_job_t *)malloc(sizeof(cf_job_t) * nthreads);
+    if (!th || !jobs) { free(th); free(jobs); return ORACLE_ERR_NOMEM; }
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        cf_job_t jb = {q, k, S, T, M, g, nthreads, i, end_cf, len_cf, 0};
+        jobs[i] = jb;
+        if (i == 0) continue;
+        if (pthread_create(&th[i], NULL, cf_worker, &jobs[i]) != 0) break;
+        started = i;
+    }
+    cf_worker(&jobs[0]);
+    int rc = jobs[0].rc;
+    for (int i = 1; i <= started; ++i) {
+        pthread_join(th[i], NULL);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    for (int i = started + 1; i < nthreads; ++i) {
+        cf_worker(&jobs[i]);
         if (jobs[i].rc) rc = jobs[i].rc;
     }
     free(th);
