@@ -10,8 +10,9 @@ setting (arXiv 2602.02499: section 3.2 multi-route symbol streams, section
 
 1. ``binary-4k``       1 stream, T=4096, K=2, i.i.d. Bernoulli(0.5), q = k.
 2. ``planted-16``      4 x 32 streams, T=16384, K=16 uniform with planted
-                       copy segments (length 32..256) covering >= 5% of each
-                       stream, q = k.
+                       copy segments (length 32..256) whose disjoint
+                       destinations cover 5% of each stream (a later copy may
+                       overwrite an earlier one's source), q = k.
 3. ``qwen-proj-64``    B=1, T=32768: bf16 hidden states N(0,1) of width 2048,
                        seeded Gaussian projections W_q, W_k (N(0, 1/2048)) to
                        64 channels; M=1 gives 64 binary routes; value rows
