@@ -10,7 +10,10 @@
  * Conventions shared by every call:
  *   - All tensor pointers are DEVICE pointers into memory the caller owns
  *     (cudaMalloc, a torch tensor, ...).  The library allocates nothing and
- *     keeps no state between calls.
+ *     keeps no state between calls, with one exception: rosa_match_noalloc
+ *     (below) takes its scratch from a fixed device array the library
+ *     reserves on every GPU that loads it, which keeps the last call's
+ *     contents.
  *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the
  *     call returns without waiting for it, except where stated.
  *   - Argument errors are detected on the host before anything is enqueued
@@ -65,6 +68,14 @@ ROSA_API const char *rosa_status_string(int status);
  */
 ROSA_API int rosa_discretize(const rosa_bf16 *x, int B, int T, int C, int M,
                     uint8_t *sym, cudaStream_t stream);
+
+/*
+ * rosa_discretize of the query and the key projections (two tensors of the
+ * same shape) in one launch: xq -> symq, xk -> symk, each as above.
+ * Requires B <= 32767; otherwise the same conditions as rosa_discretize.
+ */
+ROSA_API int rosa_discretize_pair(const rosa_bf16 *xq, const rosa_bf16 *xk, int B, int T, int C, int M,
+                                  uint8_t *symq, uint8_t *symk, cudaStream_t stream);
 
 /*
  * Bytes of workspace rosa_match needs for S streams of length T over an
@@ -136,14 +147,27 @@ ROSA_API int rosa_match_device_status(const void *workspace, cudaStream_t stream
  * q != k over 256 symbols.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any
- * stream capture.  All calls share the one array and it keeps the last
- * call's contents: calls that overlap on the GPU (different streams or
- * threads) race and must be serialised by the caller.
+ * stream capture.  The address is cached for the life of the process: after
+ * cudaDeviceReset on a device, do not call this entry point on that device
+ * again (the cached address may no longer be the array's).  All calls share
+ * the one array and it keeps the last call's contents: calls that overlap on
+ * the GPU (different streams or threads) race and must be serialised by the
+ * caller.  Symbols >= K are masked and flagged as for rosa_match; the flag
+ * is read with rosa_match_noalloc_device_status.
  */
 #define ROSA_NOALLOC_SCRATCH_BYTES (64u << 20)
 ROSA_API int rosa_match_noalloc(const uint8_t *q, const uint8_t *k, const uint8_t *v,
                                 int S, int T, int K, int g,
                                 int32_t *end_idx, int32_t *len, int32_t *sym, cudaStream_t stream);
+
+/*
+ * The device status word (ROSA_DEV_* bits) the last rosa_match_noalloc call
+ * on the current device left in the fixed array; the counterpart of
+ * rosa_match_device_status for callers without a workspace.  Synchronises
+ * `stream`.  Returns ROSA_OK, ROSA_ERR_INVALID_ARG (NULL status) or
+ * ROSA_ERR_CUDA.
+ */
+ROSA_API int rosa_match_noalloc_device_status(cudaStream_t stream, uint32_t *status);
 
 /*
  * Read-out of value rows at tau (appendix C.4 with the Eq. 17 mask).

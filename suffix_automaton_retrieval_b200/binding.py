@@ -29,6 +29,8 @@ lib.rosa_status_string.argtypes = [_i]
 lib.rosa_status_string.restype = ctypes.c_char_p
 lib.rosa_discretize.argtypes = [_vp, _i, _i, _i, _i, _vp, _vp]
 lib.rosa_discretize.restype = _i
+lib.rosa_discretize_pair.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]
+lib.rosa_discretize_pair.restype = _i
 lib.rosa_match_workspace_size.argtypes = [_i, _i, _i]
 lib.rosa_match_workspace_size.restype = ctypes.c_size_t
 lib.rosa_match.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -40,7 +42,7 @@ lib.rosa_match_device_status.restype = _i
 lib.rosa_gather.argtypes = [_vp, _i64, _i64, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.rosa_gather.restype = _i
 
-EXPORTED = ("rosa_status_string", "rosa_discretize", "rosa_match_workspace_size", "rosa_match",
+EXPORTED = ("rosa_status_string", "rosa_discretize", "rosa_discretize_pair", "rosa_match_workspace_size", "rosa_match",
             "rosa_match_launch_count", "rosa_match_device_status", "rosa_gather")
 
 DEV_SYMBOL_RANGE = 1
@@ -88,6 +90,27 @@ def discretize(x: torch.Tensor, M: int, out: torch.Tensor | None = None) -> torc
         out = torch.empty((B, C // M, T), dtype=torch.uint8, device=x.device)
     _check(lib.rosa_discretize(_ptr(x), B, T, C, M, _ptr(out), _stream(x.device)), "rosa_discretize")
     return out
+
+
+def discretize_pair(xq: torch.Tensor, xk: torch.Tensor, M: int, out=None):
+    """The query and key projections, both bf16 ``[B, T, C]``, discretised in
+    one launch -> ``(sym_q, sym_k)``, each uint8 ``[B, C // M, T]``."""
+    _need_cuda(xq, xk)
+    for x in (xq, xk):
+        if x.dtype != torch.bfloat16 or x.dim() != 3:
+            raise ValueError("xq and xk must be bf16 tensors [B, T, C]")
+    if xq.shape != xk.shape:
+        raise ValueError("xq and xk must have the same shape")
+    xq, xk = xq.contiguous(), xk.contiguous()
+    B, T, C = xq.shape
+    if M < 1 or M > 8 or C % M:
+        raise ValueError("need 1 <= M <= 8 and C % M == 0")
+    if out is None:
+        out = tuple(torch.empty((B, C // M, T), dtype=torch.uint8, device=xq.device) for _ in range(2))
+    sq, sk = out
+    _check(lib.rosa_discretize_pair(_ptr(xq), _ptr(xk), B, T, C, M, _ptr(sq), _ptr(sk), _stream(xq.device)),
+           "rosa_discretize_pair")
+    return sq, sk
 
 
 def match_workspace_size(S: int, T: int, K: int) -> int:

@@ -7,8 +7,6 @@
 
 namespace rosa {
 
-constexpr int kNumSMs = 148;   // B200: 2 dies x 74 SMs
-
 __host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

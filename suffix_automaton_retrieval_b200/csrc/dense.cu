@@ -32,12 +32,16 @@ __device__ __forceinline__ uint8_t positive_bit(uint16_t h) {
     return __bfloat162float(__ushort_as_bfloat16(h)) > 0.0f ? 1 : 0;
 }
 
-// grid: (t tiles, channel tiles, B)
+// grid: (t tiles, channel tiles, B x tensors); tensor i = blockIdx.z / B
+// reads x_i and writes sym_i (the query and key projections share a launch).
 __global__ void __launch_bounds__(kDiscThreads)
-discretize_kernel(const uint16_t *__restrict__ x, int T, int C, int M, int CC, bool vec,
-                  uint8_t *__restrict__ sym) {
+discretize_kernel(const uint16_t *__restrict__ x0, const uint16_t *__restrict__ x1, int B, int T, int C, int M,
+                  int CC, bool vec, uint8_t *__restrict__ sym0, uint8_t *__restrict__ sym1) {
     __shared__ uint8_t bits[kDiscTT][kDiscCC];
-    const int b = blockIdx.z;
+    const int which = blockIdx.z >= (unsigned)B;
+    const int b = blockIdx.z - which * B;
+    const uint16_t *__restrict__ x = which ? x1 : x0;
+    uint8_t *__restrict__ sym = which ? sym1 : sym0;
     const int t0 = blockIdx.x * kDiscTT;
     const int c0 = blockIdx.y * CC;
     const int cc = min(CC, C - c0);
@@ -81,15 +85,17 @@ discretize_kernel(const uint16_t *__restrict__ x, int T, int C, int M, int CC, b
 
 }  // namespace
 
-cudaError_t launch_discretize(const uint16_t *x, int B, int T, int C, int M, uint8_t *sym,
-                              cudaStream_t stream) {
-    if (B == 0 || T == 0) return cudaSuccess;
+cudaError_t launch_discretize(const uint16_t *const *x, uint8_t *const *sym, int count, int B, int T, int C,
+                              int M, cudaStream_t stream) {
+    if (B == 0 || T == 0 || count < 1) return cudaSuccess;
     int CC = (kDiscCC / M) * M;
     if (CC > C) CC = C;
     // vector path: every tile starts on a 16-byte boundary and covers whole 8-channel groups
-    const bool vec = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (C % 8 == 0) && (CC % 8 == 0);
-    dim3 grid((unsigned)ceil_div(T, kDiscTT), (unsigned)ceil_div(C, CC), (unsigned)B);
-    discretize_kernel<<<grid, kDiscThreads, 0, stream>>>(x, T, C, M, CC, vec, sym);
+    bool vec = (C % 8 == 0) && (CC % 8 == 0);
+    for (int i = 0; i < count; ++i) vec = vec && (reinterpret_cast<uintptr_t>(x[i]) % 16 == 0);
+    dim3 grid((unsigned)ceil_div(T, kDiscTT), (unsigned)ceil_div(C, CC), (unsigned)(B * count));
+    discretize_kernel<<<grid, kDiscThreads, 0, stream>>>(x[0], x[count - 1], B, T, C, M, CC, vec, sym[0],
+                                                         sym[count - 1]);
     return cudaGetLastError();
 }
 

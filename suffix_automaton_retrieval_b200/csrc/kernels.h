@@ -6,8 +6,13 @@
 
 namespace rosa {
 
-cudaError_t launch_discretize(const uint16_t *x, int B, int T, int C, int M, uint8_t *sym,
-                              cudaStream_t stream);
+// Streaming multiprocessors of the current device (queried once per device);
+// grids of grid-stride kernels are sized in multiples of it.
+int device_sm_count();
+
+// One launch for `count` (1 or 2) tensors of the same shape.
+cudaError_t launch_discretize(const uint16_t *const *x, uint8_t *const *sym, int count, int B, int T, int C,
+                              int M, cudaStream_t stream);
 
 cudaError_t launch_gather(const uint16_t *V, int64_t vrow, int64_t rho, const int32_t *end_idx,
                           int B, int R, int T, int d, uint16_t *out, cudaStream_t stream);

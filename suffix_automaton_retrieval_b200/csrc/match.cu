@@ -1845,6 +1845,20 @@ cudaError_t tile_smem_optin() {
 
 }  // namespace
 
+int device_sm_count() {
+    static std::mutex mu;
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 148;
+        sms[dev] = n;
+    }
+    return sms[dev];
+}
+
 int match_launch_count(int S, int T, int K, bool same) {
     if (S == 0 || T == 0) return 0;
     const Geometry G = make_geometry(S, T, K, 1, same);
@@ -1893,20 +1907,21 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
                                           W.kcount, W.counts + 10);
     // 1d. doubling rounds while some string is longer than the sorted depth
     int lb = 0;
-    const unsigned wgrid = kNumSMs * 8;   // 8 CTAs of 8 warps per SM, grid-stride over groups
+    const int sms = device_sm_count();
+    const unsigned wgrid = sms * 8;   // 8 CTAs of 8 warps per SM, grid-stride over groups
     for (int64_t h = G.D0; h < T; h *= 2) {
         int *cnt = W.counts + 2 * lb;
         int *cnt_next = W.counts + 2 * (lb ^ 1);
         dbl_keys_sort_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, h, sa, W.rank, W.k2);
-        dbl_sort_large_kernel<<<kNumSMs * 2, kLargeThreads, 0, st>>>(W.lists[lb][1], cnt, sa, W.k2, scratch);
+        dbl_sort_large_kernel<<<sms * 2, kLargeThreads, 0, st>>>(W.lists[lb][1], cnt, sa, W.k2, scratch);
         if ((err = cudaMemsetAsync(cnt_next, 0, 2 * sizeof(int), st)) != cudaSuccess) return err;
         dbl_regroup_kernel<<<wgrid, 256, 0, st>>>(W.lists[lb][0], W.lists[lb][1], cnt, G, 2 * h, sa, W.k2, W.rank,
                                                   W.lists[lb ^ 1][0], W.lists[lb ^ 1][1], cnt_next);
         lb ^= 1;
     }
     // 2. LCP
-    lcp_ties_kernel<<<kNumSMs * 16, 256, 0, st>>>(q, k, G, sa, W.lcp, W.kcount, W.counts + 10, W.hard, W.counts + 6);
-    lcp_long_kernel<<<kNumSMs * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
+    lcp_ties_kernel<<<sms * 16, 256, 0, st>>>(q, k, G, sa, W.lcp, W.kcount, W.counts + 10, W.hard, W.counts + 6);
+    lcp_long_kernel<<<sms * 8, 256, 0, st>>>(q, k, G, sa, W.lcp, W.hard, W.counts + 6);
     // 3a. summaries
     summary_kernel<<<(unsigned)(G.S * G.nb2), 256, 0, st>>>(G, sa, W.lcp, W.minpos1, W.emin1, W.ein1,
                                                            W.minpos2, W.emin2, W.ein2);
@@ -1931,13 +1946,13 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
         G, A, vs, end_idx, len, sym, W.hard, hard_count, W.hardb, hardb_count, W.hardw, hardw_count, W.btask,
         btask_count, W.wq, wq_count);
-    resolve_hard_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
-    resolve_bounds_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardb, hardb_count, W.wq,
+    resolve_hard_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
+    resolve_bounds_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardb, hardb_count, W.wq,
                                                         wq_count);
-    bound_task_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, W.btask, btask_count, W.btab);
-    bound_finish_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardw, hardw_count, W.btab, W.wq,
+    bound_task_kernel<<<sms * 16, 256, 0, st>>>(G, A, W.btask, btask_count, W.btab);
+    bound_finish_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardw, hardw_count, W.btab, W.wq,
                                                       wq_count);
-    wavelet_query_kernel<<<kNumSMs * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
+    wavelet_query_kernel<<<sms * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
     return cudaGetLastError();
 }
 

@@ -60,3 +60,16 @@ extern "C" int rosa_match_noalloc(const uint8_t *q, const uint8_t *k, const uint
                ? ROSA_OK
                : ROSA_ERR_CUDA;
 }
+
+extern "C" int rosa_match_noalloc_device_status(cudaStream_t stream, uint32_t *status) {
+    if (!status) return ROSA_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess) return ROSA_ERR_CUDA;
+    uint32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, static_cast<const char *>(scratch) + rosa::kStatusOffset, sizeof h,
+                                    cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return ROSA_ERR_CUDA;
+    *status = h;
+    return ROSA_OK;
+}

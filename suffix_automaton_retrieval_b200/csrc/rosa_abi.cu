@@ -37,7 +37,18 @@ const char *rosa_status_string(int status) {
 int rosa_discretize(const rosa_bf16 *x, int B, int T, int C, int M, uint8_t *sym, cudaStream_t stream) {
     if (B < 0 || T < 0 || C < 1 || M < 1 || M > 8 || C % M != 0 || B > 65535) return ROSA_ERR_INVALID_ARG;
     if ((int64_t)B * T > 0 && (!x || !sym)) return ROSA_ERR_INVALID_ARG;
-    return cuda_status(rosa::launch_discretize(x, B, T, C, M, sym, stream));
+    const uint16_t *xs[1] = {x};
+    uint8_t *ss[1] = {sym};
+    return cuda_status(rosa::launch_discretize(xs, ss, 1, B, T, C, M, stream));
+}
+
+int rosa_discretize_pair(const rosa_bf16 *xq, const rosa_bf16 *xk, int B, int T, int C, int M, uint8_t *symq,
+                         uint8_t *symk, cudaStream_t stream) {
+    if (B < 0 || T < 0 || C < 1 || M < 1 || M > 8 || C % M != 0 || B > 32767) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!xq || !xk || !symq || !symk)) return ROSA_ERR_INVALID_ARG;
+    const uint16_t *xs[2] = {xq, xk};
+    uint8_t *ss[2] = {symq, symk};
+    return cuda_status(rosa::launch_discretize(xs, ss, 2, B, T, C, M, stream));
 }
 
 size_t rosa_match_workspace_size(int S, int T, int K) {

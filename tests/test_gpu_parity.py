@@ -193,6 +193,25 @@ def test_discretize_parity(rosa, B, T, C, M):
     assert np.array_equal(got.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("B,T,C,M,misalign", [(1, 65, 64, 1, False), (2, 40, 24, 3, False), (1, 33, 48, 2, True)])
+def test_discretize_pair_parity(rosa, B, T, C, M, misalign):
+    """Query and key in one launch: each equals the oracle's discretisation;
+    with one operand at an odd element offset both take the scalar path."""
+    rng = np.random.default_rng(7 * B + T + C + M)
+    bq, bk = _bf16_bits_special(rng, (B, T, C)), _bf16_bits_special(rng, (B, T, C))
+    xq = torch.from_numpy(bq.view(np.int16)).to(DEV).view(torch.bfloat16)
+    xk = torch.from_numpy(bk.view(np.int16)).to(DEV).view(torch.bfloat16)
+    if misalign:
+        buf = torch.empty(xk.numel() + 1, dtype=torch.bfloat16, device=DEV)
+        view = buf[1:].view(xk.shape)
+        view.copy_(xk)
+        xk = view
+    sq, sk = rosa.discretize_pair(xq, xk, M)
+    torch.cuda.synchronize()
+    assert np.array_equal(sq.cpu().numpy(), oracle.discretize(bq, M))
+    assert np.array_equal(sk.cpu().numpy(), oracle.discretize(bk, M))
+
+
 def test_discretize_unaligned_view(rosa):
     rng = np.random.default_rng(3)
     bits = _bf16_bits_special(rng, (1, 50, 65))

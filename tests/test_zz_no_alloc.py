@@ -37,16 +37,31 @@ def lib():
     return b
 
 
-def _noalloc(b, q, k, v, K, g):
+def _noalloc_rc(b, q, k, v, K, g):
     S, T = q.shape
     outs = [torch.full((S, T), 12345, dtype=torch.int32, device=DEV) for _ in range(3)]
     vp = ctypes.c_void_p
     rc = b.lib.rosa_match_noalloc(vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()) if v is not None else None,
                                   S, T, K, g, vp(outs[0].data_ptr()), vp(outs[1].data_ptr()),
                                   vp(outs[2].data_ptr()), vp(torch.cuda.current_stream().cuda_stream))
-    assert rc == 0, b.status_string(rc)
     torch.cuda.synchronize()
+    return rc, outs
+
+
+def _noalloc(b, q, k, v, K, g):
+    rc, outs = _noalloc_rc(b, q, k, v, K, g)
+    assert rc == 0, b.status_string(rc)
     return [o.cpu().numpy() for o in outs]
+
+
+def _noalloc_status(b):
+    st = ctypes.c_uint32(0xdead)
+    f = b.lib.rosa_match_noalloc_device_status
+    f.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
+    f.restype = ctypes.c_int
+    rc = f(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream), ctypes.byref(st))
+    assert rc == 0, b.status_string(rc)
+    return st.value
 
 
 def _regular(b, q, k, v, K, g):
@@ -87,3 +102,50 @@ def test_no_alloc_rejects_sizes_beyond_the_array(lib):
     fake = vp(0x10000)   # never dereferenced: the size check comes first
     rc = lib.lib.rosa_match_noalloc(fake, vp(0x20000), None, S, T, K, 2, fake, fake, fake, None)
     assert rc == 2      # ROSA_ERR_WORKSPACE
+
+
+def test_no_alloc_near_the_limit(lib):
+    """The array almost full: the largest q != k problem of 16384-symbol
+    streams over 256 symbols that fits, then a self-retrieval problem as
+    large as the array admits, both bit-exact against rosa_match."""
+    T, K = 16384, 256
+    S = 1
+    while lib.match_workspace_size(S + 1, T, K) <= SCRATCH_BYTES:
+        S += 1
+    assert lib.match_workspace_size(S, T, K) > 0.9 * SCRATCH_BYTES
+    w = workloads.zipf_planted(S=S, T=T, K=K, seed_q=11, seed_k=12, seed_plant=13, lmax=512)
+    q, k = torch.from_numpy(w.q).to(DEV), torch.from_numpy(w.k).to(DEV)
+    want = _regular(lib, q, k, None, K, w.g)
+    got = _noalloc(lib, q, k, None, K, w.g)
+    for a, b_ in zip(got, want):
+        assert np.array_equal(a, b_)
+    assert _noalloc_status(lib) == 0
+    # self-retrieval needs about half the scratch per position: grow S until rejected
+    wq = workloads.planted_copies(B=1, R=3 * S, T=T, K=16, seed=21)
+    Sq = 3 * S
+    while True:
+        qq = torch.from_numpy(np.ascontiguousarray(wq.q[:Sq])).to(DEV)
+        rc, _ = _noalloc_rc(lib, qq, qq, None, 16, wq.g)
+        if rc == 0:
+            break
+        assert rc == 2          # ROSA_ERR_WORKSPACE, nothing launched
+        Sq -= 1
+    assert Sq < 3 * S           # the limit was reached, not the start size
+    assert Sq > S               # the self-retrieval form admits more streams
+    want = _regular(lib, qq, qq, None, 16, wq.g)
+    got = _noalloc(lib, qq, qq, None, 16, wq.g)
+    for a, b_ in zip(got, want):
+        assert np.array_equal(a, b_)
+
+
+def test_no_alloc_reports_out_of_range_symbols(lib):
+    rng = np.random.default_rng(3)
+    qh = rng.integers(0, 4, (2, 700)).astype(np.uint8)
+    qh[1, 350] = 9                            # >= K = 4: masked and flagged
+    q = torch.from_numpy(qh).to(DEV)
+    _noalloc(lib, q, q, None, 4, 2)
+    assert _noalloc_status(lib) & lib.DEV_SYMBOL_RANGE
+    qh[1, 350] = 1
+    q = torch.from_numpy(qh).to(DEV)
+    _noalloc(lib, q, q, None, 4, 2)
+    assert _noalloc_status(lib) == 0          # cleared by the next call
