@@ -1258,7 +1258,6 @@ __device__ __forceinline__ int warp_prefix_min(int x, int lane) {
 // Queries are resolved in three uniform phases (see resolve_tile_kernel).
 constexpr int kSpLevels = 11;          // lifting reaches 2^11 - 1 ranks: a whole side of the window
 constexpr int kProbe = 16;             // ranks a lane probes on each side before its warp helps
-constexpr int kWarpSteps = 24;         // 32-rank steps of a warp-cooperative scan (768 ranks)
 constexpr int kNeedWarp = -1;          // qL codes
 constexpr int kNeedHard = -2;
 
@@ -1276,6 +1275,9 @@ struct WinSmem {
     int16_t dhi[kRTile];     // (their query indices reuse bq)
     unsigned long long need[2];   // lengths L < 64 whose interval leaves the window below / above
     int nq, nb, nd;
+    int bkp[kRWin / 32];     // per 32-rank block: smallest key position,
+    int beL[kRWin / 32];     //   LCP minimum crossed walking down through it (lc[32B+1 .. 32B+32]),
+    int beR[kRWin / 32];     //   and walking up through it (lc[32B .. 32B+31])
     uint8_t sp[kSpLevels][kRWin];
 };
 
@@ -1291,32 +1293,69 @@ __device__ __forceinline__ void defer_wavelet(const Geometry &G, int s, int t, i
     wq[atomicAdd(wq_count, 1)] = (int32_t)o;
 }
 
-// Warp-cooperative nearest admissible key in direction dir, 32 ranks per
-// step: the LCP with it when that exceeds lim, 0 when the running LCP falls
-// to lim first, kNeedHard when the answer lies beyond the window or the steps.
+// Warp-cooperative nearest admissible key in direction dir: the LCP with it
+// when that exceeds lim, 0 when the running LCP falls to lim first,
+// kNeedHard when the answer lies beyond the window.  The ranks up to the end
+// of jl's 32-rank block are scanned directly; beyond it the warp takes 32
+// whole blocks per step from their summaries (smallest key position, LCP
+// minimum) and scans only the first block that holds an admissible key.
 __device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int lim, int lane) {
-    int carry = INT_MAX;
-    for (int step = 0; step < kWarpSteps; ++step) {
-        const int r = jl + dir * (1 + step * 32 + lane);
-        int e;
-        bool valid;
-        if (dir < 0) {
-            e = r >= -1 ? w.lc[r + 1] : kNeedHard;
-            valid = r >= 0 && w.kp[r] <= X;
+    constexpr int kNB = kRWin / 32;
+    int blk, cnt0, r;
+    if (dir < 0) {
+        const int rtop = jl - 1;
+        blk = rtop >> 5;
+        cnt0 = (rtop & 31) + 1;
+        r = rtop - lane;
+    } else {
+        const int rbot = jl + 1;
+        blk = rbot >> 5;
+        cnt0 = 32 - (rbot & 31);
+        r = rbot + lane;
+    }
+    int e = lane < cnt0 ? (dir < 0 ? w.lc[r + 1] : w.lc[r]) : INT_MAX;
+    const bool valid = lane < cnt0 && w.kp[r] <= X;
+    int pm = warp_prefix_min(e, lane);
+    unsigned sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
+    const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid && pm > lim);
+    int fs = sm ? __ffs(sm) - 1 : 32;
+    const int fv = vm ? __ffs(vm) - 1 : 32;
+    if (fv < fs) return __shfl_sync(ROSA_FULL_MASK, pm, fv);
+    if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
+    int carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
+    for (int B0 = blk + dir;; B0 += 32 * dir) {   // ends at the window edge at the latest
+        const int B = B0 + dir * lane;
+        bool has = false;
+        if (B >= 0 && B < kNB) {
+            e = dir < 0 ? w.beL[B] : w.beR[B];
+            has = w.bkp[B] <= X;
+        } else if (B == -1 || B == kNB) {   // the edge out of the window, then unknown ranks
+            const int edge = B < 0 ? w.lc[0] : w.lc[kRWin];
+            e = edge <= lim ? edge : kNeedHard;
         } else {
-            e = r <= kRWin ? w.lc[r] : kNeedHard;
-            valid = r < kRWin && w.kp[r] <= X;
+            e = kNeedHard;
         }
-        const int pm = min(carry, warp_prefix_min(e, lane));
-        const unsigned sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
-        const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid && pm > lim);
-        const int fs = sm ? __ffs(sm) - 1 : 32;
-        const int fv = vm ? __ffs(vm) - 1 : 32;
-        if (fv < fs) return __shfl_sync(ROSA_FULL_MASK, pm, fv);
+        pm = min(carry, warp_prefix_min(e, lane));
+        sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
+        const unsigned hm = __ballot_sync(ROSA_FULL_MASK, has);
+        fs = sm ? __ffs(sm) - 1 : 32;
+        const int fh = hm ? __ffs(hm) - 1 : 32;
+        if (fh < 32 && fh <= fs) {   // the first block with an admissible key, entered above lim
+            const int before = __shfl_up_sync(ROSA_FULL_MASK, pm, 1);
+            int cin = __shfl_sync(ROSA_FULL_MASK, before, fh);
+            if (fh == 0) cin = carry;
+            const int Bh = B0 + dir * fh;
+            const int rr = dir < 0 ? 32 * Bh + 31 - lane : 32 * Bh + lane;
+            const int e2 = dir < 0 ? w.lc[rr + 1] : w.lc[rr];
+            const int pm2 = min(cin, warp_prefix_min(e2, lane));
+            const unsigned sm2 = __ballot_sync(ROSA_FULL_MASK, pm2 <= lim);
+            const unsigned vm2 = __ballot_sync(ROSA_FULL_MASK, w.kp[rr] <= X && pm2 > lim);
+            const int fs2 = sm2 ? __ffs(sm2) - 1 : 32, fv2 = vm2 ? __ffs(vm2) - 1 : 32;
+            return fv2 < fs2 ? __shfl_sync(ROSA_FULL_MASK, pm2, fv2) : 0;
+        }
         if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
         carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
     }
-    return kNeedHard;
 }
 
 // Interval of local ranks around jl whose LCP with jl is >= L.  A side that
@@ -1398,6 +1437,17 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         }
     }
     __syncthreads();
+    for (int B = warp; B < kRWin / 32; B += kRThreads / 32) {
+        const int r = 32 * B + lane;
+        int kmin = w.kp[r], el = w.lc[r + 1], er = w.lc[r];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            kmin = min(kmin, __shfl_xor_sync(ROSA_FULL_MASK, kmin, o));
+            el = min(el, __shfl_xor_sync(ROSA_FULL_MASK, el, o));
+            er = min(er, __shfl_xor_sync(ROSA_FULL_MASK, er, o));
+        }
+        if (lane == 0) { w.bkp[B] = kmin; w.beL[B] = el; w.beR[B] = er; }
+    }
     // sparse table levels, four byte entries per step with byte-wise SIMD minima
     for (int k = 1; k < kSpLevels; ++k) {
         const int h = 1 << (k - 1);
@@ -1550,20 +1600,30 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
     }
     __syncthreads();
-    // Phase D: mid-size intervals, one warp each, 32 ranks per step
+    // Phase D: mid-size intervals, 8 lanes each (4 per warp), 8 ranks per step
     const int nd = w.nd;
-    for (int di = warp; di < nd; di += kRThreads / 32) {
-        const int qi = w.bq[di];
-        const int lo = w.dlo[di], hi = w.dhi[di];
-        const int X = w.qt[qi] - G.g;
-        int best = -1;
-        for (int r = lo + lane; r <= hi; r += 32) {
-            const int c = w.kp[r];
-            if (c <= X) best = max(best, c);
-        }
+    {
+        constexpr int kSub = 8;
+        const int grp = lane / kSub, sl = lane % kSub;
+        for (int d0 = warp * (32 / kSub); d0 < nd; d0 += (kRThreads / 32) * (32 / kSub)) {
+            const int di = d0 + grp;
+            const bool act = di < nd;
+            int qi = 0, lo = 0, hi = -1, X = -1;
+            if (act) {
+                qi = w.bq[di];
+                lo = w.dlo[di];
+                hi = w.dhi[di];
+                X = w.qt[qi] - G.g;
+            }
+            int best = -1;
+            for (int r = lo + sl; r <= hi; r += kSub) {
+                const int c = w.kp[r];
+                if (c <= X) best = max(best, c);
+            }
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
-        if (lane == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
+            for (int o = kSub / 2; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
+            if (act && sl == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
+        }
     }
     // one bound task per (side, L) this tile needs beyond its window
     if (threadIdx.x < 2 * kBoundShared) {
