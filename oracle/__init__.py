@@ -15,6 +15,11 @@ Enhancing Windowed Attention with Global Recall" (arXiv 2602.02499):
 * ``match_sam`` -- the online suffix automaton of section 2.2 run in lockstep
   with the query stream (appendix B.3: tau = endpos + 1).
 * ``gather`` -- appendix C.4 read-out at tau with the Eq. (17) mask.
+* ``match_rle_brute`` / ``match_rle_sam`` -- run-level retrieval with
+  adjacent folding (section 3.3, the run-length encoding paragraph): both
+  streams folded into runs, the answer taken per query run at its start
+  time and mapped back to the start of the next key run (definition and
+  automaton forms).
 * ``match_cf_brute`` / ``match_cf_sam`` -- the per-bit counterfactual
   destinations of section 3.5: every query bit forced to 0 and to 1, one
   retrieval step each from the same historical state (definition and
@@ -57,10 +62,13 @@ def _load():
         lib.oracle_match_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
         lib.oracle_gather.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, i32p,
                                       c_int, c_int, c_int, c_int, u16p]
+        lib.oracle_match_rle_brute.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p]
+        lib.oracle_match_rle_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
         lib.oracle_match_cf_brute.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p]
         lib.oracle_match_cf_sam.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p, c_int]
         for f in (lib.oracle_discretize, lib.oracle_match_brute, lib.oracle_match_sam, lib.oracle_gather,
-                  lib.oracle_match_cf_brute, lib.oracle_match_cf_sam):
+                  lib.oracle_match_cf_brute, lib.oracle_match_cf_sam, lib.oracle_match_rle_brute,
+                  lib.oracle_match_rle_sam):
             f.restype = c_int
         _lib = lib
     return _lib
@@ -107,11 +115,9 @@ def _match(fn: str, q, k, v, g, threads=None):
     lib = _load()
     args = [_ptr(q, ctypes.c_uint8), _ptr(k, ctypes.c_uint8), _ptr(v, ctypes.c_uint8), S, T, g,
             _ptr(end, ctypes.c_int32), _ptr(ln, ctypes.c_int32), _ptr(sym, ctypes.c_int32)]
-    if fn == "sam":
+    if fn in ("sam", "rle_sam"):
         args.append(threads if threads else (os.cpu_count() or 1))
-        _check(lib.oracle_match_sam(*args), "match_sam")
-    else:
-        _check(lib.oracle_match_brute(*args), "match_brute")
+    _check(getattr(lib, "oracle_match_" + fn)(*args), "match_" + fn)
     return end, ln, sym
 
 
@@ -123,6 +129,18 @@ def match_brute(q, k, v=None, g: int = 2):
 def match_sam(q, k, v=None, g: int = 2, threads: int | None = None):
     """Online suffix-automaton matcher over host threads.  Returns (end_idx, len, sym)."""
     return _match("sam", q, k, v, g, threads)
+
+
+def match_rle_brute(q, k, v=None, g: int = 2):
+    """Run-level retrieval by the definition over runs, O(runs^2) per stream.
+    Returns per-time-step (end_idx, len, sym); tau = end_idx + 1 is the start
+    of the key run after the matched one, len counts runs."""
+    return _match("rle_brute", q, k, v, g)
+
+
+def match_rle_sam(q, k, v=None, g: int = 2, threads: int | None = None):
+    """Run-level retrieval with suffix automata over the key runs, host threads."""
+    return _match("rle_sam", q, k, v, g, threads)
 
 
 def _match_cf(fn: str, q, k, M, g, threads=None):

@@ -21,6 +21,9 @@
  *   section 3.5                    counterfactual branches: each query bit forced
  *                                  to 0 and to 1, one retrieval step each from
  *                                  the same historical state
+ *   section 3.3 (folding)          adjacent folding of repeated symbols into
+ *                                  runs; the hit maps to the start of the next
+ *                                  run (oracle_match_rle_*)
  *
  * Readings taken where the pages are garbled or silent (Eq. 16 itself is lost
  * in the page text):
@@ -512,6 +515,265 @@ int oracle_match_cf_sam(const uint8_t *q, const uint8_t *k, int S, int T, int M,
     free(th);
     free(jobs);
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Run-level retrieval with adjacent folding (section 3.3, the run-length    */
+/* encoding paragraph; appendix C.5-C.6 for the per-run bookkeeping).        */
+/*                                                                           */
+/* Consecutive equal symbols form one run.  Key runs: symbols c[l], start    */
+/* times s[l]; query runs: symbols d[m], start times u[m].  The retrieval    */
+/* state changes only at run boundaries, so the answer is taken once per     */
+/* query run, at its start time u[m], and held for every t of the run.       */
+/* A hit on key run l maps back to the time axis as the start of the next    */
+/* key run, tau = s[l+1]; it must exist and satisfy tau <= u[m] - g + 1       */
+/* (g = 2: tau <= t - 1, read strictly from the past), and this restriction  */
+/* applies before maximising, as for the plain operator.  With              */
+/*   D(m, l) = d[m] == c[l] ? 1 + D(m-1, l-1) : 0   (run-level common suffix) */
+/* the run-level length is L_m = max over admissible l of D(m, l) and l* the */
+/* largest admissible l reaching it (L_m > 0).  Outputs for t in run m:      */
+/*   end_idx[t] = s[l*+1] - 1  (the last time index of run l*, so that       */
+/*                              tau = end_idx + 1 as for the plain operator) */
+/*   len[t]     = L_m          (in runs)                                     */
+/*   sym[t]     = v[s[l*+1]]                                                 */
+/* or (-1, 0, -1) when L_m = 0.  Without adjacent repeats every run is one   */
+/* symbol long and this is the plain operator above.                        */
+/* ------------------------------------------------------------------------ */
+
+/* Runs of x[0..T): symbol and start time of each; returns their number. */
+static int fold_runs(const uint8_t *x, int T, uint8_t *rsym, int32_t *rstart)
+{
+    int n = 0;
+    for (int t = 0; t < T; ++t)
+        if (t == 0 || x[t] != x[t - 1]) {
+            rsym[n] = x[t];
+            rstart[n] = t;
+            ++n;
+        }
+    return n;
+}
+
+/* Writes run m's answer (key run lstar, run length L) to every t of the run. */
+static void rle_emit(const int32_t *u, int nq, int T, const int32_t *s, const uint8_t *v,
+                     int m, int lstar, int L, int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    int t1 = (m + 1 < nq) ? u[m + 1] : T;
+    for (int t = u[m]; t < t1; ++t) {
+        if (L > 0) {
+            int tau = s[lstar + 1];
+            end_idx[t] = tau - 1;
+            len[t] = L;
+            sym[t] = (int32_t)v[tau];
+        } else {
+            end_idx[t] = -1;
+            len[t] = 0;
+            sym[t] = -1;
+        }
+    }
+}
+
+typedef struct {
+    uint8_t *d, *c;
+    int32_t *u, *s;
+    int nq, nk;
+} runs_t;
+
+static int runs_make(runs_t *r, const uint8_t *q, const uint8_t *k, int T)
+{
+    r->d = (uint8_t *)malloc((size_t)T + 1);
+    r->c = (uint8_t *)malloc((size_t)T + 1);
+    r->u = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T + 1));
+    r->s = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T + 1));
+    if (!r->d || !r->c || !r->u || !r->s) return ORACLE_ERR_NOMEM;
+    r->nq = fold_runs(q, T, r->d, r->u);
+    r->nk = fold_runs(k, T, r->c, r->s);
+    return ORACLE_OK;
+}
+
+static void runs_free(runs_t *r)
+{
+    free(r->d); free(r->c); free(r->u); free(r->s);
+}
+
+/* Number of key runs admissible for a query run starting at time u0: runs l  */
+/* with a successor whose start s[l+1] <= u0 - g + 1 (a prefix l = 0..n-1).   */
+/* Counting resumes from `from`, a count already known to be admissible.     */
+static int rle_admissible(const runs_t *r, int u0, int g, int from)
+{
+    int n = from;
+    while (n + 1 < r->nk && r->s[n + 1] <= u0 - g + 1) ++n;
+    return n;
+}
+
+static int rle_brute_stream(const uint8_t *q, const uint8_t *k, const uint8_t *v, int T, int g,
+                            int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    runs_t r;
+    int rc = runs_make(&r, q, k, T);
+    int32_t *prev = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));
+    int32_t *cur = (int32_t *)calloc((size_t)T + 1, sizeof(int32_t));
+    if (rc || !prev || !cur) { runs_free(&r); free(prev); free(cur); return ORACLE_ERR_NOMEM; }
+    for (int m = 0; m < r.nq; ++m) {
+        for (int l = 0; l < r.nk; ++l)
+            cur[l] = (r.d[m] == r.c[l]) ? 1 + ((m > 0 && l > 0) ? prev[l - 1] : 0) : 0;
+        int nadm = rle_admissible(&r, r.u[m], g, 0);
+        int best = 0, best_l = -1;
+        for (int l = 0; l < nadm; ++l)
+            if (cur[l] > 0 && cur[l] >= best) { best = cur[l]; best_l = l; }   /* later l wins ties */
+        rle_emit(r.u, r.nq, T, r.s, v, m, best_l, best, end_idx, len, sym);
+        int32_t *tmp = prev; prev = cur; cur = tmp;
+    }
+    runs_free(&r);
+    free(prev);
+    free(cur);
+    return ORACLE_OK;
+}
+
+int oracle_match_rle_brute(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                           int S, int T, int g, int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    if (S < 0 || T < 0 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    if (!v) v = k;
+    for (int s = 0; s < S; ++s) {
+        size_t o = (size_t)s * T;
+        int rc = rle_brute_stream(q + o, k + o, v + o, T, g, end_idx + o, len + o, sym + o);
+        if (rc) return rc;
+    }
+    return ORACLE_OK;
+}
+
+/* One matching step of (state, L) with symbol c against automaton a. */
+static void sam_step(const sam_t *a, int *st, int *L, uint8_t c)
+{
+    while (*st != 0 && sam_get(a, *st, c) < 0) {
+        *st = a->link[*st];
+        *L = a->len[*st];
+    }
+    int nx = sam_get(a, *st, c);
+    if (nx >= 0) { *st = nx; *L += 1; } else { *st = 0; *L = 0; }
+}
+
+/*
+ * The automaton form (section 3.3: the automaton runs over the run-level
+ * key symbols and keeps the run start times).  An online automaton holds
+ * exactly the admissible key runs of the current query run; each query run
+ * takes one matching step.  When two or more key runs entered the automaton
+ * since the previous query run, the carried matching state may miss a
+ * longer suffix that ends in one of them, so the state is rebuilt from the
+ * root over the last U query runs, where U (the longest suffix of the query
+ * runs that occurs anywhere in the key runs) bounds the answer; U comes from
+ * a second automaton over all key runs.
+ */
+static int rle_sam_stream(const uint8_t *q, const uint8_t *k, const uint8_t *v, int T, int g,
+                          int32_t *end_idx, int32_t *len, int32_t *sym)
+{
+    runs_t r;
+    int rc = runs_make(&r, q, k, T);
+    int32_t *U = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T + 1));
+    sam_t full, on;
+    int rf = sam_init(&full, T), ro = sam_init(&on, T);
+    if (rc || !U || rf || ro) {
+        runs_free(&r); free(U); sam_free(&full); sam_free(&on);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int l = 0; l < r.nk; ++l)
+        if ((rc = sam_extend(&full, r.c[l], l))) break;
+    if (!rc) {
+        int st = 0, L = 0;
+        for (int m = 0; m < r.nq; ++m) {
+            sam_step(&full, &st, &L, r.d[m]);
+            U[m] = L;
+        }
+        int inserted = 0, prev_adm = 0;
+        st = 0;
+        L = 0;
+        for (int m = 0; m < r.nq && !rc; ++m) {
+            int nadm = rle_admissible(&r, r.u[m], g, prev_adm);
+            while (inserted < nadm && !rc) {
+                rc = sam_extend(&on, r.c[inserted], inserted);
+                ++inserted;
+            }
+            if (rc) break;
+            if (nadm - prev_adm >= 2) {
+                st = 0;
+                L = 0;
+                for (int j = (m - U[m] + 1 > 0 ? m - U[m] + 1 : 0); j <= m; ++j)
+                    sam_step(&on, &st, &L, r.d[j]);
+            } else {
+                sam_step(&on, &st, &L, r.d[m]);
+            }
+            prev_adm = nadm;
+            rle_emit(r.u, r.nq, T, r.s, v, m, L > 0 ? on.last_end[st] : -1, L, end_idx, len, sym);
+        }
+    }
+    runs_free(&r);
+    free(U);
+    sam_free(&full);
+    sam_free(&on);
+    return rc;
+}
+
+typedef int (*stream_fn_t)(const uint8_t *, const uint8_t *, const uint8_t *, int, int,
+                           int32_t *, int32_t *, int32_t *);
+
+typedef struct {
+    stream_fn_t fn;
+    const uint8_t *q, *k, *v;
+    int S, T, g, nthreads, tid;
+    int32_t *end_idx, *len, *sym;
+    int rc;
+} gen_job_t;
+
+static void *gen_worker(void *arg)
+{
+    gen_job_t *j = (gen_job_t *)arg;
+    j->rc = ORACLE_OK;
+    for (int s = j->tid; s < j->S; s += j->nthreads) {
+        size_t o = (size_t)s * j->T;
+        int rc = j->fn(j->q + o, j->k + o, j->v + o, j->T, j->g, j->end_idx + o, j->len + o, j->sym + o);
+        if (rc) { j->rc = rc; break; }
+    }
+    return NULL;
+}
+
+/* Streams ([S, T] row-major) spread over nthreads host threads. */
+static int run_streams(stream_fn_t fn, const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                       int S, int T, int g, int32_t *end_idx, int32_t *len, int32_t *sym, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > S) nthreads = S > 0 ? S : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    gen_job_t *jobs = (gen_job_t *)malloc(sizeof(gen_job_t) * nthreads);
+    if (!th || !jobs) { free(th); free(jobs); return ORACLE_ERR_NOMEM; }
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        gen_job_t jb = {fn, q, k, v, S, T, g, nthreads, i, end_idx, len, sym, 0};
+        jobs[i] = jb;
+        if (i == 0) continue;
+        if (pthread_create(&th[i], NULL, gen_worker, &jobs[i]) != 0) break;
+        started = i;
+    }
+    gen_worker(&jobs[0]);
+    int rc = jobs[0].rc;
+    for (int i = 1; i <= started; ++i) {
+        pthread_join(th[i], NULL);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    for (int i = started + 1; i < nthreads; ++i) {
+        gen_worker(&jobs[i]);
+        if (jobs[i].rc) rc = jobs[i].rc;
+    }
+    free(th);
+    free(jobs);
+    return rc;
+}
+
+int oracle_match_rle_sam(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                         int S, int T, int g, int32_t *end_idx, int32_t *len, int32_t *sym, int nthreads)
+{
+    if (S < 0 || T < 0 || g < 1 || !q || !k) return ORACLE_ERR_ARG;
+    if (!v) v = k;
+    return run_streams(rle_sam_stream, q, k, v, S, T, g, end_idx, len, sym, nthreads);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -54,3 +54,71 @@ def check_stream(q, k, v, g, end, ln, sym, full=True, sample=None, rng=None):
         for j in range(i + 1, hi + 1):
             if j - L + 1 >= 0:
                 assert not np.array_equal(k[j - L + 1:j + 1], pat), f"t={t}: later end {j} than {i}"
+
+
+def _runs(x):
+    """Run symbols, start times and the run index of every position."""
+    x = np.asarray(x, np.int64)
+    T = len(x)
+    start = np.ones(T, bool)
+    start[1:] = x[1:] != x[:-1]
+    idx = np.cumsum(start) - 1
+    st = np.flatnonzero(start)
+    return x[st], st, idx
+
+
+def check_rle_stream(q, k, v, g, end, ln, sym, full=True, sample=None, rng=None):
+    """Raise AssertionError on the first violated property of one stream of
+    run-level retrieval (adjacent folding): both streams fold into runs of
+    equal symbols, the answer is taken at each query run's start time u and
+    held over the run, key run l is admissible iff the next key run starts
+    at or before u - g + 1, and tau = end + 1 is that next run's start.
+
+    Always (every t): constant over each query run; L = 0 <=> end = -1 <=>
+    sym = -1; tau is a key-run start with tau <= u - g + 1; the L query runs
+    ending at t's run equal the L key runs ending at the run of tau - 1;
+    sym = v[tau].  With ``full`` or at ``sample`` query runs: maximality (no
+    admissible key run with a longer run-level match) and recency (no later
+    admissible key run with as long a match).
+    """
+    q = np.asarray(q, np.int64)
+    k = np.asarray(k, np.int64)
+    v = np.asarray(v, np.int64)
+    T = len(q)
+    d, u, qrun = _runs(q)
+    c, s, krun = _runs(k)
+    for t in range(T):
+        m = int(qrun[t])
+        t0 = int(u[m])
+        L, i, y = int(ln[t]), int(end[t]), int(sym[t])
+        assert (L, i, y) == (int(ln[t0]), int(end[t0]), int(sym[t0])), f"t={t}: differs from its run start {t0}"
+        if L == 0:
+            assert i == -1 and y == -1, f"t={t}: L=0 but end={i}, sym={y}"
+            continue
+        tau = i + 1
+        assert 1 <= tau <= t0 - g + 1, f"t={t}: tau={tau} not admissible for the run starting at {t0}"
+        assert k[tau] != k[tau - 1], f"t={t}: tau={tau} is not a key-run start"
+        assert y == v[tau], f"t={t}: sym={y} != v[tau]={v[tau]}"
+        lk = int(krun[tau - 1])
+        assert m - L + 1 >= 0 and lk - L + 1 >= 0, f"t={t}: match of {L} runs starts before a stream start"
+        assert np.array_equal(d[m - L + 1:m + 1], c[lk - L + 1:lk + 1]), f"t={t}: run symbols differ"
+    if full:
+        ms = range(len(d))
+    elif sample:
+        rng = rng or np.random.default_rng(0)
+        ms = rng.choice(len(d), size=min(sample, len(d)), replace=False)
+    else:
+        ms = []
+    for m in ms:
+        m = int(m)
+        t0 = int(u[m])
+        L, i = int(ln[t0]), int(end[t0])
+        adm = [l for l in range(len(c) - 1) if s[l + 1] <= t0 - g + 1]
+        lstar = int(krun[i]) if L > 0 else -1
+        for l in adm:
+            n = 0
+            while n <= m and n <= l and d[m - n] == c[l - n]:
+                n += 1
+            assert n <= L, f"run {m} (t={t0}): key run {l} matches {n} > {L} runs"
+            if L > 0:
+                assert not (n == L and l > lstar), f"run {m} (t={t0}): later key run {l} than {lstar}"
