@@ -20,6 +20,10 @@ Enhancing Windowed Attention with Global Recall" (arXiv 2602.02499):
   streams folded into runs, the answer taken per query run at its start
   time and mapped back to the start of the next key run (definition and
   automaton forms).
+* ``inject`` -- appendix C.3, Eqs. (21)-(22): the recalled bits embedded as
+  y = m((1 - b)e0 + b e1) and injected as W_out y (double precision).
+* ``ln_project`` / ``ln_project_discretize`` -- section 3.2: U = LN(H),
+  the query and key projections, then the strict threshold and packing.
 * ``match_cf_brute`` / ``match_cf_sam`` -- the per-bit counterfactual
   destinations of section 3.5: every query bit forced to 0 and to 1, one
   retrieval step each from the same historical state (definition and
@@ -44,7 +48,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared", "-fPIC",
-                               "-o", tmp, _SRC, "-lpthread"])
+                               "-o", tmp, _SRC, "-lpthread", "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -62,13 +66,17 @@ def _load():
         lib.oracle_match_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
         lib.oracle_gather.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, i32p,
                                       c_int, c_int, c_int, c_int, u16p]
+        f64p = ctypes.POINTER(ctypes.c_double)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_inject.argtypes = [i32p, u16p, u16p, u16p, c_int, c_int, c_int, c_int, c_int, f64p]
+        lib.oracle_ln_project.argtypes = [u16p, f32p, f32p, u16p, c_int, c_int, c_int, ctypes.c_double, f64p, f64p]
         lib.oracle_match_rle_brute.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p]
         lib.oracle_match_rle_sam.argtypes = [u8p, u8p, u8p, c_int, c_int, c_int, i32p, i32p, i32p, c_int]
         lib.oracle_match_cf_brute.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p]
         lib.oracle_match_cf_sam.argtypes = [u8p, u8p, c_int, c_int, c_int, c_int, i32p, i32p, c_int]
         for f in (lib.oracle_discretize, lib.oracle_match_brute, lib.oracle_match_sam, lib.oracle_gather,
                   lib.oracle_match_cf_brute, lib.oracle_match_cf_sam, lib.oracle_match_rle_brute,
-                  lib.oracle_match_rle_sam):
+                  lib.oracle_match_rle_sam, lib.oracle_inject, lib.oracle_ln_project):
             f.restype = c_int
         _lib = lib
     return _lib
@@ -195,3 +203,60 @@ def gather(V_bits: np.ndarray, end_idx: np.ndarray, R: int, d: int, rho: int) ->
     _check(_load().oracle_gather(_ptr(V_bits, ctypes.c_uint16), Cv, rho, _ptr(end_idx, ctypes.c_int32),
                                  B, R, T, d, _ptr(out, ctypes.c_uint16)), "gather")
     return out
+
+
+def inject(sym: np.ndarray, e0_bits: np.ndarray, e1_bits: np.ndarray, W_bits: np.ndarray, B: int, R: int,
+           M: int) -> np.ndarray:
+    """Read-out embedding and injection (appendix C.3).  ``sym``: int32
+    ``[B*R, T]`` recalled value symbols (-1: no match); ``e0_bits``,
+    ``e1_bits``: uint16 ``[C]`` (C = R*M, bf16 bits); ``W_bits``: uint16
+    ``[D, C]``.  Returns float64 ``[B, T, D]``."""
+    sym = np.ascontiguousarray(sym, dtype=np.int32)
+    e0 = np.ascontiguousarray(e0_bits, dtype=np.uint16)
+    e1 = np.ascontiguousarray(e1_bits, dtype=np.uint16)
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    if sym.ndim != 2 or sym.shape[0] != B * R:
+        raise ValueError("sym must be [B*R, T]")
+    T = sym.shape[1]
+    C = R * M
+    if e0.shape != (C,) or e1.shape != (C,) or W.ndim != 2 or W.shape[1] != C:
+        raise ValueError("e0, e1 must be [C] and W [D, C] with C = R*M")
+    D = W.shape[0]
+    out = np.empty((B, T, D), np.float64)
+    _check(_load().oracle_inject(_ptr(sym, ctypes.c_int32), _ptr(e0, ctypes.c_uint16), _ptr(e1, ctypes.c_uint16),
+                                 _ptr(W, ctypes.c_uint16), B, R, M, T, D, _ptr(out, ctypes.c_double)), "inject")
+    return out
+
+
+def ln_project(H_bits: np.ndarray, W_bits: np.ndarray, gamma=None, beta=None, eps: float = 1e-5):
+    """U = LN(H) then U W (section 3.2), double precision.  ``H_bits``: uint16
+    ``[rows, D]``; ``W_bits``: uint16 ``[D, N]``; ``gamma``, ``beta``: float32
+    ``[D]`` or None.  Returns (P ``[rows, N]``, A ``[rows, N]``) with
+    A = sum_k |u_k W[k, n]| (the scale of rounding errors in P)."""
+    H = np.ascontiguousarray(H_bits, dtype=np.uint16)
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, D = H.shape
+    if W.shape[0] != D:
+        raise ValueError("W must be [D, N]")
+    N = W.shape[1]
+    g = None if gamma is None else np.ascontiguousarray(gamma, dtype=np.float32)
+    b = None if beta is None else np.ascontiguousarray(beta, dtype=np.float32)
+    out = np.empty((rows, N), np.float64)
+    mag = np.empty((rows, N), np.float64)
+    f32 = ctypes.POINTER(ctypes.c_float)
+    _check(_load().oracle_ln_project(_ptr(H, ctypes.c_uint16), _ptr(g, ctypes.c_float) if g is not None
+                                     else ctypes.cast(None, f32), _ptr(b, ctypes.c_float) if b is not None
+                                     else ctypes.cast(None, f32), _ptr(W, ctypes.c_uint16), rows, D, N, float(eps),
+                                     _ptr(out, ctypes.c_double), _ptr(mag, ctypes.c_double)), "ln_project")
+    return out, mag
+
+
+def pack_bits(P: np.ndarray, B: int, T: int, M: int) -> np.ndarray:
+    """Strict threshold and multi-route packing of section 3.2 (Eqs. 10-15)
+    on real values ``P`` ``[B*T, C]``: symbols ``[B, C//M, T]``."""
+    C = P.shape[1]
+    bits = (P > 0).astype(np.uint8).reshape(B, T, C // M, M)
+    sym = np.zeros((B, T, C // M), np.uint8)
+    for j in range(M):
+        sym += bits[..., j] << j
+    return np.ascontiguousarray(sym.transpose(0, 2, 1))

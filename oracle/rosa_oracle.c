@@ -24,6 +24,10 @@
  *   section 3.3 (folding)          adjacent folding of repeated symbols into
  *                                  runs; the hit maps to the start of the next
  *                                  run (oracle_match_rle_*)
+ *   appendix C.3, Eqs. (21)-(22)   read-out embedding y = m((1-b)e0 + b e1) and
+ *                                  injection inj = W_out y (oracle_inject)
+ *   section 3.2 (before Eq. 10)    U = LN(H), Q = U W_q, K = U W_k before the
+ *                                  threshold (oracle_ln_project)
  *
  * Readings taken where the pages are garbled or silent (Eq. 16 itself is lost
  * in the page text):
@@ -40,6 +44,7 @@
  * online suffix automaton over the key stream, advanced in lockstep with the
  * query stream.  The two share nothing but the output convention.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -655,60 +660,48 @@ static void sam_step(const sam_t *a, int *st, int *L, uint8_t c)
 
 /*
  * The automaton form (section 3.3: the automaton runs over the run-level
- * key symbols and keeps the run start times).  An online automaton holds
- * exactly the admissible key runs of the current query run; each query run
- * takes one matching step.  When two or more key runs entered the automaton
- * since the previous query run, the carried matching state may miss a
- * longer suffix that ends in one of them, so the state is rebuilt from the
- * root over the last U query runs, where U (the longest suffix of the query
- * runs that occurs anywhere in the key runs) bounds the answer; U comes from
- * a second automaton over all key runs.
+ * key symbols and keeps the run start times).  The online automaton holds
+ * exactly the key runs admissible so far, and the matching state (state, L)
+ * is the longest suffix of the query runs seen so far that occurs in it.
+ * Before query run m takes its matching step, the key runs that became
+ * admissible since the previous query run enter one by one; each can only
+ * add occurrences that end in itself, so after inserting run l the state is
+ * raised to the suffix of length D (the run-level common suffix of the query
+ * runs so far and the key runs 0..l, compared directly) when D >= L: that
+ * suffix is a suffix of the whole key-run prefix, so its state lies on the
+ * suffix-link chain of the newest state.  Then the query run's symbol takes
+ * one ordinary matching step, and last_end of the state is the most recent
+ * admissible key run l*.
  */
 static int rle_sam_stream(const uint8_t *q, const uint8_t *k, const uint8_t *v, int T, int g,
                           int32_t *end_idx, int32_t *len, int32_t *sym)
 {
     runs_t r;
     int rc = runs_make(&r, q, k, T);
-    int32_t *U = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T + 1));
-    sam_t full, on;
-    int rf = sam_init(&full, T), ro = sam_init(&on, T);
-    if (rc || !U || rf || ro) {
-        runs_free(&r); free(U); sam_free(&full); sam_free(&on);
-        return ORACLE_ERR_NOMEM;
-    }
-    for (int l = 0; l < r.nk; ++l)
-        if ((rc = sam_extend(&full, r.c[l], l))) break;
-    if (!rc) {
-        int st = 0, L = 0;
-        for (int m = 0; m < r.nq; ++m) {
-            sam_step(&full, &st, &L, r.d[m]);
-            U[m] = L;
-        }
-        int inserted = 0, prev_adm = 0;
-        st = 0;
-        L = 0;
-        for (int m = 0; m < r.nq && !rc; ++m) {
-            int nadm = rle_admissible(&r, r.u[m], g, prev_adm);
-            while (inserted < nadm && !rc) {
-                rc = sam_extend(&on, r.c[inserted], inserted);
-                ++inserted;
-            }
+    sam_t on;
+    int ro = sam_init(&on, T);
+    if (rc || ro) { runs_free(&r); sam_free(&on); return ORACLE_ERR_NOMEM; }
+    int st = 0, L = 0, inserted = 0;
+    for (int m = 0; m < r.nq && !rc; ++m) {
+        int nadm = rle_admissible(&r, r.u[m], g, inserted);
+        while (inserted < nadm && !rc) {
+            int l = inserted++;
+            rc = sam_extend(&on, r.c[l], l);
             if (rc) break;
-            if (nadm - prev_adm >= 2) {
-                st = 0;
-                L = 0;
-                for (int j = (m - U[m] + 1 > 0 ? m - U[m] + 1 : 0); j <= m; ++j)
-                    sam_step(&on, &st, &L, r.d[j]);
-            } else {
-                sam_step(&on, &st, &L, r.d[m]);
+            int D = 0;   /* common suffix of d[0..m-1] and c[0..l] */
+            while (D < m && D <= l && r.d[m - 1 - D] == r.c[l - D]) ++D;
+            if (D > 0 && D >= L) {
+                int x = on.last;
+                while (on.link[x] > 0 && on.len[on.link[x]] >= D) x = on.link[x];
+                st = x;
+                L = D;
             }
-            prev_adm = nadm;
-            rle_emit(r.u, r.nq, T, r.s, v, m, L > 0 ? on.last_end[st] : -1, L, end_idx, len, sym);
         }
+        if (rc) break;
+        sam_step(&on, &st, &L, r.d[m]);
+        rle_emit(r.u, r.nq, T, r.s, v, m, L > 0 ? on.last_end[st] : -1, L, end_idx, len, sym);
     }
     runs_free(&r);
-    free(U);
-    sam_free(&full);
     sam_free(&on);
     return rc;
 }
@@ -802,5 +795,99 @@ int oracle_gather(const uint16_t *V, int64_t v_row_stride, int64_t rho,
                     for (int m = 0; m < d; ++m) dst[m] = src[m];
                 }
             }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Read-out embedding and injection (appendix C.3; Eq. 17 mask).             */
+/*                                                                           */
+/* For position (b, t) and channel c = r*M + j of route r: the recalled bit  */
+/* b^ = bit j of the recalled value symbol sym[b*R + r, t], the mask         */
+/* m = I[tau >= 0] (sym = -1 when nothing matched), and                      */
+/*   y[b, t, c]   = m * ((1 - b^) e0[c] + b^ e1[c])                          */
+/*   inj[b, t, d] = sum_c W_out[d, c] * y[b, t, c]                           */
+/* in double precision.  e0, e1: [C] bf16 bits; W_out: [D, C] bf16 bits,     */
+/* row-major; out: [B, T, D] doubles.                                        */
+/* ------------------------------------------------------------------------ */
+
+int oracle_inject(const int32_t *sym, const uint16_t *e0, const uint16_t *e1, const uint16_t *W,
+                  int B, int R, int M, int T, int D, double *out)
+{
+    if (B < 0 || R < 0 || T < 0 || D < 0 || M < 1 || M > 8) return ORACLE_ERR_ARG;
+    int C = R * M;
+    double *y = (double *)malloc(sizeof(double) * (C > 0 ? C : 1));
+    if (!y) return ORACLE_ERR_NOMEM;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            for (int r = 0; r < R; ++r) {
+                int32_t a = sym[((size_t)b * R + r) * T + t];
+                for (int j = 0; j < M; ++j) {
+                    int c = r * M + j;
+                    if (a < 0) {
+                        y[c] = 0.0;   /* m = 0 */
+                    } else {
+                        int bit = (a >> j) & 1;
+                        double v0 = bf16_bits_to_float(e0[c]), v1 = bf16_bits_to_float(e1[c]);
+                        y[c] = (1 - bit) * v0 + bit * v1;
+                    }
+                }
+            }
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int c = 0; c < C; ++c)
+                    acc += (double)bf16_bits_to_float(W[(size_t)d * C + c]) * y[c];
+                out[((size_t)b * T + t) * D + d] = acc;
+            }
+        }
+    free(y);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Layer norm and projection before the threshold (section 3.2).             */
+/*                                                                           */
+/* U = LN(H): per row, mu = mean(h), var = mean((h - mu)^2) (population),    */
+/* u = gamma * (h - mu) / sqrt(var + eps) + beta; then the projection         */
+/* P = U W with W: [D, N] (the query and key projections side by side), in   */
+/* double precision.  Also returns, per entry, the magnitude                 */
+/* A[row, n] = sum_k |u_k W[k, n]| that bounds how far a rounded evaluation  */
+/* of P can stray.  H: [rows, D] bf16 bits; gamma, beta: [D] floats (NULL:   */
+/* 1 and 0); out, mag: [rows, N] doubles.                                    */
+/* ------------------------------------------------------------------------ */
+
+int oracle_ln_project(const uint16_t *H, const float *gamma, const float *beta, const uint16_t *W,
+                      int rows, int D, int N, double eps, double *out, double *mag)
+{
+    if (rows < 0 || D < 1 || N < 0 || eps < 0.0) return ORACLE_ERR_ARG;
+    double *u = (double *)malloc(sizeof(double) * D);
+    if (!u) return ORACLE_ERR_NOMEM;
+    for (int i = 0; i < rows; ++i) {
+        const uint16_t *h = H + (size_t)i * D;
+        double mu = 0.0;
+        for (int k = 0; k < D; ++k) mu += bf16_bits_to_float(h[k]);
+        mu /= D;
+        double var = 0.0;
+        for (int k = 0; k < D; ++k) {
+            double x = bf16_bits_to_float(h[k]) - mu;
+            var += x * x;
+        }
+        var /= D;
+        double rstd = 1.0 / sqrt(var + eps);
+        for (int k = 0; k < D; ++k) {
+            double g = gamma ? gamma[k] : 1.0, bb = beta ? beta[k] : 0.0;
+            u[k] = g * (bf16_bits_to_float(h[k]) - mu) * rstd + bb;
+        }
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0, a = 0.0;
+            for (int k = 0; k < D; ++k) {
+                double term = u[k] * bf16_bits_to_float(W[(size_t)k * N + n]);
+                acc += term;
+                a += fabs(term);
+            }
+            out[(size_t)i * N + n] = acc;
+            if (mag) mag[(size_t)i * N + n] = a;
+        }
+    }
+    free(u);
     return ORACLE_OK;
 }
