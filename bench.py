@@ -59,6 +59,12 @@ def parse():
     ap.add_argument("--split", default="streams", choices=["streams", "replicas"],
                     help="N > 1: split one workload's streams over the ranks (strong scaling, default) "
                          "or give every rank a full copy with shifted seeds (weak scaling)")
+    ap.add_argument("--rle", action="store_true",
+                    help="time the run-level operator (adjacent folding of repeated symbols, section 3.3) "
+                         "as the match step")
+    ap.add_argument("--cf", action="store_true",
+                    help="time the counterfactual op (ordinary retrieval plus every query bit forced to 0 and "
+                         "to 1, section 3.5; M = log2 K bits) as the match step")
     ap.add_argument("--streams", type=int, default=0,
                     help="profiling aid: keep only the first N streams of a symbol workload")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel eagerly instead of graph replay")
@@ -192,6 +198,9 @@ def algorithmic_bytes(wl):
         out["discretize"] = 2 * (B * T * C * 2 + B * (C // wl["M"]) * T)
     # q (1 B) + k (1 B, unless q = k) + three int32 outputs
     out["match"] = S * T * ((1 if wl["same"] else 2) + 12)
+    if wl.get("cf"):
+        # plus three int32 outputs per (bit, forced value) of the counterfactual tables
+        out["match"] += S * T * wl["M_cf"] * 2 * 12
     if "gather" in wl["ops"]:
         # end_idx (4 B) + d bf16 read + d bf16 written per (position, route)
         out["gather"] = wl["B"] * T * wl["R"] * (4 + 2 * wl["d"] * 2)
@@ -206,8 +215,16 @@ class Runner:
         import suffix_automaton_retrieval_b200.binding as rosa
         self.rosa, self.wl, self.torch = rosa, wl, torch
         S, T = wl["S"], wl["T"]
-        self.ws = rosa.alloc_workspace(S, T, wl["K"], device)
+        if wl.get("rle"):
+            self.ws = torch.empty(rosa.match_rle_workspace_size(S, T, wl["K"]), dtype=torch.uint8, device=device)
+        elif wl.get("cf"):
+            self.ws = torch.empty(rosa.match_cf_workspace_size(S, T, wl["M_cf"]), dtype=torch.uint8, device=device)
+        else:
+            self.ws = rosa.alloc_workspace(S, T, wl["K"], device)
         self.outs = tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))
+        if wl.get("cf"):
+            self.outs += tuple(torch.empty((S, T, wl["M_cf"], 2), dtype=torch.int32, device=device)
+                               for _ in range(3))
         if "discretize" in wl["ops"]:
             B, _, C = wl["qvec"].shape
             self.sq = torch.empty((B, C // wl["M"], T), dtype=torch.uint8, device=device)
@@ -221,7 +238,9 @@ class Runner:
         torch, wl = self.torch, self.wl
         torch.cuda.synchronize()
         bits = lambda t: t.cpu().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
-        out = {"match": tuple(o.cpu().numpy() for o in self.outs)}
+        out = {"match": tuple(o.cpu().numpy() for o in self.outs[:3])}
+        if wl.get("cf"):
+            out["cf"] = tuple(o.cpu().numpy() for o in self.outs[3:])
         if "discretize" in wl["ops"]:
             out["discretize"] = (self.sq.cpu().numpy(), self.sk.cpu().numpy())
         if "gather" in wl["ops"]:
@@ -231,7 +250,11 @@ class Runner:
 
     def launches(self):
         wl = self.wl
-        n = self.rosa.match_launch_count(wl["S"], wl["T"], wl["K"], wl["same"])
+        if wl.get("cf"):
+            n = self.rosa.match_cf_launch_count(wl["S"], wl["T"], wl["M_cf"], wl["same"])
+        else:
+            count = self.rosa.match_rle_launch_count if wl.get("rle") else self.rosa.match_launch_count
+            n = count(wl["S"], wl["T"], wl["K"], wl["same"])
         n += 1 if "discretize" in wl["ops"] else 0
         n += 1 if "gather" in wl["ops"] else 0
         return n
@@ -245,7 +268,12 @@ class Runner:
                 q, k = self.sq.view(wl["S"], wl["T"]), self.sk.view(wl["S"], wl["T"])
             else:
                 q, k = wl["q"], wl["k"]
-            rosa.match(q, None if wl["same"] else k, K=wl["K"], g=wl["g"], out=self.outs, workspace=self.ws)
+            if wl.get("cf"):
+                rosa.match_cf(q, None if wl["same"] else k, M=wl["M_cf"], g=wl["g"], out=self.outs,
+                              workspace=self.ws)
+            else:
+                fn = rosa.match_rle if wl.get("rle") else rosa.match
+                fn(q, None if wl["same"] else k, K=wl["K"], g=wl["g"], out=self.outs[:3], workspace=self.ws)
         elif name == "gather":
             rosa.gather(wl["V"], self.outs[0], wl["R"], wl["d"], wl["rho"], out=self.gout)
 
@@ -412,12 +440,19 @@ def cpu_oracle_baseline(wl, target_seconds=(10.0, 30.0), forced_streams=0, keep_
     (the first n), which the parity check compares with the GPU's."""
     import oracle
     q, k, disc = oracle_symbols(wl)
+    match_fn = oracle.match_rle_sam if wl.get("rle") else oracle.match_sam
+    kind = "run-level suffix automata" if wl.get("rle") else "online suffix automaton"
+    if wl.get("cf"):
+        def match_fn(qq, kk, g, threads):   # noqa: E306 - the counterfactual tables and the ordinary result
+            return oracle.match_cf_sam(qq, kk, wl["M_cf"], g=g, threads=threads) + \
+                oracle.match_sam(qq, kk, g=g, threads=threads)
+        kind = "online suffix automaton, every query bit forced both ways"
     cores = os.cpu_count() or 1
     S = wl["S"]
     n = forced_streams or min(S, cores)
     while True:
         t0 = time.perf_counter()
-        res = oracle.match_sam(q[:n], k[:n] if not wl["same"] else q[:n], g=wl["g"], threads=cores)
+        res = match_fn(q[:n], k[:n] if not wl["same"] else q[:n], g=wl["g"], threads=cores)
         dt = time.perf_counter() - t0
         if forced_streams or dt >= target_seconds[0] or n >= S:
             break
@@ -427,15 +462,20 @@ def cpu_oracle_baseline(wl, target_seconds=(10.0, 30.0), forced_streams=0, keep_
     m, dt1 = 0, 0.0
     while m < S and (m == 0 or dt1 < 1.0):
         t1 = time.perf_counter()
-        oracle.match_sam(q[m:m + 1], k[m:m + 1] if not wl["same"] else q[m:m + 1], g=wl["g"], threads=1)
+        match_fn(q[m:m + 1], k[m:m + 1] if not wl["same"] else q[m:m + 1], g=wl["g"], threads=1)
         dt1 += time.perf_counter() - t1
         m += 1
     out = {"value": n * wl["T"] / dt, "unit": UNIT, "cores": used, "kind": "oracle",
-           "sample": f"{n} of {S} streams x T={wl['T']} (full length), online suffix automaton, "
+           "sample": f"{n} of {S} streams x T={wl['T']} (full length), {kind}, "
                      f"{used} threads, {dt:.1f} s", "seconds": dt,
            "single_core": {"value": m * wl["T"] / dt1, "unit": UNIT, "cores": 1,
                            "sample": f"{m} streams x T={wl['T']}, one thread, {dt1:.1f} s"}}
     if keep_outputs:
+        if wl.get("cf"):
+            vk = (k[:n] if not wl["same"] else q[:n]).astype(np.int32)
+            e = res[0].reshape(n, -1)
+            ycf = np.where(e >= 0, np.take_along_axis(vk, np.maximum(e + 1, 0), axis=1), -1).reshape(res[0].shape)
+            return out, {"n": n, "match": res[2:], "cf": (res[0], res[1], ycf), "discretize": disc}
         return out, {"n": n, "match": res, "discretize": disc}
     return out
 
@@ -473,6 +513,11 @@ def check_parity(wl, got, ref):
         if not np.array_equal(a[:n], b):
             return False, f"match {name} differs at {_first_diff(a[:n], b)}"
     checked.append(f"match ({n} of {wl['S']} streams)")
+    if "cf" in ref:
+        for name, a, b in zip(("end_cf", "len_cf", "sym_cf"), got["cf"], ref["cf"]):
+            if not np.array_equal(a[:n], b):
+                return False, f"counterfactual {name} differs at {_first_diff(a[:n], b)}"
+        checked.append("counterfactual tables")
     if "gather" in got and n == wl["S"]:
         R, d, rho = wl["R"], wl["d"], wl["rho"]
         end = ref["match"][0]
@@ -516,6 +561,12 @@ def main():
                         shard=None if replicas else (world, rank))
     if args.streams and wl["cfg"] != 3 and args.streams < wl["S"]:
         shrink_streams(wl, args.streams)
+    wl["rle"] = args.rle
+    wl["cf"] = args.cf
+    if args.cf:
+        wl["M_cf"] = max(1, (wl["K"] - 1).bit_length())
+        if 1 << wl["M_cf"] != wl["K"]:
+            raise SystemExit("--cf needs an alphabet of 2^M symbols")
     runner = Runner(wl, device)
     ab = algorithmic_bytes(wl)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -575,7 +626,7 @@ def main():
                 "ms": round(mean_op[dom], 4), "ops_ms": {o: round(v, 4) for o, v in mean_op.items()}}
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.cf:   # the counterfactual op is measured on the device only
         e2e = end_to_end(wl, device, args.steps)
         # every rank takes the same collective steps
         e_ms, e_units = reduce_over_ranks(e2e["ms_per_step"] * args.steps, positions * args.steps, device)
@@ -599,6 +650,9 @@ def main():
             "config": {"workload": wl["name"], "streams": wl["S"],
                        "streams_per_rank": wl["S"], "T": wl["T"], "K": wl["K"], "g": wl["g"],
                        "q_equals_k": wl["same"], "ops": wl["ops"],
+                       "operator": ("run-level: adjacent folding, answered per query run" if args.rle
+                                    else (f"counterfactual: ordinary plus {wl.get('M_cf')} query bits forced "
+                                          "both ways" if args.cf else "plain: longest suffix match per position")),
                        "parallelism": (f"{world} replicas (weak)" if replicas else
                                        f"streams split over {world} rank(s), no exchange (strong)"),
                        "shard_rank0": wl.get("shard"),
@@ -641,8 +695,9 @@ def end_to_end(wl, device, steps):
             hin.append(torch.from_numpy(wl["k_host"]).pin_memory())
 
     def make_set():
-        b = {"din": [torch.empty_like(h, device=device) for h in hin],
-             "ws": rosa.alloc_workspace(S, T, wl["K"], device),
+        ws = (torch.empty(rosa.match_rle_workspace_size(S, T, wl["K"]), dtype=torch.uint8, device=device)
+              if wl.get("rle") else rosa.alloc_workspace(S, T, wl["K"], device))
+        b = {"din": [torch.empty_like(h, device=device) for h in hin], "ws": ws,
              "outs": tuple(torch.empty((S, T), dtype=torch.int32, device=device) for _ in range(3))}
         if "gather" in wl["ops"]:
             b["gout"] = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
@@ -664,7 +719,8 @@ def end_to_end(wl, device, steps):
         else:
             q = din[0]
             k = None if wl["same"] else din[1]
-        e, l, s = rosa.match(q, k, K=wl["K"], g=wl["g"], out=b["outs"], workspace=b["ws"])
+        fn = rosa.match_rle if wl.get("rle") else rosa.match
+        e, l, s = fn(q, k, K=wl["K"], g=wl["g"], out=b["outs"], workspace=b["ws"])
         if "gather" in wl["ops"]:
             rosa.gather(din[-1], e, wl["R"], wl["d"], wl["rho"], out=b["gout"])
             hout[0].copy_(b["gout"], non_blocking=True)
@@ -734,11 +790,12 @@ def run_reference(args, rank, world):
                           "qwen-proj-64 needs the GPU projection set-up; reference arm runs on symbol workloads"}))
         return 0
     sw = W.WORKLOADS[cfg]["make"]()
+    match_fn = oracle.match_rle_sam if args.rle else oracle.match_sam
     cores = os.cpu_count() or 1
     n = args.cpu_sample_streams or min(sw.S, cores)
     # size the per-step sample so the whole run stays within a few minutes
     t0 = time.perf_counter()
-    oracle.match_sam(sw.q[:n], sw.k[:n] if not sw.same_qk else sw.q[:n], g=sw.g, threads=cores)
+    match_fn(sw.q[:n], sw.k[:n] if not sw.same_qk else sw.q[:n], g=sw.g, threads=cores)
     probe = time.perf_counter() - t0
     budget = 150.0 / max(1, args.steps + args.warmup)
     while probe * 2 < budget and n * 2 <= sw.S:
@@ -749,11 +806,11 @@ def run_reference(args, rank, world):
         probe /= 2
     qs, ks = sw.q[:n], (sw.q[:n] if sw.same_qk else sw.k[:n])
     for _ in range(args.warmup):
-        oracle.match_sam(qs, ks, g=sw.g, threads=cores)
+        match_fn(qs, ks, g=sw.g, threads=cores)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.match_sam(qs, ks, g=sw.g, threads=cores)
+        match_fn(qs, ks, g=sw.g, threads=cores)
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = n * sw.T * args.steps / total

@@ -124,11 +124,75 @@ ROSA_API int rosa_match(const uint8_t *q, const uint8_t *k, const uint8_t *v,
 ROSA_API int rosa_match_launch_count(int S, int T, int K, int q_is_k);
 
 /*
- * Reads the device status word a previous rosa_match left in `workspace`
- * (0 = no device-side check fired, otherwise a bit set of ROSA_DEV_*).
+ * Per-bit counterfactual destinations (section 3.5: every query bit is a
+ * discrete decision switch; the branches "force the bit to 0" and "force
+ * it to 1" each take one retrieval step from the same history; appendix
+ * C.5 precomputes tau^(0), tau^(1) for the gradients).
+ *
+ * Symbols carry M bits (K = 2^M, 1 <= M <= 8).  For position t, bit j < M
+ * and beta in {0, 1}, the branch symbol is q[s, t] with bit j set to beta;
+ * q[s, 0..t-1] and the keys stay as they are, and the branch's destination
+ * is the ordinary retrieval of that symbol (longest admissible match ending
+ * at t, most recent end, same lag g).  The branch that keeps the actual bit
+ * is the ordinary result, which is also returned:
+ *   end_idx, len, sym  [S, T]        as rosa_match
+ *   end_cf, len_cf, sym_cf [S, T, M, 2] int32, beta last:
+ *     end_cf[s, t, j, beta] = i*' (-1 if no match), len_cf = L',
+ *     sym_cf = v[s, i*' + 1] (-1 if no match)
+ * All outputs are written in full.  Requires 1 <= M <= 8, g >= 1,
+ * S*T*(2+M) < 2^31 and symbols < 2^M; workspace of at least
+ * rosa_match_cf_workspace_size(S, T, M) bytes, 256-byte aligned (status
+ * word read with rosa_match_device_status).  Key-bit branches are not
+ * computed.
+ */
+ROSA_API size_t rosa_match_cf_workspace_size(int S, int T, int M);
+ROSA_API int rosa_match_cf(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                           int S, int T, int M, int g,
+                           int32_t *end_idx, int32_t *len, int32_t *sym,
+                           int32_t *end_cf, int32_t *len_cf, int32_t *sym_cf,
+                           void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Kernel launches one rosa_match_cf call enqueues (-1 for invalid sizes). */
+ROSA_API int rosa_match_cf_launch_count(int S, int T, int M, int q_is_k);
+
+/*
+ * Run-level retrieval with adjacent folding (section 3.3, the run-length
+ * encoding paragraph; appendix C.5-C.6 for the per-run bookkeeping).
+ *
+ * Consecutive equal symbols of a stream form one run; both q and k fold.
+ * Key runs have symbols c_l and start times s_l, query runs d_m and u_m.
+ * The retrieval moves only at run boundaries: query run m is answered once,
+ * at its start time u_m, and every t of the run reports that answer.  Key
+ * run l is admissible iff the next key run starts at s_{l+1} <= u_m - g + 1
+ * (g = 2: tau <= t - 1, read strictly from the past).  With L the longest
+ * run-level common suffix of d_0..d_m and c_0..c_l over admissible l, and
+ * l* the largest admissible l reaching it, for every t of query run m:
+ *   end_idx[s, t] = s_{l*+1} - 1   (-1 if L = 0)   -- tau = end_idx + 1 is
+ *                                    the start of the key run after l*
+ *   len[s, t]     = L              (counted in runs)
+ *   sym[s, t]     = v[s, s_{l*+1}]  (-1 if L = 0)
+ * Without adjacent repeats every run is one symbol and this is rosa_match.
+ * Shapes, ownership and errors as for rosa_match; the workspace is at least
+ * rosa_match_rle_workspace_size(S, T, K) bytes (256-byte aligned) and its
+ * status word is read with rosa_match_device_status.
+ */
+ROSA_API size_t rosa_match_rle_workspace_size(int S, int T, int K);
+ROSA_API int rosa_match_rle(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                            int S, int T, int K, int g,
+                            int32_t *end_idx, int32_t *len, int32_t *sym,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Kernel launches one rosa_match_rle call enqueues (-1 for invalid sizes). */
+ROSA_API int rosa_match_rle_launch_count(int S, int T, int K, int q_is_k);
+
+/*
+ * Reads the device status word a previous rosa_match (or rosa_match_rle)
+ * left in `workspace` (0 = no device-side check fired, otherwise a bit set
+ * of ROSA_DEV_*).
  * Synchronises `stream`.  Returns ROSA_OK or ROSA_ERR_CUDA.
  */
 #define ROSA_DEV_SYMBOL_RANGE 1u   /* some input symbol was >= K */
+#define ROSA_DEV_TIMEOUT 2u        /* a bounded wait inside a kernel ran out */
 ROSA_API int rosa_match_device_status(const void *workspace, cudaStream_t stream, uint32_t *status);
 
 /*
@@ -168,6 +232,27 @@ ROSA_API int rosa_match_noalloc(const uint8_t *q, const uint8_t *k, const uint8_
  * ROSA_ERR_CUDA.
  */
 ROSA_API int rosa_match_noalloc_device_status(cudaStream_t stream, uint32_t *status);
+
+/*
+ * Read-out embedding and injection (appendix C.3, Eqs. 21-22 of the main
+ * text, with the Eq. 17 mask), on the tensor cores.
+ *
+ *   sym    [B*R, T] int32: the recalled value symbol of route r at position
+ *          t (rosa_match's sym output; -1 where nothing matched).
+ *   e0, e1 [C] bf16, C = R*M: the embedding of a recalled 0 / 1 bit.
+ *   W_out  [D, C] bf16, row-major.
+ *   inj    [B, T, D] bf16, written in full:
+ *     y[b, t, r*M + j] = m * ((1 - bit_j) * e0[r*M + j] + bit_j * e1[r*M + j])
+ *       with bit_j = (sym >> j) & 1 and m = I[sym >= 0];
+ *     inj[b, t, d] = bf16(sum_c W_out[d, c] * y[b, t, c])  (fp32 accumulation)
+ * dev_status: optional device word; ROSA_DEV_TIMEOUT is or-ed into it if a
+ * kernel's bounded wait ran out (the affected tiles are not written).
+ * Requires B, T >= 0, 1 <= M <= 8, R >= 1, D >= 1; any alignment (rows of
+ * W_out that are 16-byte aligned take the vector path).
+ */
+ROSA_API int rosa_inject(const int32_t *sym, const rosa_bf16 *e0, const rosa_bf16 *e1, const rosa_bf16 *W_out,
+                         int B, int R, int M, int T, int D, rosa_bf16 *inj, uint32_t *dev_status,
+                         cudaStream_t stream);
 
 /*
  * Read-out of value rows at tau (appendix C.4 with the Eq. 17 mask).

@@ -35,15 +35,31 @@ lib.rosa_match_workspace_size.argtypes = [_i, _i, _i]
 lib.rosa_match_workspace_size.restype = ctypes.c_size_t
 lib.rosa_match.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.rosa_match.restype = _i
+lib.rosa_match_cf_workspace_size.argtypes = [_i, _i, _i]
+lib.rosa_match_cf_workspace_size.restype = ctypes.c_size_t
+lib.rosa_match_cf.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.rosa_match_cf.restype = _i
+lib.rosa_match_cf_launch_count.argtypes = [_i, _i, _i, _i]
+lib.rosa_match_cf_launch_count.restype = _i
+lib.rosa_match_rle_workspace_size.argtypes = [_i, _i, _i]
+lib.rosa_match_rle_workspace_size.restype = ctypes.c_size_t
+lib.rosa_match_rle.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.rosa_match_rle.restype = _i
+lib.rosa_match_rle_launch_count.argtypes = [_i, _i, _i, _i]
+lib.rosa_match_rle_launch_count.restype = _i
 lib.rosa_match_launch_count.argtypes = [_i, _i, _i, _i]
 lib.rosa_match_launch_count.restype = _i
 lib.rosa_match_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
 lib.rosa_match_device_status.restype = _i
+lib.rosa_inject.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]
+lib.rosa_inject.restype = _i
 lib.rosa_gather.argtypes = [_vp, _i64, _i64, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.rosa_gather.restype = _i
 
 EXPORTED = ("rosa_status_string", "rosa_discretize", "rosa_discretize_pair", "rosa_match_workspace_size", "rosa_match",
-            "rosa_match_launch_count", "rosa_match_device_status", "rosa_gather")
+            "rosa_match_launch_count", "rosa_match_device_status", "rosa_gather", "rosa_match_rle",
+            "rosa_match_rle_workspace_size", "rosa_match_rle_launch_count", "rosa_match_cf",
+            "rosa_match_cf_workspace_size", "rosa_match_cf_launch_count", "rosa_inject")
 
 DEV_SYMBOL_RANGE = 1
 
@@ -155,6 +171,88 @@ def match(q: torch.Tensor, k: torch.Tensor | None = None, v: torch.Tensor | None
     return end_idx, ln, sym
 
 
+def _match_args(q, k, v):
+    same = k is None or k is q
+    if q.dtype != torch.uint8 or q.dim() != 2:
+        raise ValueError("q must be uint8 [S, T]")
+    q = q.contiguous()
+    k = q if same else k.contiguous()
+    if k.shape != q.shape or k.dtype != torch.uint8:
+        raise ValueError("k must be uint8 with the shape of q")
+    if v is not None:
+        v = v.contiguous()
+        if v.shape != q.shape or v.dtype != torch.uint8:
+            raise ValueError("v must be uint8 with the shape of q")
+    return q, k, v
+
+
+def match_cf_workspace_size(S: int, T: int, M: int) -> int:
+    n = lib.rosa_match_cf_workspace_size(S, T, M)
+    if n == 0:
+        raise ValueError(f"invalid counterfactual sizes S={S} T={T} M={M}")
+    return n
+
+
+def match_cf(q: torch.Tensor, k: torch.Tensor | None = None, v: torch.Tensor | None = None, *, M: int,
+             g: int = 2, out=None, workspace: torch.Tensor | None = None):
+    """Ordinary retrieval plus the per-bit counterfactual destinations
+    (section 3.5, appendix C.5): for every position and query bit j < M the
+    branches with bit j forced to 0 and to 1.  Returns
+    ``(end_idx, len, sym, end_cf, len_cf, sym_cf)``: int32 ``[S, T]`` and
+    int32 ``[S, T, M, 2]`` (forced bit value last)."""
+    _need_cuda(q, k, v, workspace)
+    q, k, v = _match_args(q, k, v)
+    S, T = q.shape
+    if out is None:
+        out = tuple(torch.empty((S, T), dtype=torch.int32, device=q.device) for _ in range(3)) + \
+            tuple(torch.empty((S, T, M, 2), dtype=torch.int32, device=q.device) for _ in range(3))
+    if workspace is None:
+        workspace = torch.empty(match_cf_workspace_size(S, T, M), dtype=torch.uint8, device=q.device)
+    _check(lib.rosa_match_cf(_ptr(q), _ptr(k), _ptr(v), S, T, M, g, *(_ptr(o) for o in out),
+                             _vp(workspace.data_ptr()), workspace.numel(), _stream(q.device)), "rosa_match_cf")
+    return out
+
+
+def match_cf_launch_count(S: int, T: int, M: int, same: bool) -> int:
+    n = lib.rosa_match_cf_launch_count(S, T, M, 1 if same else 0)
+    if n < 0:
+        raise ValueError("invalid counterfactual sizes")
+    return n
+
+
+def match_rle_workspace_size(S: int, T: int, K: int) -> int:
+    n = lib.rosa_match_rle_workspace_size(S, T, K)
+    if n == 0:
+        raise ValueError(f"invalid match sizes S={S} T={T} K={K}")
+    return n
+
+
+def match_rle(q: torch.Tensor, k: torch.Tensor | None = None, v: torch.Tensor | None = None, *, K: int = 256,
+              g: int = 2, out=None, workspace: torch.Tensor | None = None):
+    """Run-level retrieval with adjacent folding (section 3.3): both streams
+    fold into runs of equal symbols, each query run is answered at its start
+    and the hit maps to the start of the next key run.  Same arguments and
+    outputs as ``match``; ``len`` counts runs."""
+    _need_cuda(q, k, v, workspace)
+    q, k, v = _match_args(q, k, v)
+    S, T = q.shape
+    if out is None:
+        out = tuple(torch.empty((S, T), dtype=torch.int32, device=q.device) for _ in range(3))
+    end_idx, ln, sym = out
+    if workspace is None:
+        workspace = torch.empty(match_rle_workspace_size(S, T, K), dtype=torch.uint8, device=q.device)
+    _check(lib.rosa_match_rle(_ptr(q), _ptr(k), _ptr(v), S, T, K, g, _ptr(end_idx), _ptr(ln), _ptr(sym),
+                              _vp(workspace.data_ptr()), workspace.numel(), _stream(q.device)), "rosa_match_rle")
+    return end_idx, ln, sym
+
+
+def match_rle_launch_count(S: int, T: int, K: int, same: bool) -> int:
+    n = lib.rosa_match_rle_launch_count(S, T, K, 1 if same else 0)
+    if n < 0:
+        raise ValueError("invalid match sizes")
+    return n
+
+
 def match_launch_count(S: int, T: int, K: int, same: bool) -> int:
     """Kernel launches one ``match`` call enqueues (reported by the library)."""
     n = lib.rosa_match_launch_count(S, T, K, 1 if same else 0)
@@ -191,4 +289,27 @@ def gather(V: torch.Tensor, end_idx: torch.Tensor, R: int, d: int, rho: int | No
         out = torch.empty((B, T, R * d), dtype=torch.bfloat16, device=V.device)
     _check(lib.rosa_gather(_ptr(V), V.stride(1), rho, _ptr(end_idx), B, R, T, d, _ptr(out),
                            _stream(V.device)), "rosa_gather")
+    return out
+
+
+def inject(sym: torch.Tensor, e0: torch.Tensor, e1: torch.Tensor, W_out: torch.Tensor, B: int, R: int, M: int,
+           out: torch.Tensor | None = None, status: torch.Tensor | None = None) -> torch.Tensor:
+    """Read-out embedding and injection (appendix C.3) on the tensor cores:
+    ``sym`` int32 ``[B*R, T]`` recalled value symbols (-1: none), ``e0``,
+    ``e1`` bf16 ``[R*M]``, ``W_out`` bf16 ``[D, R*M]`` -> bf16 ``[B, T, D]``."""
+    _need_cuda(sym, e0, e1, W_out, out, status)
+    if sym.dtype != torch.int32 or sym.dim() != 2 or sym.shape[0] != B * R:
+        raise ValueError("sym must be int32 [B*R, T]")
+    for t_ in (e0, e1, W_out):
+        if t_.dtype != torch.bfloat16:
+            raise ValueError("e0, e1 and W_out must be bf16")
+    C = R * M
+    if e0.numel() != C or e1.numel() != C or W_out.dim() != 2 or W_out.shape[1] != C:
+        raise ValueError("e0, e1 must have R*M entries and W_out must be [D, R*M]")
+    sym, e0, e1, W_out = sym.contiguous(), e0.contiguous(), e1.contiguous(), W_out.contiguous()
+    T, D = sym.shape[1], W_out.shape[0]
+    if out is None:
+        out = torch.empty((B, T, D), dtype=torch.bfloat16, device=sym.device)
+    _check(lib.rosa_inject(_ptr(sym), _ptr(e0), _ptr(e1), _ptr(W_out), B, R, M, T, D, _ptr(out),
+                           _ptr(status), _stream(sym.device)), "rosa_inject")
     return out

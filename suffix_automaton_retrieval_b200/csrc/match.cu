@@ -56,8 +56,15 @@ int bits_for(int v) {   // number of bits to hold values 0..v
 }
 
 struct Geometry {
+    const int32_t *xb;       // per-query admissibility bound [S, T], or null for t - g
     int S, T, K, g, n;
     bool same;
+    // Item kinds of a stream, T items each: keys (0), queries (1, unless
+    // q == k, when the keys are the queries), then mcf counterfactual branch
+    // kinds (bit j of the query symbol flipped).  br0 is the first branch
+    // item; allkeys: every item is a key (q == k without branches).
+    int mcf, br0, nkinds;
+    bool allkeys;
     int bps, D0, idbits, keybits;
     int64_t N;
     int ntps, nb1, nb2;
@@ -65,10 +72,14 @@ struct Geometry {
     int wlev;                // levels built: the rest (kWLeafBits) is scanned in the leaf
 };
 
-Geometry make_geometry(int S, int T, int K, int g, bool same) {
+Geometry make_geometry(int S, int T, int K, int g, bool same, int mcf = 0) {
     Geometry G{};
     G.S = S; G.T = T; G.K = K; G.g = g; G.same = same;
-    G.n = same ? T : 2 * T;
+    G.mcf = mcf;
+    G.br0 = same ? T : 2 * T;
+    G.nkinds = (same ? 1 : 2) + mcf;
+    G.allkeys = same && mcf == 0;
+    G.n = G.nkinds * T;
     G.N = (int64_t)S * G.n;
     G.bps = bits_for(K - 1);
     if (G.bps < 1) G.bps = 1;
@@ -117,6 +128,7 @@ struct Workspace {
     int *wcnt;               // [level][stream][tile] ones per wavelet tile
     void *words;             // [stream][level][word] rank directory + bits (16 B each)
     int *wz;                 // [stream][level] zeros per level
+    int32_t *flip[3];        // counterfactual runs: flipped-bit end / len / sym [S, T, mcf]
     size_t bytes;
 };
 
@@ -152,9 +164,10 @@ Workspace carve(const Geometry &G, void *base) {
     W.emin2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.ein2 = (int32_t *)take((size_t)G.S * G.nb2 * 4);
     W.hard = (int32_t *)take(N * 4);
-    W.wq = (int32_t *)take((size_t)G.S * G.T * 4);
-    W.hardb = (int32_t *)take((size_t)G.S * G.T * 4);
-    W.hardw = (int32_t *)take((size_t)G.S * G.T * 4);
+    const size_t nqueries = (size_t)G.S * G.T * (1 + G.mcf);   // queries and branch queries
+    W.wq = (int32_t *)take(nqueries * 4);
+    W.hardb = (int32_t *)take(nqueries * 4);
+    W.hardw = (int32_t *)take(nqueries * 4);
     const size_t ntiles_resolve = (size_t)G.S * ceil_div(G.n, 1024);
     W.btask = (int32_t *)take(ntiles_resolve * 128 * 4);
     W.btab = (int32_t *)take(ntiles_resolve * 128 * 4);
@@ -165,12 +178,25 @@ Workspace carve(const Geometry &G, void *base) {
     W.wcnt = (int *)take((size_t)G.wbits * G.S * G.ntw * 4);
     W.words = take((size_t)G.S * G.wbits * G.nw * 16);
     W.wz = (int *)take((size_t)G.S * G.wbits * 4);
+    if (G.mcf > 0) {   // counterfactual runs: the flipped-bit results before assembly
+        const size_t nf = (size_t)G.S * G.T * G.mcf;
+        for (int i = 0; i < 3; ++i) W.flip[i] = (int32_t *)take(nf * 4);
+    }
     W.bytes = off;
     return W;
 }
 
+// Largest admissible key position for the query at position t of stream s:
+// t - g, or the caller's bound where one is given (run-level retrieval).
+__device__ __forceinline__ int query_bound(const Geometry &G, int s, int t) {
+    return G.xb ? __ldg(G.xb + (int64_t)s * G.T + t) : t - G.g;
+}
+
 // Position of item x in its string (keys 0..T-1, then queries).
-__device__ __forceinline__ int item_pos(uint32_t x, int T) { return (int)x < T ? (int)x : (int)x - T; }
+__device__ __forceinline__ int item_pos(uint32_t x, int T) {
+    const int i = (int)x;
+    return i < T ? i : (i < 2 * T ? i - T : (int)(x % (uint32_t)T));
+}
 // Stream of a global item index (item counts stay below 2^31).
 __device__ __forceinline__ int stream_of(int64_t gi, int n) { return (int)((uint32_t)gi / (uint32_t)n); }
 
@@ -195,9 +221,10 @@ keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geome
     __shared__ uint64_t sk[kKeysThreads * 9];   // 9 words per thread: conflict-free
     const int ntile = ceil_div(G.T, kKeysTile);
     const int sp = blockIdx.x / ntile, tile = blockIdx.x - sp * ntile;
-    const int s = G.same ? sp : sp >> 1;
-    const bool isq = !G.same && (sp & 1);
-    const uint8_t *a = (isq ? q : k) + (int64_t)s * G.T;
+    const int s = sp / G.nkinds, kind = sp - s * G.nkinds;
+    const int kind0 = G.same ? 1 : 2;                 // first branch kind
+    const int flip = kind >= kind0 ? 1 << (kind - kind0) : 0;   // branch: this query bit flipped
+    const uint8_t *a = (kind == 0 ? k : q) + (int64_t)s * G.T;
     const int p0 = tile * kKeysTile;
     const int lim = min(kKeysTile, G.T - p0);
     for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysThreads) {
@@ -216,21 +243,22 @@ keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geome
         for (int u = 0; u < 8 && j0 + u < lim; ++u) {
             if (u > 0) chars = (chars >> G.bps) | ((uint64_t)((uint32_t)e[u] & symmask) << top);
             bad |= (uint32_t)e[u] >= (uint32_t)G.K;
-            const int x = (isq ? G.T : 0) + p0 + j0 + u;
-            sk[threadIdx.x * 9 + u] = (chars << G.idbits) | (uint64_t)x;
+            const int x = kind * G.T + p0 + j0 + u;
+            uint64_t c = chars;
+            if (flip) c ^= (uint64_t)flip << top;       // the branch symbol, then the query history
+            sk[threadIdx.x * 9 + u] = (c << G.idbits) | (uint64_t)x;
         }
     }
     if (bad) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
     __syncthreads();
-    // Initial place: the short strings first, by length, a key before the
-    // query of the same length; then the rest in item order.  Equal symbols
+    // Initial place: the short strings first, by length, then by kind (key,
+    // query, branches); then the rest by kind and position.  Equal symbols
     // then sort as (length, item id), the order of the full comparison.
     uint64_t *out = keys + (int64_t)s * G.n;
     const int m0 = min(G.D0, G.T);
     for (int i = threadIdx.x; i < lim; i += kKeysThreads) {
         const int p = p0 + i;
-        int pos = p;
-        if (!G.same) pos = p < m0 ? 2 * p + (int)isq : (isq ? G.T + p : m0 + p);
+        const int pos = p < m0 ? p * G.nkinds + kind : G.nkinds * m0 + kind * (G.T - m0) + (p - m0);
         out[pos] = sk[(i >> 3) * 9 + (i & 7)];
     }
 }
@@ -554,6 +582,14 @@ groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geo
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t pair_key(uint32_t k2, uint32_t x) { return ((uint64_t)k2 << 32) | x; }
 
+// The item whose string is item x's with its first h symbols removed: the
+// same kind h positions back, except that a branch's history is the query's
+// (a branch differs from its query only in the first symbol).
+__device__ __forceinline__ uint32_t back_item(const Geometry &G, uint32_t x, int64_t h) {
+    if ((int)x < G.br0) return x - (uint32_t)h;
+    return (uint32_t)((G.same ? 0 : G.T) + item_pos(x, G.T) - h);
+}
+
 // Small groups: one thread computes its members' keys and insertion-sorts
 // them in place.  Large groups: one warp computes the keys.
 __global__ void dbl_keys_sort_kernel(const int2 *__restrict__ small, const int2 *__restrict__ large,
@@ -568,7 +604,7 @@ __global__ void dbl_keys_sort_kernel(const int2 *__restrict__ small, const int2 
         uint32_t *gs = sa + gr.x;
         uint32_t *gk = k2 + gr.x;
         // keys first: the members' rank loads are independent of each other
-        for (int m = 0; m < gr.y; ++m) gk[m] = (uint32_t)rank[seg + gs[m] - h];
+        for (int m = 0; m < gr.y; ++m) gk[m] = (uint32_t)rank[seg + back_item(G, gs[m], h)];
         for (int m = 1; m < gr.y; ++m) {   // insertion sort of (key, id) pairs
             const uint32_t x = gs[m], kk = gk[m];
             const uint64_t key = pair_key(kk, x);
@@ -588,7 +624,7 @@ __global__ void dbl_keys_sort_kernel(const int2 *__restrict__ small, const int2 
         const int64_t seg = (gr.x / G.n) * (int64_t)G.n;
         for (int m = lane; m < gr.y; m += 32) {
             const uint32_t x = sa[gr.x + m];
-            k2[gr.x + m] = (uint32_t)rank[seg + x - h];
+            k2[gr.x + m] = (uint32_t)rank[seg + back_item(G, x, h)];
         }
     }
 }
@@ -824,9 +860,8 @@ __global__ void lcp_long_kernel(const uint8_t *__restrict__ q, const uint8_t *__
 //     strictly inside the block) per 32 and per 1024 ranks, and the LCP edge
 //     entering each 32-block from below.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T, bool same) {
-    return (same || (int)x < T) ? (int)x : INT_MAX;
-}
+// Keys are the items below T (with q == k they are the queries as well).
+__device__ __forceinline__ int key_pos_or_inf(uint32_t x, int T) { return (int)x < T ? (int)x : INT_MAX; }
 
 // One CTA of 256 threads per 1024 ranks; thread t loads ranks t + 256u
 // (u < 4) up front, so that each warp's u-th group is one 32-rank block.
@@ -847,7 +882,7 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
         pos[u] = INT_MAX;
         l[u] = INT_MAX;
         if (j < G.n) {
-            pos[u] = key_pos_or_inf(sa[seg + j], G.T, G.same);
+            pos[u] = key_pos_or_inf(sa[seg + j], G.T);
             l[u] = lcp[seg + j];
         }
     }
@@ -938,7 +973,7 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
     const int ntw = ceil_div(G.T, kWTile);
     if (threadIdx.x == 0) {
         int p = 0;
-        if (G.same) p = tt * kRadixTile;
+        if (G.allkeys) p = tt * kRadixTile;
         else for (int i = 0; i < tt; ++i) p += ktile[(int64_t)s * G.ntps + i];
         pre_s = p;
     }
@@ -960,7 +995,7 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
         const int i = u * 256 + threadIdx.x;
         const bool ok = i < lim;
         const uint32_t x = xs[u];
-        const bool key = ok && (G.same || (int)x < G.T);
+        const bool key = ok && (int)x < G.T;
         const unsigned bal = __ballot_sync(ROSA_FULL_MASK, key);
         if (lane == 0) wk[warp] = __popc(bal);
         __syncthreads();
@@ -970,7 +1005,7 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
             rtot += wk[w];
         }
         const int kidx = run + wpre + __popc(bal & lanemask_lt());
-        if (ok && !G.same) kcount[base + i] = kidx;
+        if (ok && !G.allkeys) kcount[base + i] = kidx;
         if (key) {
             a0[(int64_t)s * G.T + kidx] = x;
             if ((x >> (nbits - 1)) & 1u) {
@@ -1198,7 +1233,7 @@ struct StreamView {
     bool same;
 };
 
-__device__ __forceinline__ int kpos(const StreamView &v, int r) { return key_pos_or_inf(v.sa[r], v.T, v.same); }
+__device__ __forceinline__ int kpos(const StreamView &v, int r) { return key_pos_or_inf(v.sa[r], v.T); }
 
 // number of keys at ranks below r (r in [0, n])
 __device__ __forceinline__ int kc(const StreamView &v, int r) {
@@ -1222,20 +1257,48 @@ __device__ __forceinline__ StreamView make_view(const Geometry &G, int s, const 
                       A.ein1 + (int64_t)s * G.nb1, A.mp2 + (int64_t)s * G.nb2, A.em2 + (int64_t)s * G.nb2,
                       A.ein2 + (int64_t)s * G.nb2, A.kcount ? A.kcount + seg : nullptr,
                       A.words + (int64_t)s * A.nbits * nw, A.wz + (int64_t)s * A.nbits, G.n, G.T, G.nb1, G.nb2,
-                      A.nbits, nw, G.same};
+                      A.nbits, nw, G.allkeys};
 }
 
-__device__ __forceinline__ void write_result(const Geometry &G, const uint8_t *vsym, int s, int t, int L, int ib,
-                                             int32_t *end_idx, int32_t *len, int32_t *sym) {
-    const int64_t o = (int64_t)s * G.T + t;
+// Output slots.  The query at (s, t) writes slot s*T + t of the caller's
+// arrays; branch j of (s, t) (query bit j flipped) writes slot
+// S*T + (s*T + t)*mcf + j, i.e. entry (s*T + t)*mcf + j of the branch arrays.
+// Deferred lookups park their key range in the same slots.
+struct Outs {
+    int32_t *e0, *l0, *y0;   // [S, T]
+    int32_t *e1, *l1, *y1;   // [S, T, mcf]
+    int64_t n0;              // S * T
+    __device__ __forceinline__ int32_t &E(int64_t o) const { return o < n0 ? e0[o] : e1[o - n0]; }
+    __device__ __forceinline__ int32_t &L(int64_t o) const { return o < n0 ? l0[o] : l1[o - n0]; }
+    __device__ __forceinline__ int32_t &Y(int64_t o) const { return o < n0 ? y0[o] : y1[o - n0]; }
+};
+
+// Slot of query item x (a query or a branch) of stream s.
+__device__ __forceinline__ int64_t out_slot(const Geometry &G, int s, uint32_t x) {
+    const int t = item_pos(x, G.T);
+    if ((int)x < G.br0) return (int64_t)s * G.T + t;
+    const int j = ((int)x - G.br0) / G.T;
+    return (int64_t)G.S * G.T + ((int64_t)s * G.T + t) * G.mcf + j;
+}
+
+// Stream and time of an output slot.
+__device__ __forceinline__ void slot_stream_time(const Geometry &G, int64_t o, int &s, int &t) {
+    const int64_t n0 = (int64_t)G.S * G.T;
+    const int64_t st = o < n0 ? o : (o - n0) / G.mcf;
+    s = (int)(st / G.T);
+    t = (int)(st - (int64_t)s * G.T);
+}
+
+__device__ __forceinline__ void write_result(const uint8_t *vsym, const Outs &O, int64_t o, int64_t srow, int L,
+                                             int ib) {
     if (L > 0 && ib >= 0) {
-        end_idx[o] = ib;
-        len[o] = L;
-        sym[o] = (int32_t)vsym[(int64_t)s * G.T + ib + 1];
+        O.E(o) = ib;
+        O.L(o) = L;
+        O.Y(o) = (int32_t)vsym[srow + ib + 1];
     } else {
-        end_idx[o] = -1;
-        len[o] = 0;
-        sym[o] = -1;
+        O.E(o) = -1;
+        O.L(o) = 0;
+        O.Y(o) = -1;
     }
 }
 
@@ -1254,7 +1317,7 @@ __device__ __forceinline__ int warp_prefix_min(int x, int lane) {
 //   lc[i]  LCP edge between local ranks i-1 and i (0 at the stream start,
 //          -1 past the stream end); lc[kRWin] is the edge just past the window;
 //   sp[k][i] min(lc[i .. i+2^k-1]) capped to 255 (u8);
-//   per query of the tile: local rank qj, time index qt, match length qL.
+//   per query of the tile: local rank qj, item id qt, match length qL.
 // Queries are resolved in three uniform phases (see resolve_tile_kernel).
 constexpr int kSpLevels = 11;          // lifting reaches 2^11 - 1 ranks: a whole side of the window
 constexpr int kProbe = 16;             // ranks a lane probes on each side before its warp helps
@@ -1283,13 +1346,11 @@ struct WinSmem {
 
 // Parks a query whose interval is too wide to scan: its key range goes into
 // the output slots until wavelet_query_kernel replaces it with the answer.
-__device__ __forceinline__ void defer_wavelet(const Geometry &G, int s, int t, int L, int klo, int khi,
-                                              int32_t *end_idx, int32_t *len, int32_t *sym, int32_t *wq,
+__device__ __forceinline__ void defer_wavelet(const Outs &O, int64_t o, int L, int klo, int khi, int32_t *wq,
                                               int *wq_count) {
-    const int64_t o = (int64_t)s * G.T + t;
-    len[o] = L;
-    end_idx[o] = klo;
-    sym[o] = khi;
+    O.L(o) = L;
+    O.E(o) = klo;
+    O.Y(o) = khi;
     wq[atomicAdd(wq_count, 1)] = (int32_t)o;
 }
 
@@ -1397,8 +1458,7 @@ __device__ void window_bounds(const WinSmem &w, bool at_start, int jl, int L, in
 //   Phase D: one warp per listed interval, 32 ranks per step.
 // Queries whose answer needs ranks outside the window go to the hard lists.
 __global__ void __launch_bounds__(kRThreads, 4)
-resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, int32_t *__restrict__ end_idx,
-                    int32_t *__restrict__ len, int32_t *__restrict__ sym, int32_t *__restrict__ hard,
+resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, Outs O, int32_t *__restrict__ hard,
                     int *hard_count, int32_t *__restrict__ hardb, int *hardb_count, int32_t *__restrict__ hardw,
                     int *hardw_count, int32_t *__restrict__ btask, int *btask_count, int32_t *__restrict__ wq,
                     int *wq_count) {
@@ -1430,7 +1490,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
             const int r = w0 + i;
             const int l = ls[u];
             if (i < kRWin) {
-                w.kp[i] = (r >= 0 && r < G.n) ? key_pos_or_inf(xs[u], G.T, G.same) : INT_MAX;
+                w.kp[i] = (r >= 0 && r < G.n) ? key_pos_or_inf(xs[u], G.T) : INT_MAX;
                 w.sp[0][i] = (uint8_t)(l < 0 ? 0 : (l > 255 ? 255 : l));
             }
             w.lc[i] = l;
@@ -1489,7 +1549,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
         if (isq) {
             const int slot = base + __popc(bal & lanemask_lt());
             w.qj[slot] = (int16_t)(i + kRHalo);
-            w.qt[slot] = G.same ? (int)x : (int)x - G.T;
+            w.qt[slot] = (int)x;
         }
     }
     __syncthreads();
@@ -1497,7 +1557,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     // Phase A
     for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
         const int jl = w.qj[qi];
-        const int X = w.qt[qi] - G.g;
+        const int X = query_bound(G, s, item_pos(w.qt[qi], G.T));
         int L = 0;
         if (X >= 0) {
             int m = INT_MAX, Ll = -1;
@@ -1534,7 +1594,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     for (int bi = warp; bi < nb; bi += kRThreads / 32) {
         const int qi = w.bq[bi];
         const int jl = w.qj[qi];
-        const int X = w.qt[qi] - G.g;
+        const int X = query_bound(G, s, item_pos(w.qt[qi], G.T));
         const int Ll = warp_nearest_smem(w, jl, X, -1, 0, lane);
         int L = Ll;
         if (Ll != kNeedHard) {
@@ -1549,8 +1609,9 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     const StreamView v = make_view(G, s, A);
     for (int qi = threadIdx.x; qi < nq; qi += kRThreads) {
         const int jl = w.qj[qi];
-        const int t = w.qt[qi];
-        const int X = t - G.g;
+        const uint32_t qx = (uint32_t)w.qt[qi];
+        const int X = query_bound(G, s, item_pos(qx, G.T));
+        const int64_t o = out_slot(G, s, qx);
         const int L = w.qL[qi];
         int lo = 0, hi = -1;
         if (L == kNeedHard) {
@@ -1562,10 +1623,9 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
             if (lo < 0 || hi < 0) {
                 // L is known; only the interval's far end lies outside the window.  That
                 // end depends on (tile, side, L) alone, so short L share one scan.
-                const int64_t o = (int64_t)s * G.T + t;
-                len[o] = L;
-                end_idx[o] = lo < 0 ? -1 : w0 + lo;
-                sym[o] = hi < 0 ? -1 : w0 + hi;
+                O.L(o) = L;
+                O.E(o) = lo < 0 ? -1 : w0 + lo;
+                O.Y(o) = hi < 0 ? -1 : w0 + hi;
                 if (L < kBoundShared) {
                     if (lo < 0) atomicOr(&w.need[0], 1ull << L);
                     if (hi < 0) atomicOr(&w.need[1], 1ull << L);
@@ -1593,11 +1653,11 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                 w.qL[qi] = L;
                 continue;
             } else {
-                defer_wavelet(G, s, t, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), end_idx, len, sym, wq, wq_count);
+                defer_wavelet(O, o, L, kc(v, w0 + lo), kc(v, w0 + hi + 1), wq, wq_count);
                 continue;
             }
         }
-        write_result(G, vsym, s, t, L, ib, end_idx, len, sym);
+        write_result(vsym, O, o, (int64_t)s * G.T, L, ib);
     }
     __syncthreads();
     // Phase D: mid-size intervals, 8 lanes each (4 per warp), 8 ranks per step
@@ -1613,7 +1673,7 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
                 qi = w.bq[di];
                 lo = w.dlo[di];
                 hi = w.dhi[di];
-                X = w.qt[qi] - G.g;
+                X = query_bound(G, s, item_pos(w.qt[qi], G.T));
             }
             int best = -1;
             for (int r = lo + sl; r <= hi; r += kSub) {
@@ -1622,7 +1682,8 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
             }
 #pragma unroll
             for (int o = kSub / 2; o >= 1; o >>= 1) best = max(best, __shfl_xor_sync(ROSA_FULL_MASK, best, o));
-            if (act && sl == 0) write_result(G, vsym, s, w.qt[qi], w.qL[qi], best, end_idx, len, sym);
+            if (act && sl == 0)
+                write_result(vsym, O, out_slot(G, s, (uint32_t)w.qt[qi]), (int64_t)s * G.T, w.qL[qi], best);
         }
     }
     // one bound task per (side, L) this tile needs beyond its window
@@ -1756,8 +1817,7 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
 
 // One warp per listed query: scans for L and the interval bounds; the most
 // recent admissible end is left to wavelet_query_kernel.
-__global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
-                                    int32_t *__restrict__ len, int32_t *__restrict__ sym,
+__global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, Outs O,
                                     const int32_t *__restrict__ hard, const int *__restrict__ hard_count,
                                     int32_t *__restrict__ wq, int *wq_count) {
     const int nh = *hard_count;
@@ -1769,8 +1829,8 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restri
         const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
-        const int t = G.same ? (int)x : (int)x - G.T;
-        const int X = t - G.g;
+        const int X = query_bound(G, s, item_pos(x, G.T));
+        const int64_t o = out_slot(G, s, x);
         const StreamView v = make_view(G, s, A);
         const int bl = warp_scan<NEAREST>(v, j, -1, X, 0, lane);
         const int br = warp_scan<NEAREST>(v, j, +1, X, bl, lane);
@@ -1778,12 +1838,11 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restri
         if (L > 0) {
             const int lo = warp_scan<BOUND>(v, j, -1, X, L, lane);
             const int hi = warp_scan<BOUND>(v, j, +1, X, L, lane);
-            if (lane == 0) defer_wavelet(G, s, t, L, kc(v, lo), kc(v, hi + 1), end_idx, len, sym, wq, wq_count);
+            if (lane == 0) defer_wavelet(O, o, L, kc(v, lo), kc(v, hi + 1), wq, wq_count);
         } else if (lane == 0) {
-            const int64_t o = (int64_t)s * G.T + t;
-            end_idx[o] = -1;
-            len[o] = 0;
-            sym[o] = -1;
+            O.E(o) = -1;
+            O.L(o) = 0;
+            O.Y(o) = -1;
         }
     }
 }
@@ -1791,8 +1850,7 @@ __global__ void resolve_hard_kernel(Geometry G, ResolveArgs A, int32_t *__restri
 // Queries whose L is known but whose interval runs past the staged window:
 // one warp scans outward from the window edge on each open side, then the
 // query is parked for the wavelet lookup.
-__global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
-                                      const int32_t *__restrict__ len, int32_t *__restrict__ sym,
+__global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, Outs O,
                                       const int32_t *__restrict__ hardb, const int *__restrict__ hardb_count,
                                       int32_t *__restrict__ wq, int *wq_count) {
     const int nh = *hardb_count;
@@ -1804,18 +1862,17 @@ __global__ void resolve_bounds_kernel(Geometry G, ResolveArgs A, int32_t *__rest
         const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
-        const int t = G.same ? (int)x : (int)x - G.T;
-        const int X = t - G.g;
-        const int64_t o = (int64_t)s * G.T + t;
-        const int L = len[o];
-        int lo = end_idx[o], hi = sym[o];
+        const int X = query_bound(G, s, item_pos(x, G.T));
+        const int64_t o = out_slot(G, s, x);
+        const int L = O.L(o);
+        int lo = O.E(o), hi = O.Y(o);
         const int w0 = (j / kRTile) * kRTile - kRHalo;
         const StreamView v = make_view(G, s, A);
         if (lo < 0) lo = warp_scan<BOUND>(v, w0, -1, X, L, lane);
         if (hi < 0) hi = warp_scan<BOUND>(v, w0 + kRWin - 1, +1, X, L, lane);
         if (lane == 0) {
-            end_idx[o] = kc(v, lo);
-            sym[o] = kc(v, hi + 1);
+            O.E(o) = kc(v, lo);
+            O.Y(o) = kc(v, hi + 1);
             wq[atomicAdd(wq_count, 1)] = (int32_t)o;
         }
     }
@@ -1843,8 +1900,7 @@ __global__ void bound_task_kernel(Geometry G, ResolveArgs A, const int32_t *__re
 
 // Queries waiting for a shared bound: fill the open side(s) from the table
 // and park the query for the wavelet lookup.
-__global__ void bound_finish_kernel(Geometry G, ResolveArgs A, int32_t *__restrict__ end_idx,
-                                    const int32_t *__restrict__ len, int32_t *__restrict__ sym,
+__global__ void bound_finish_kernel(Geometry G, ResolveArgs A, Outs O,
                                     const int32_t *__restrict__ hardw, const int *__restrict__ hardw_count,
                                     const int32_t *__restrict__ btab, int32_t *__restrict__ wq, int *wq_count) {
     const int nh = *hardw_count;
@@ -1854,36 +1910,34 @@ __global__ void bound_finish_kernel(Geometry G, ResolveArgs A, int32_t *__restri
         const int s = stream_of(gi, G.n);
         const int j = (int)(gi - (int64_t)s * G.n);
         const uint32_t x = A.sa[gi];
-        const int t = G.same ? (int)x : (int)x - G.T;
-        const int64_t o = (int64_t)s * G.T + t;
-        const int L = len[o];
+        const int64_t o = out_slot(G, s, x);
+        const int L = O.L(o);
         const int64_t tb = ((int64_t)s * ntr + j / kRTile) * 2 * kBoundShared;
-        int lo = end_idx[o], hi = sym[o];
+        int lo = O.E(o), hi = O.Y(o);
         if (lo < 0) lo = btab[tb + L];
         if (hi < 0) hi = btab[tb + kBoundShared + L];
         const StreamView v = make_view(G, s, A);
-        end_idx[o] = kc(v, lo);
-        sym[o] = kc(v, hi + 1);
+        O.E(o) = kc(v, lo);
+        O.Y(o) = kc(v, hi + 1);
         wq[atomicAdd(wq_count, 1)] = (int32_t)o;
     }
 }
 
 // Largest admissible key position inside each parked query's key range.
-__global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
-                                     int32_t *__restrict__ end_idx, int32_t *__restrict__ sym,
+__global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, Outs O,
                                      const int32_t *__restrict__ wq, const int *__restrict__ wq_count) {
     const int nq = *wq_count;
     const int nw = (G.T >> 6) + 1;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t o = wq[i];
-        const int s = stream_of(o, G.T);
-        const int t = (int)(o - (int64_t)s * G.T);
-        const int klo = end_idx[o], khi = sym[o];
+        int s, t;
+        slot_stream_time(G, o, s, t);
+        const int klo = O.E(o), khi = O.Y(o);
         const WWord *W = A.words + (int64_t)s * A.nbits * nw;
         const int ib = wavelet_max_le(W, A.wz + (int64_t)s * A.nbits, A.leaf + (int64_t)s * G.T, A.nbits, A.nlev, nw,
-                                      klo, khi, t - G.g);
-        end_idx[o] = ib;
-        sym[o] = ib >= 0 ? (int32_t)vsym[(int64_t)s * G.T + ib + 1] : -1;
+                                      klo, khi, query_bound(G, s, t));
+        O.E(o) = ib;
+        O.Y(o) = ib >= 0 ? (int32_t)vsym[(int64_t)s * G.T + ib + 1] : -1;
     }
 }
 
@@ -1919,36 +1973,58 @@ int device_sm_count() {
     return sms[dev];
 }
 
-int match_launch_count(int S, int T, int K, bool same) {
+int match_launch_count(int S, int T, int K, bool same, int mcf) {
     if (S == 0 || T == 0) return 0;
-    const Geometry G = make_geometry(S, T, K, 1, same);
+    const Geometry G = make_geometry(S, T, K, 1, same, mcf);
     int rounds = 0;
     for (int64_t h = G.D0; h < T; h *= 2) ++rounds;
     const int passes = ceil_div(G.keybits - G.idbits, kRadixBits);
     // keys0 + 3 per radix pass + groups0 + 3 per doubling round + 2 lcp + summary
-    // + wavelet (key count when q != k, compaction, one per level) + 6 resolve
-    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (same ? 0 : 1) + 1 + G.wlev + 6;
+    // + wavelet (key count unless every item is a key, compaction, one per level)
+    // + 6 resolve (+ the counterfactual assembly)
+    return 1 + 3 * passes + 1 + 3 * rounds + 3 + (G.allkeys ? 0 : 1) + 1 + G.wlev + 6 + (mcf > 0 ? 1 : 0);
 }
 
-size_t match_workspace_bytes(int S, int T, int K, bool same) {
-    const Geometry G = make_geometry(S, T, K, 1, same);
+size_t match_workspace_bytes(int S, int T, int K, bool same, int mcf) {
+    const Geometry G = make_geometry(S, T, K, 1, same, mcf);
     return carve(G, nullptr).bytes;
 }
 
-cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int K, int g,
-                         int32_t *end_idx, int32_t *len, int32_t *sym, void *workspace, size_t ws_bytes,
-                         cudaStream_t st) {
-    const bool same = (q == k);
-    const Geometry G = make_geometry(S, T, K, g, same);
-    Workspace W = carve(G, workspace);
-    if (W.bytes > ws_bytes) return cudaErrorInvalidValue;
+namespace {
+
+// Counterfactual tables [S, T, M, 2] (beta last): the branch that keeps
+// query bit j is the ordinary result; the other one is the flipped branch.
+__global__ void cf_assemble_kernel(const uint8_t *__restrict__ q, int64_t ST, int M, const int32_t *__restrict__ oe,
+                                   const int32_t *__restrict__ ol, const int32_t *__restrict__ oy,
+                                   const int32_t *__restrict__ fe, const int32_t *__restrict__ fl,
+                                   const int32_t *__restrict__ fy, int32_t *__restrict__ end_cf,
+                                   int32_t *__restrict__ len_cf, int32_t *__restrict__ sym_cf) {
+    const int64_t total = ST * M;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t o = i / M;
+        const int j = (int)(i - o * M);
+        const int keep = (q[o] >> j) & 1;
+        const int64_t b = i * 2;
+        end_cf[b + keep] = oe[o];
+        len_cf[b + keep] = ol[o];
+        sym_cf[b + keep] = oy[o];
+        end_cf[b + 1 - keep] = fe[i];
+        len_cf[b + 1 - keep] = fl[i];
+        sym_cf[b + 1 - keep] = fy[i];
+    }
+}
+
+cudaError_t run_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, const Geometry &G, const Workspace &W,
+                      Outs O, cudaStream_t st) {
     cudaError_t err;
     if ((err = cudaMemsetAsync(W.status, 0, 256 + 256, st)) != cudaSuccess) return err;   // status + counts
-    if (S == 0 || T == 0) return cudaSuccess;
+    if (G.S == 0 || G.T == 0) return cudaSuccess;
+    const int T = G.T;
     const uint8_t *vs = v ? v : k;
 
     // 1a. keys
-    keys0_kernel<<<(unsigned)((int64_t)G.S * (G.same ? 1 : 2) * ceil_div(T, kKeysTile)), kKeysThreads, 0, st>>>(
+    keys0_kernel<<<(unsigned)((int64_t)G.S * G.nkinds * ceil_div(T, kKeysTile)), kKeysThreads, 0, st>>>(
         q, k, G, W.keys[0], W.status);
     // 1b. radix sort over the key bits above the item id, 8 bits per pass
     int cur = 0;
@@ -1987,7 +2063,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
                                                            W.minpos2, W.emin2, W.ein2);
     // 3b. wavelet matrix over key positions in rank order
     if ((err = cudaMemsetAsync(W.wcnt, 0, (size_t)G.wbits * G.S * G.ntw * 4, st)) != cudaSuccess) return err;
-    if (!G.same) key_tile_count_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile);
+    if (!G.allkeys) key_tile_count_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, sa, W.ktile);
     wavelet_compact_kernel<<<(unsigned)(G.S * G.ntps), 256, 0, st>>>(G, G.wbits, sa, W.ktile, W.kcount, W.wvals[0],
                                                                       W.wcnt);
     WWord *words = static_cast<WWord *>(W.words);
@@ -1996,7 +2072,7 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
                                                                        W.wvals[(lv + 1) & 1], W.wcnt, words, W.wz);
     // 3c. resolve: thread per query, then warp per query for the long scans
     if ((err = tile_smem_optin()) != cudaSuccess) return err;
-    ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.same ? nullptr : W.kcount,
+    ResolveArgs A{sa, W.lcp, W.minpos1, W.emin1, W.ein1, W.minpos2, W.emin2, W.ein2, G.allkeys ? nullptr : W.kcount,
                   words, W.wz, W.wvals[G.wlev & 1], G.wbits, G.wlev};
     int *hard_count = W.counts + 4;
     int *wq_count = W.counts + 5;
@@ -2004,15 +2080,41 @@ cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, i
     int *hardw_count = W.counts + 8;
     int *btask_count = W.counts + 9;
     resolve_tile_kernel<<<(unsigned)(G.S * ceil_div(G.n, kRTile)), kRThreads, sizeof(WinSmem), st>>>(
-        G, A, vs, end_idx, len, sym, W.hard, hard_count, W.hardb, hardb_count, W.hardw, hardw_count, W.btask,
-        btask_count, W.wq, wq_count);
-    resolve_hard_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hard, hard_count, W.wq, wq_count);
-    resolve_bounds_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardb, hardb_count, W.wq,
-                                                        wq_count);
+        G, A, vs, O, W.hard, hard_count, W.hardb, hardb_count, W.hardw, hardw_count, W.btask, btask_count, W.wq,
+        wq_count);
+    resolve_hard_kernel<<<sms * 16, 256, 0, st>>>(G, A, O, W.hard, hard_count, W.wq, wq_count);
+    resolve_bounds_kernel<<<sms * 16, 256, 0, st>>>(G, A, O, W.hardb, hardb_count, W.wq, wq_count);
     bound_task_kernel<<<sms * 16, 256, 0, st>>>(G, A, W.btask, btask_count, W.btab);
-    bound_finish_kernel<<<sms * 16, 256, 0, st>>>(G, A, end_idx, len, sym, W.hardw, hardw_count, W.btab, W.wq,
-                                                      wq_count);
-    wavelet_query_kernel<<<sms * 16, 256, 0, st>>>(G, A, vs, end_idx, sym, W.wq, wq_count);
+    bound_finish_kernel<<<sms * 16, 256, 0, st>>>(G, A, O, W.hardw, hardw_count, W.btab, W.wq, wq_count);
+    wavelet_query_kernel<<<sms * 16, 256, 0, st>>>(G, A, vs, O, W.wq, wq_count);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int K, int g,
+                         int32_t *end_idx, int32_t *len, int32_t *sym, void *workspace, size_t ws_bytes,
+                         cudaStream_t st, const int32_t *xbound) {
+    Geometry G = make_geometry(S, T, K, g, q == k);
+    G.xb = xbound;
+    const Workspace W = carve(G, workspace);
+    if (W.bytes > ws_bytes) return cudaErrorInvalidValue;
+    const Outs O{end_idx, len, sym, nullptr, nullptr, nullptr, (int64_t)S * T};
+    return run_match(q, k, v, G, W, O, st);
+}
+
+cudaError_t launch_match_cf(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int M, int g,
+                            int32_t *end_idx, int32_t *len, int32_t *sym, int32_t *end_cf, int32_t *len_cf,
+                            int32_t *sym_cf, void *workspace, size_t ws_bytes, cudaStream_t st) {
+    const Geometry G = make_geometry(S, T, 1 << M, g, q == k, M);
+    const Workspace W = carve(G, workspace);
+    if (W.bytes > ws_bytes) return cudaErrorInvalidValue;
+    const Outs O{end_idx, len, sym, W.flip[0], W.flip[1], W.flip[2], (int64_t)S * T};
+    cudaError_t e = run_match(q, k, v, G, W, O, st);
+    if (e != cudaSuccess || S == 0 || T == 0) return e;
+    const int64_t ST = (int64_t)S * T;
+    cf_assemble_kernel<<<(unsigned)(device_sm_count() * 8), 256, 0, st>>>(
+        q, ST, M, end_idx, len, sym, W.flip[0], W.flip[1], W.flip[2], end_cf, len_cf, sym_cf);
     return cudaGetLastError();
 }
 

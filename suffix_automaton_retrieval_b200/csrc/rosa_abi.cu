@@ -66,6 +66,56 @@ int rosa_match(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int 
     return cuda_status(rosa::launch_match(q, k, v, S, T, K, g, end_idx, len, sym, workspace, ws_bytes, stream));
 }
 
+namespace {
+bool cf_sizes_ok(int S, int T, int M) {
+    if (S < 0 || T < 0 || M < 1 || M > 8) return false;
+    // every item index (keys, queries and M branch kinds per position) fits a signed 32-bit integer
+    return (int64_t)S * T * (2 + M) < ((int64_t)1 << 31);
+}
+}  // namespace
+
+size_t rosa_match_cf_workspace_size(int S, int T, int M) {
+    if (!cf_sizes_ok(S, T, M)) return 0;
+    return rosa::match_workspace_bytes(S, T, 1 << M, /*same=*/false, M);
+}
+
+int rosa_match_cf(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int M, int g,
+                  int32_t *end_idx, int32_t *len, int32_t *sym, int32_t *end_cf, int32_t *len_cf, int32_t *sym_cf,
+                  void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!cf_sizes_ok(S, T, M) || g < 1) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)S * T > 0 && (!q || !k || !end_idx || !len || !sym || !end_cf || !len_cf || !sym_cf))
+        return ROSA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256)) return ROSA_ERR_WORKSPACE;
+    if (ws_bytes < rosa::match_workspace_bytes(S, T, 1 << M, q == k, M)) return ROSA_ERR_WORKSPACE;
+    return cuda_status(rosa::launch_match_cf(q, k, v, S, T, M, g, end_idx, len, sym, end_cf, len_cf, sym_cf,
+                                             workspace, ws_bytes, stream));
+}
+
+int rosa_match_cf_launch_count(int S, int T, int M, int q_is_k) {
+    if (!cf_sizes_ok(S, T, M)) return -1;
+    return rosa::match_launch_count(S, T, 1 << M, q_is_k != 0, M);
+}
+
+size_t rosa_match_rle_workspace_size(int S, int T, int K) {
+    if (!match_sizes_ok(S, T, K)) return 0;
+    return rosa::match_rle_workspace_bytes(S, T, K, /*same=*/false);
+}
+
+int rosa_match_rle(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int K, int g,
+                   int32_t *end_idx, int32_t *len, int32_t *sym, void *workspace, size_t ws_bytes,
+                   cudaStream_t stream) {
+    if (!match_sizes_ok(S, T, K) || g < 1) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)S * T > 0 && (!q || !k || !end_idx || !len || !sym)) return ROSA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256)) return ROSA_ERR_WORKSPACE;
+    if (ws_bytes < rosa::match_rle_workspace_bytes(S, T, K, q == k)) return ROSA_ERR_WORKSPACE;
+    return cuda_status(rosa::launch_match_rle(q, k, v, S, T, K, g, end_idx, len, sym, workspace, ws_bytes, stream));
+}
+
+int rosa_match_rle_launch_count(int S, int T, int K, int q_is_k) {
+    if (!match_sizes_ok(S, T, K)) return -1;
+    return rosa::match_rle_launch_count(S, T, K, q_is_k != 0);
+}
+
 int rosa_match_launch_count(int S, int T, int K, int q_is_k) {
     if (!match_sizes_ok(S, T, K)) return -1;
     return rosa::match_launch_count(S, T, K, q_is_k != 0);
@@ -80,6 +130,14 @@ int rosa_match_device_status(const void *workspace, cudaStream_t stream, uint32_
     if (e != cudaSuccess) return ROSA_ERR_CUDA;
     *status = h;
     return ROSA_OK;
+}
+
+int rosa_inject(const int32_t *sym, const rosa_bf16 *e0, const rosa_bf16 *e1, const rosa_bf16 *W_out, int B, int R,
+                int M, int T, int D, rosa_bf16 *inj, uint32_t *dev_status, cudaStream_t stream) {
+    if (B < 0 || T < 0 || R < 1 || M < 1 || M > 8 || D < 1) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)B * T >= ((int64_t)1 << 31) / 2 || (int64_t)R * M > (1 << 20)) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!sym || !e0 || !e1 || !W_out || !inj)) return ROSA_ERR_INVALID_ARG;
+    return cuda_status(rosa::launch_inject(sym, e0, e1, W_out, B, R, M, T, D, inj, dev_status, stream));
 }
 
 int rosa_gather(const rosa_bf16 *V, int64_t v_row_stride, int64_t v_route_stride, const int32_t *end_idx,
