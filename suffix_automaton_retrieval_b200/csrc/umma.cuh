@@ -137,3 +137,29 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
 
 }  // namespace umma
 }  // namespace rosa
+
+// ---------------------------------------------------------------------------
+// Tensor Memory Accelerator (TMA) loads, local GPU only (no cluster multicast).
+// ---------------------------------------------------------------------------
+namespace rosa {
+namespace umma {
+
+// One thread: expect `bytes` more transaction bytes on `bar`, then arrive.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// One thread: 2-D tiled load of the box at (x, y) (x innermost, in elements;
+// x * element size must be a multiple of 16 bytes) into shared memory,
+// completing `bar`'s transaction count.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+}  // namespace umma
+}  // namespace rosa
