@@ -65,6 +65,12 @@ def parse():
     ap.add_argument("--cf", action="store_true",
                     help="time the counterfactual op (ordinary retrieval plus every query bit forced to 0 and "
                          "to 1, section 3.5; M = log2 K bits) as the match step")
+    ap.add_argument("--fused", action="store_true",
+                    help="qwen-proj-64: start from the hidden states with the fused layer norm + projection + "
+                         "discretisation kernel (section 3.2) instead of a set-up projection")
+    ap.add_argument("--inject", action="store_true",
+                    help="qwen-proj-64 / markov-4-train: add the read-out embedding and injection (appendix C.3) "
+                         "on the tensor cores to the step")
     ap.add_argument("--streams", type=int, default=0,
                     help="profiling aid: keep only the first N streams of a symbol workload")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel eagerly instead of graph replay")
@@ -103,7 +109,29 @@ def shard_plan(B: int, R: int, has_rows: bool, world: int, rank: int):
     return "streams", lo, hi
 
 
-def build_workload(cfg: int, device, seed_offset: int = 0, shard=None):
+def dense_params(wl, cfg, device, fused, inject):
+    """Seeded parameters of the dense NEXT ops: layer-norm scale / shift
+    (fused front end) and the read-out embedding e0, e1 with the injection
+    matrix W_out (D_out = the model width 2048 for qwen-proj-64, the channel
+    count for markov-4-train)."""
+    import torch
+    from suffix_automaton_retrieval_b200 import workloads as W
+    if fused:
+        D = wl["H"].shape[2]
+        g = torch.Generator().manual_seed(35)
+        wl["gamma"] = (1 + 0.2 * torch.randn(D, generator=g)).float().to(device)
+        wl["beta"] = (0.05 * torch.randn(D, generator=g)).float().to(device)
+    if inject:
+        M = wl.get("M", max(1, (wl["K"] - 1).bit_length()))
+        C = wl["R"] * M
+        D_out = 2048 if cfg == 3 else C
+        wl["M_inj"], wl["D_out"] = M, D_out
+        wl["e0"] = W.bf16_normal((C,), 36, device)
+        wl["e1"] = W.bf16_normal((C,), 37, device)
+        wl["W_out"] = W.bf16_normal((D_out, C), 38, device, std=C ** -0.5)
+
+
+def build_workload(cfg: int, device, seed_offset: int = 0, shard=None, fused=False):
     """Returns a dict with device inputs and the sizes of every op of a step.
 
     ``shard`` = (world, rank) keeps only this rank's streams (stream split);
@@ -120,17 +148,23 @@ def build_workload(cfg: int, device, seed_offset: int = 0, shard=None):
                                              seed_h=3 + 1000 * seed_offset)
         R_all = ch // M
         _, r0, r1 = shard_plan(1, R_all, True, world, rank)
-        # projection = set-up, outside the timed step; a rank keeps its routes' channels
-        wl["qvec"] = (H @ Wq)[:, :, r0 * M:r1 * M].contiguous()
-        wl["kvec"] = (H @ Wk)[:, :, r0 * M:r1 * M].contiguous()
-        del H
+        if fused:
+            # the step starts from the hidden states: layer norm + projection + discretisation
+            wl["H"] = H
+            wl["Wq"] = Wq[:, r0 * M:r1 * M].contiguous()
+            wl["Wk"] = Wk[:, r0 * M:r1 * M].contiguous()
+        else:
+            # projection = set-up, outside the timed step; a rank keeps its routes' channels
+            wl["qvec"] = (H @ Wq)[:, :, r0 * M:r1 * M].contiguous()
+            wl["kvec"] = (H @ Wk)[:, :, r0 * M:r1 * M].contiguous()
+            del H
         R = r1 - r0
         wl.update(name=c["name"], B=1, R=R, T=T, K=2 ** M, g=2, S=R, same=False, M=M, d=d, rho=rho,
                   shard={"routes": [r0, r1], "of": R_all})
         V = W.value_rows(1, T, R_all * rho, seed=c["seed_v"] + 1000 * seed_offset, device=device)
         wl["V"] = V[:, :, r0 * rho:r1 * rho].contiguous()
         del V
-        wl["ops"] = ["discretize", "match", "gather"]
+        wl["ops"] = ["ln_project" if fused else "discretize", "match", "gather"]
         return wl
     c = W.WORKLOADS[cfg]
     if seed_offset:
@@ -204,6 +238,25 @@ def algorithmic_bytes(wl):
     if "gather" in wl["ops"]:
         # end_idx (4 B) + d bf16 read + d bf16 written per (position, route)
         out["gather"] = wl["B"] * T * wl["R"] * (4 + 2 * wl["d"] * 2)
+    if "ln_project" in wl["ops"]:
+        # hidden states read (bf16) + query and key symbols written (1 B per route each)
+        B_, _, D = wl["H"].shape
+        out["ln_project"] = B_ * T * D * 2 + 2 * B_ * wl["R"] * T
+    if "inject" in wl["ops"]:
+        # recalled symbols read (int32 per route) + injection written (bf16 per output column)
+        out["inject"] = wl["B"] * T * (wl["R"] * 4 + wl["D_out"] * 2)
+    return out
+
+
+def algorithmic_flops(wl):
+    """Dense contractions of the step (2 flops per multiply-add)."""
+    T = wl["T"]
+    out = {}
+    if "ln_project" in wl["ops"]:
+        B_, _, D = wl["H"].shape
+        out["ln_project"] = 2 * B_ * T * D * 2 * wl["R"] * wl["M"]
+    if "inject" in wl["ops"]:
+        out["inject"] = 2 * wl["B"] * T * wl["R"] * wl["M_inj"] * wl["D_out"]
     return out
 
 
@@ -231,6 +284,14 @@ class Runner:
             self.sk = torch.empty_like(self.sq)
         if "gather" in wl["ops"]:
             self.gout = torch.empty((wl["B"], T, wl["R"] * wl["d"]), dtype=torch.bfloat16, device=device)
+        if "ln_project" in wl["ops"]:
+            B_, _, D = wl["H"].shape
+            self.sq = torch.empty((B_, wl["R"], T), dtype=torch.uint8, device=device)
+            self.sk = torch.empty_like(self.sq)
+            self.lws = torch.empty(rosa.ln_project_workspace_size(D, wl["R"] * wl["M"], wl["M"]), dtype=torch.uint8,
+                                   device=device)
+        if "inject" in wl["ops"]:
+            self.iout = torch.empty((wl["B"], T, wl["D_out"]), dtype=torch.bfloat16, device=device)
         self.graphs = None
 
     def host_outputs(self):
@@ -241,8 +302,10 @@ class Runner:
         out = {"match": tuple(o.cpu().numpy() for o in self.outs[:3])}
         if wl.get("cf"):
             out["cf"] = tuple(o.cpu().numpy() for o in self.outs[3:])
-        if "discretize" in wl["ops"]:
+        if "discretize" in wl["ops"] or "ln_project" in wl["ops"]:
             out["discretize"] = (self.sq.cpu().numpy(), self.sk.cpu().numpy())
+        if "inject" in wl["ops"]:
+            out["inject"] = self.iout
         if "gather" in wl["ops"]:
             out["gather"] = lambda b: bits(self.gout[b:b + 1])
             out["V_bits"] = lambda b: bits(wl["V"][b:b + 1])
@@ -256,6 +319,8 @@ class Runner:
             count = self.rosa.match_rle_launch_count if wl.get("rle") else self.rosa.match_launch_count
             n = count(wl["S"], wl["T"], wl["K"], wl["same"])
         n += 1 if "discretize" in wl["ops"] else 0
+        n += 2 if "ln_project" in wl["ops"] else 0
+        n += 1 if "inject" in wl["ops"] else 0
         n += 1 if "gather" in wl["ops"] else 0
         return n
 
@@ -263,8 +328,13 @@ class Runner:
         rosa, wl = self.rosa, self.wl
         if name == "discretize":
             rosa.discretize_pair(wl["qvec"], wl["kvec"], wl["M"], out=(self.sq, self.sk))
+        elif name == "ln_project":
+            rosa.ln_project_discretize(wl["H"], wl["Wq"], wl["Wk"], wl["M"], wl["gamma"], wl["beta"],
+                                       out=(self.sq, self.sk), workspace=self.lws)
+        elif name == "inject":
+            rosa.inject(self.outs[2], wl["e0"], wl["e1"], wl["W_out"], wl["B"], wl["R"], wl["M_inj"], out=self.iout)
         elif name == "match":
-            if "discretize" in wl["ops"]:
+            if "discretize" in wl["ops"] or "ln_project" in wl["ops"]:
                 q, k = self.sq.view(wl["S"], wl["T"]), self.sk.view(wl["S"], wl["T"])
             else:
                 q, k = wl["q"], wl["k"]
@@ -410,6 +480,14 @@ def profiled_traffic(workload: str, op: str):
     return nbytes if digest == cuda_source_digest() else None
 
 
+def load_tensor_peak():
+    """Dense bf16 tensor-core peak in TFLOP/s (measured burst figure, else the fallback)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p)).get("bf16_tflops", 1590.0))
+    return 1590.0
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -425,11 +503,12 @@ def oracle_symbols(wl):
     streams, or for the hidden-state workload the oracle's discretisation of
     the same projected bf16 tensors."""
     import oracle
-    if wl["cfg"] == 3:
+    if "qvec" in wl:
         import torch
         bits = lambda t: t.cpu().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
         sq, sk = oracle.discretize(bits(wl["qvec"]), wl["M"]), oracle.discretize(bits(wl["kvec"]), wl["M"])
         return sq.reshape(wl["S"], wl["T"]), sk.reshape(wl["S"], wl["T"]), (sq, sk)
+    # symbol workloads, and the fused front end (whose symbols are checked on their own)
     return wl["q_host"], wl["k_host"], None
 
 
@@ -527,7 +606,74 @@ def check_parity(wl, got, ref):
             if not np.array_equal(have, want):
                 return False, f"gather differs in batch element {b} at {_first_diff(have, want)}"
         checked.append("gather (whole output)")
+    if "ln_project" in wl.get("ops", ()):
+        ok, text = check_ln_project(wl, got["discretize"])
+        if not ok:
+            return False, text
+        checked.append(text)
+    if "inject" in got:
+        ok, text = check_inject(wl, got["inject"], ref["match"][2], n)
+        if not ok:
+            return False, text
+        checked.append(text)
     return True, "bit-exact vs the CPU oracle: " + ", ".join(checked)
+
+
+def _f64(bits):
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def check_ln_project(wl, sym_pair, rows=4096):
+    """Fused layer norm + projection + discretisation on the first ``rows``
+    positions: every bit whose exact projection lies outside the kernel's
+    rounding band must match (the band is derived in tests/test_gpu_ln_project.py)."""
+    import oracle
+    import torch
+    bits = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    H = bits(wl["H"])[0, :rows]
+    W = np.concatenate([bits(wl["Wq"]), bits(wl["Wk"])], axis=1)
+    g, b = wl["gamma"].cpu().numpy(), wl["beta"].cpu().numpy()
+    P, _ = oracle.ln_project(H, W, g, b, eps=1e-5)
+    D = H.shape[1]
+    h = _f64(H)
+    mu = h.mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(((h - mu) ** 2).mean(axis=1, keepdims=True) + 1e-5)
+    gw = np.abs(g.astype(np.float64)[:, None] * _f64(W))
+    bw = np.abs(b.astype(np.float64)[:, None] * _f64(W)).sum(axis=0)
+    band = (rstd * (2.0 ** -16 + 2 * D * 2.0 ** -24) * (np.abs(h) @ gw)
+            + D * 2.0 ** -24 * (np.abs(mu) * rstd * gw.sum(axis=0) + bw) + 2.0 ** -20 * np.abs(P))
+    M, R = wl["M"], wl["R"]
+    got = []
+    for sym in sym_pair:                      # [1, R, T] -> [rows, R*M] bits
+        s_ = sym[0, :, :rows].T
+        got.append(((s_[..., None] >> np.arange(M)) & 1).reshape(rows, R * M))
+    got = np.concatenate(got, axis=1)
+    sure = np.abs(P) > band
+    bad = (got != (P > 0)) & sure
+    if bad.any():
+        return False, f"fused front end: {bad.sum()} bits outside the rounding band differ"
+    return True, f"fused front end ({rows} positions; {float((~sure).mean()):.4%} of bits inside the rounding band)"
+
+
+def check_inject(wl, inj, sym_oracle, n, positions=2048):
+    """Injection on the first ``positions`` of every batch element, within the
+    fp32-accumulation / bf16-rounding bound (tests/test_gpu_inject.py)."""
+    import oracle
+    import torch
+    bits = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    B, R, M, T = wl["B"], wl["R"], wl["M_inj"], wl["T"]
+    if n != wl["S"]:
+        return True, "injection (not checked: the oracle leg covered part of the streams)"
+    ts = min(T, positions)
+    sym = np.ascontiguousarray(sym_oracle.reshape(B * R, T)[:, :ts])
+    e0, e1, W = bits(wl["e0"]), bits(wl["e1"]), bits(wl["W_out"])
+    ref = oracle.inject(sym, e0, e1, W, B, R, M)
+    mag = oracle.inject(sym, e0 & 0x7FFF, e1 & 0x7FFF, W & 0x7FFF, B, R, M)
+    got = _f64(bits(inj[:, :ts]))
+    tol = 2.0 ** -8 * np.abs(ref) + R * M * 2.0 ** -23 * mag + 1e-30
+    if (np.abs(got - ref) > tol).any():
+        return False, f"injection: {(np.abs(got - ref) > tol).sum()} entries outside the error bound"
+    return True, f"injection ({ts} positions per batch element, within the fp32/bf16 bound)"
 
 
 # --------------------------------------------------------------------------- main
@@ -557,8 +703,15 @@ def main():
         dist.barrier()
 
     replicas = args.split == "replicas"
+    if args.fused and args.config != 3:
+        raise SystemExit("--fused applies to qwen-proj-64 (--config 3), the workload that starts from hidden states")
+    if args.inject and args.config not in (3, 5):
+        raise SystemExit("--inject applies to the workloads with recalled values: --config 3 or 5")
     wl = build_workload(args.config, device, seed_offset=rank if replicas else 0,
-                        shard=None if replicas else (world, rank))
+                        shard=None if replicas else (world, rank), fused=args.fused)
+    dense_params(wl, args.config, device, args.fused, args.inject)
+    if args.inject:
+        wl["ops"].append("inject")
     if args.streams and wl["cfg"] != 3 and args.streams < wl["S"]:
         shrink_streams(wl, args.streams)
     wl["rle"] = args.rle
@@ -605,6 +758,10 @@ def main():
         dist.barrier()
     clocks = sampler.stop()
     timed_outputs = runner.host_outputs()   # the last timed step's results, for the parity check
+    if "ln_project" in wl["ops"]:
+        # the match is checked on the symbols the fused front end produced (checked on their own)
+        sq, sk = timed_outputs["discretize"]
+        wl["q_host"], wl["k_host"] = sq.reshape(wl["S"], wl["T"]), sk.reshape(wl["S"], wl["T"])
 
     step_ms = [a.elapsed_time(b) for a, b, _ in per_step]
     for _, _, ev in per_step:
@@ -620,13 +777,24 @@ def main():
     dom = max(mean_op, key=mean_op.get)
     peak, peak_kind = load_peaks()
     achieved = ab[dom] / (mean_op[dom] / 1e3) / 1e9
+    fl = algorithmic_flops(wl)
+    tf_peak = load_tensor_peak()
+    ops_roof = {}
+    for o, v in mean_op.items():
+        gbs = ab[o] / (v / 1e3) / 1e9
+        ops_roof[o] = {"ms": round(v, 4), "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peak, 4)}
+        if o in fl:
+            tfs = fl[o] / (v / 1e3) / 1e12
+            ops_roof[o].update({"TFLOP/s": round(tfs, 1), "tensor_frac": round(tfs / tf_peak, 4)})
     roofline = {"bound": "hbm", "kernel": f"rosa_{dom}", "achieved": round(achieved, 2), "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 5),
                 "traffic": profiled_traffic(wl["name"], dom), "algorithmic_bytes": ab[dom],
-                "ms": round(mean_op[dom], 4), "ops_ms": {o: round(v, 4) for o, v in mean_op.items()}}
+                "ms": round(mean_op[dom], 4), "ops_ms": {o: round(v, 4) for o, v in mean_op.items()},
+                "ops": ops_roof}
 
     e2e = None
-    if not args.no_e2e and not args.cf:   # the counterfactual op is measured on the device only
+    # the counterfactual, fused and injection variants are measured on the device only
+    if not args.no_e2e and not args.cf and not args.fused and not args.inject:
         e2e = end_to_end(wl, device, args.steps)
         # every rank takes the same collective steps
         e_ms, e_units = reduce_over_ranks(e2e["ms_per_step"] * args.steps, positions * args.steps, device)

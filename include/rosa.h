@@ -234,6 +234,32 @@ ROSA_API int rosa_match_noalloc(const uint8_t *q, const uint8_t *k, const uint8_
 ROSA_API int rosa_match_noalloc_device_status(cudaStream_t stream, uint32_t *status);
 
 /*
+ * Layer norm, query/key projection and discretisation in one pass, on the
+ * tensor cores (section 3.2: U = LN(H), Q = U W_q, K = U W_k, then the
+ * strict threshold and packing of Eqs. 10-15).
+ *
+ *   H       [B, T, D] bf16 hidden states, row-major (16-byte aligned, D % 8 == 0).
+ *   gamma, beta [D] float layer-norm scale and shift, or NULL (1 and 0).
+ *   Wq, Wk  [D, C] bf16 projections, row-major; C % M == 0.
+ *   symq, symk [B, C/M, T] uint8, written in full:
+ *     u = gamma * (h - mean(h)) / sqrt(var(h) + eps) + beta  (population variance)
+ *     sym[b, r, t] = sum_j I[(u W)[c = r*M + j] > 0] * 2^j
+ * The layer norm is folded into the contraction (the kernels multiply the raw
+ * rows by gamma o W, kept to about 16 significant bits as a bf16 high + low
+ * pair, with fp32 accumulation), so a channel whose exact projection lies
+ * within that rounding of zero may take either bit.
+ * `workspace` holds the prepared weights: at least
+ * rosa_ln_project_workspace_size(D, C, M) bytes, 256-byte aligned.
+ * dev_status: optional device word (ROSA_DEV_TIMEOUT if a bounded wait ran out).
+ * Requires B, T >= 0, D >= 8, D % 8 == 0, 1 <= M <= 8, C >= M.
+ */
+ROSA_API size_t rosa_ln_project_workspace_size(int D, int C, int M);
+ROSA_API int rosa_ln_project_discretize(const rosa_bf16 *H, const float *gamma, const float *beta,
+                                        const rosa_bf16 *Wq, const rosa_bf16 *Wk, int B, int T, int D, int C, int M,
+                                        float eps, uint8_t *symq, uint8_t *symk, void *workspace, size_t ws_bytes,
+                                        uint32_t *dev_status, cudaStream_t stream);
+
+/*
  * Read-out embedding and injection (appendix C.3, Eqs. 21-22 of the main
  * text, with the Eq. 17 mask), on the tensor cores.
  *

@@ -51,6 +51,11 @@ lib.rosa_match_launch_count.argtypes = [_i, _i, _i, _i]
 lib.rosa_match_launch_count.restype = _i
 lib.rosa_match_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
 lib.rosa_match_device_status.restype = _i
+lib.rosa_ln_project_workspace_size.argtypes = [_i, _i, _i]
+lib.rosa_ln_project_workspace_size.restype = ctypes.c_size_t
+lib.rosa_ln_project_discretize.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp,
+                                           _vp, ctypes.c_size_t, _vp, _vp]
+lib.rosa_ln_project_discretize.restype = _i
 lib.rosa_inject.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]
 lib.rosa_inject.restype = _i
 lib.rosa_gather.argtypes = [_vp, _i64, _i64, _vp, _i, _i, _i, _i, _vp, _vp]
@@ -59,7 +64,8 @@ lib.rosa_gather.restype = _i
 EXPORTED = ("rosa_status_string", "rosa_discretize", "rosa_discretize_pair", "rosa_match_workspace_size", "rosa_match",
             "rosa_match_launch_count", "rosa_match_device_status", "rosa_gather", "rosa_match_rle",
             "rosa_match_rle_workspace_size", "rosa_match_rle_launch_count", "rosa_match_cf",
-            "rosa_match_cf_workspace_size", "rosa_match_cf_launch_count", "rosa_inject")
+            "rosa_match_cf_workspace_size", "rosa_match_cf_launch_count", "rosa_inject",
+            "rosa_ln_project_discretize", "rosa_ln_project_workspace_size")
 
 DEV_SYMBOL_RANGE = 1
 
@@ -312,4 +318,45 @@ def inject(sym: torch.Tensor, e0: torch.Tensor, e1: torch.Tensor, W_out: torch.T
         out = torch.empty((B, T, D), dtype=torch.bfloat16, device=sym.device)
     _check(lib.rosa_inject(_ptr(sym), _ptr(e0), _ptr(e1), _ptr(W_out), B, R, M, T, D, _ptr(out),
                            _ptr(status), _stream(sym.device)), "rosa_inject")
+    return out
+
+
+def ln_project_workspace_size(D: int, C: int, M: int) -> int:
+    n = lib.rosa_ln_project_workspace_size(D, C, M)
+    if n == 0:
+        raise ValueError(f"invalid sizes D={D} C={C} M={M}")
+    return n
+
+
+def ln_project_discretize(H: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, M: int,
+                          gamma: torch.Tensor | None = None, beta: torch.Tensor | None = None, eps: float = 1e-5,
+                          out=None, workspace: torch.Tensor | None = None, status: torch.Tensor | None = None):
+    """U = LN(H), the query and key projections, threshold and packing in one
+    pass (section 3.2): ``H`` bf16 ``[B, T, D]``, ``Wq``, ``Wk`` bf16
+    ``[D, C]``, ``gamma``, ``beta`` float32 ``[D]`` or None ->
+    ``(sym_q, sym_k)``, uint8 ``[B, C // M, T]`` each."""
+    _need_cuda(H, Wq, Wk, gamma, beta, workspace, status)
+    if H.dtype != torch.bfloat16 or H.dim() != 3:
+        raise ValueError("H must be bf16 [B, T, D]")
+    for w in (Wq, Wk):
+        if w.dtype != torch.bfloat16 or w.dim() != 2:
+            raise ValueError("Wq and Wk must be bf16 [D, C]")
+    for v in (gamma, beta):
+        if v is not None and v.dtype != torch.float32:
+            raise ValueError("gamma and beta must be float32 [D]")
+    H, Wq, Wk = H.contiguous(), Wq.contiguous(), Wk.contiguous()
+    gamma = None if gamma is None else gamma.contiguous()
+    beta = None if beta is None else beta.contiguous()
+    B, T, D = H.shape
+    C = Wq.shape[1]
+    if Wq.shape != (D, C) or Wk.shape != (D, C):
+        raise ValueError("Wq and Wk must both be [D, C]")
+    if out is None:
+        out = tuple(torch.empty((B, C // M, T), dtype=torch.uint8, device=H.device) for _ in range(2))
+    if workspace is None:
+        workspace = torch.empty(ln_project_workspace_size(D, C, M), dtype=torch.uint8, device=H.device)
+    _check(lib.rosa_ln_project_discretize(_ptr(H), _ptr(gamma), _ptr(beta), _ptr(Wq), _ptr(Wk), B, T, D, C, M,
+                                          float(eps), _ptr(out[0]), _ptr(out[1]), _vp(workspace.data_ptr()),
+                                          workspace.numel(), _ptr(status), _stream(H.device)),
+           "rosa_ln_project_discretize")
     return out

@@ -48,6 +48,12 @@ int match_rle_launch_count(int S, int T, int K, bool same);
 cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t *e1, const uint16_t *W, int B, int R,
                           int M, int T, int D, uint16_t *out, uint32_t *status, cudaStream_t stream);
 
+// Layer norm + projection + discretisation on the tensor cores (ln_project.cu).
+size_t ln_project_workspace_bytes(int D, int C, int M);
+cudaError_t launch_ln_project(const uint16_t *H, const float *gamma, const float *beta, const uint16_t *Wq,
+                              const uint16_t *Wk, int B, int T, int D, int C, int M, float eps, uint8_t *symq,
+                              uint8_t *symk, void *workspace, size_t ws_bytes, uint32_t *status, cudaStream_t stream);
+
 // Offset of the device status word inside a matcher workspace.
 constexpr size_t kStatusOffset = 0;
 

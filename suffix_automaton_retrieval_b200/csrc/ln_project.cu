@@ -1,0 +1,329 @@
+// Layer norm, query/key projection and discretisation fused on the tensor
+// cores.
+//
+// "ROSA-Tuning" (arXiv 2602.02499), section 3.2: U = LN(H), Q = U W_q,
+// K = U W_k, then the strict threshold I[x > 0] and multi-route packing
+// (Eqs. 10-15; channel c = r*M + j carries bit j of route r's symbol).
+//
+// The layer norm is folded into the contraction:
+//   U W = rstd * (H (gamma o W) - mu * colsum(gamma o W)) + beta W,
+// with mu and rstd the row's mean and reciprocal standard deviation.  The
+// tensor cores therefore consume the raw rows of H, which arrive in shared
+// memory by TMA (128-byte swizzle, mbarrier completion, two stages), and the
+// same shared-memory tiles give each row's sums of h and h^2.  The scaled
+// weights gamma o W are split into bf16 high and low parts (hi + lo carries
+// about 16 significant bits) that are multiplied as two halves of one MMA
+// (N = 2 x the effective columns), so the weights lose almost nothing to
+// bf16.  The epilogue reads both halves from tensor memory, applies the
+// fold, thresholds and packs the bits of each route, and writes the symbol
+// bytes of the query and key streams.
+//
+// Effective columns n < C are query channels, C <= n < 2C key channels; a
+// CTA covers NE of them (a multiple of both 8 and M, at most 128).
+#include <cstdint>
+#include <mutex>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/rosa.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "umma.cuh"
+
+namespace rosa {
+namespace {
+
+constexpr int kLnpM = 128;          // rows per tile
+constexpr int kLnpK = 64;           // K per block (one 128-byte swizzle row)
+constexpr int kLnpThreads = 128;
+constexpr int kLnpStages = 2;
+constexpr uint32_t kLnpWaitPolls = 1u << 24;
+
+int gcd_int(int a, int b) { return b ? gcd_int(b, a % b) : a; }
+
+// Effective columns per CTA: the largest multiple of lcm(M, 8) up to 128.
+int lnp_ne(int M) {
+    const int l = 8 * M / gcd_int(8, M);
+    return (128 / l) * l;
+}
+
+struct LnpSmem {
+    alignas(1024) unsigned char a[kLnpStages][kLnpM * 128];   // H block, K-major SW128
+    alignas(1024) unsigned char b[kLnpStages][256 * 128];     // hi / lo weight rows, K-major SW128
+    uint64_t full[kLnpStages], done[kLnpStages];
+    uint32_t tmem;
+    int failed;
+};
+
+struct LnpLayout {
+    uint16_t *wp;     // [NT * 2NE rows][D]: per tile NE high rows then NE low rows
+    float *cs;        // [NT * NE]: column sums of hi + lo
+    float *bv;        // [NT * NE]: beta . W
+    size_t bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+LnpLayout lnp_carve(int D, int C, int M, void *base) {
+    const int NE = lnp_ne(M), NT = ceil_div(2 * C, NE);
+    LnpLayout L{};
+    char *b = static_cast<char *>(base);
+    size_t off = 0;
+    auto take = [&](size_t n) -> void * {
+        void *p = b ? b + off : nullptr;
+        off += align256(n);
+        return p;
+    };
+    L.wp = (uint16_t *)take((size_t)NT * 2 * NE * D * 2);
+    L.cs = (float *)take((size_t)NT * NE * 4);
+    L.bv = (float *)take((size_t)NT * NE * 4);
+    L.bytes = off;
+    return L;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<const uint16_t *>(&h);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// One CTA per effective column (padding columns of the last tile write zeros).
+__global__ void __launch_bounds__(256)
+lnp_prep_kernel(const float *__restrict__ gamma, const float *__restrict__ beta, const uint16_t *__restrict__ Wq,
+                const uint16_t *__restrict__ Wk, int D, int C, int NE, uint16_t *__restrict__ wp, float *__restrict__ cs,
+                float *__restrict__ bv) {
+    __shared__ float red[2][8];
+    const int n = blockIdx.x;
+    const int tile = n / NE, cn = n - tile * NE;
+    uint16_t *hi = wp + ((int64_t)tile * 2 * NE + cn) * D;
+    uint16_t *lo = wp + ((int64_t)tile * 2 * NE + NE + cn) * D;
+    float s_cs = 0.f, s_bv = 0.f;
+    for (int k = threadIdx.x; k < D; k += 256) {
+        uint16_t h = 0, l = 0;
+        if (n < 2 * C) {
+            const float w = bf16_bits_to_float(n < C ? Wq[(int64_t)k * C + n] : Wk[(int64_t)k * C + n - C]);
+            const float ws = (gamma ? gamma[k] : 1.f) * w;
+            h = bf16_bits_rn(ws);
+            l = bf16_bits_rn(ws - bf16_bits_to_float(h));
+            s_cs += bf16_bits_to_float(h) + bf16_bits_to_float(l);
+            s_bv += (beta ? beta[k] : 0.f) * w;
+        }
+        hi[k] = h;
+        lo[k] = l;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        s_cs += __shfl_xor_sync(ROSA_FULL_MASK, s_cs, o);
+        s_bv += __shfl_xor_sync(ROSA_FULL_MASK, s_bv, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = s_cs;
+        red[1][threadIdx.x >> 5] = s_bv;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.f, c = 0.f;
+        for (int w = 0; w < 8; ++w) {
+            a += red[0][w];
+            c += red[1][w];
+        }
+        cs[n] = a;
+        bv[n] = c;
+    }
+}
+
+__global__ void __launch_bounds__(kLnpThreads, 1)
+lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, int64_t P, int T, int D,
+           int C, int M, int NE, float eps, const float *__restrict__ cs, const float *__restrict__ bv,
+           uint8_t *__restrict__ symq, uint8_t *__restrict__ symk, uint32_t *__restrict__ status) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    LnpSmem &sm = *reinterpret_cast<LnpSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t p0 = (int64_t)blockIdx.x * kLnpM;
+    const int tile = blockIdx.y;
+    const int N = 2 * NE;                               // MMA N: high then low halves
+    const uint32_t a_bytes = kLnpM * 128, b_bytes = (uint32_t)N * 128;
+    const int nkb = ceil_div(D, kLnpK);
+
+    if (tid == 0) {
+        for (int s = 0; s < kLnpStages; ++s) {
+            umma::mbar_init(&sm.full[s], 1);
+            umma::mbar_init(&sm.done[s], 1);
+        }
+        umma::fence_mbar_init();
+        sm.failed = 0;
+    }
+    if (warp == 0) umma::tmem_alloc(&sm.tmem, 256);
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+
+    if (tid == 0) {
+        for (int s = 0; s < kLnpStages && s < nkb; ++s) {
+            umma::mbar_arrive_expect_tx(&sm.full[s], a_bytes + b_bytes);
+            umma::tma_load_2d(sm.a[s], &tmH, s * kLnpK, (int)p0, &sm.full[s]);
+            umma::tma_load_2d(sm.b[s], &tmW, s * kLnpK, tile * N, &sm.full[s]);
+        }
+    }
+    const uint32_t idesc = umma::make_idesc_bf16_f32(kLnpM, N);
+    float s1 = 0.f, s2 = 0.f;   // this thread's row: sum of h and of h^2
+    for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb & 1;
+        const uint32_t ph = (uint32_t)((kb >> 1) & 1);
+        if (!umma::mbar_wait_bounded(&sm.full[s], ph, kLnpWaitPolls)) sm.failed = 1;
+        if (!sm.failed) {
+            const unsigned char *row = sm.a[s] + tid * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + ((ch ^ (tid & 7)) << 4));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float lo = __uint_as_float(w4[h] << 16), hi = __uint_as_float(w4[h] & 0xffff0000u);
+                    s1 += lo + hi;
+                    s2 += lo * lo + hi * hi;
+                }
+            }
+        }
+        if (tid == 0 && !sm.failed) {
+            umma::tc_fence_after();
+            const uint32_t abase = umma::smem_u32(sm.a[s]), bbase = umma::smem_u32(sm.b[s]);
+#pragma unroll
+            for (int kk = 0; kk < kLnpK / 16; ++kk)
+                umma::mma_bf16(tmem, umma::make_kmajor_sw128_desc(abase + kk * 32),
+                               umma::make_kmajor_sw128_desc(bbase + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            umma::mma_commit(&sm.done[s]);
+        }
+        __syncthreads();   // every row's statistics read of stage s is done
+        if (sm.failed) break;
+        if (kb + kLnpStages < nkb && tid == 0) {
+            // refill stage s once its MMAs have read it
+            if (!umma::mbar_wait_bounded(&sm.done[s], ph, kLnpWaitPolls)) {
+                sm.failed = 1;
+            } else {
+                umma::mbar_arrive_expect_tx(&sm.full[s], a_bytes + b_bytes);
+                umma::tma_load_2d(sm.a[s], &tmH, (kb + kLnpStages) * kLnpK, (int)p0, &sm.full[s]);
+                umma::tma_load_2d(sm.b[s], &tmW, (kb + kLnpStages) * kLnpK, tile * N, &sm.full[s]);
+            }
+        }
+    }
+    // the last commit covers every MMA of the tile
+    if (!sm.failed && nkb > 0) {
+        const int kl = nkb - 1;
+        if (!umma::mbar_wait_bounded(&sm.done[kl & 1], (uint32_t)((kl >> 1) & 1), kLnpWaitPolls)) sm.failed = 1;
+    }
+    __syncthreads();
+    umma::tc_fence_after();
+    if (!sm.failed) {
+        // epilogue: thread = row (TMEM lane 32*warp + lane)
+        const int64_t p = p0 + tid;
+        const float mu = s1 / (float)D;
+        const float var = fmaxf(s2 / (float)D - mu * mu, 0.f);
+        const float rstd = rsqrtf(var + eps);
+        uint32_t bits[4] = {0, 0, 0, 0};   // threshold bits of the NE effective columns
+        for (int c0 = 0; c0 < NE; c0 += 32) {
+            uint32_t h[32], l[32];
+            umma::tmem_ld_32cols(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, h);
+            umma::tmem_ld_32cols(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(NE + c0), l);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int cn = c0 + j;
+                if (cn < NE) {
+                    const int n = tile * NE + cn;
+                    const float acc = __uint_as_float(h[j]) + __uint_as_float(l[j]);
+                    const float x = rstd * (acc - mu * cs[n]) + bv[n];
+                    if (x > 0.f) bits[cn >> 5] |= 1u << (cn & 31);
+                }
+            }
+        }
+        if (p < P) {
+            const int64_t b = p / T, t = p - b * T;
+            const int R = C / M;
+            for (int cn = 0; cn < NE; cn += M) {
+                const int n = tile * NE + cn;
+                if (n >= 2 * C) break;
+                unsigned a = 0;
+                for (int j = 0; j < M; ++j) a |= ((bits[(cn + j) >> 5] >> ((cn + j) & 31)) & 1u) << j;
+                const bool isq = n < C;
+                const int r = (isq ? n : n - C) / M;
+                (isq ? symq : symk)[(b * R + r) * (int64_t)T + t] = (uint8_t)a;
+            }
+        }
+    } else if (tid == 0 && status) {
+        atomicOr(status, ROSA_DEV_TIMEOUT);
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, 256);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill outside.
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t lnp_smem_bytes() { return sizeof(LnpSmem) + 1024; }
+
+}  // namespace
+
+size_t ln_project_workspace_bytes(int D, int C, int M) { return lnp_carve(D, C, M, nullptr).bytes; }
+
+cudaError_t launch_ln_project(const uint16_t *H, const float *gamma, const float *beta, const uint16_t *Wq,
+                              const uint16_t *Wk, int B, int T, int D, int C, int M, float eps, uint8_t *symq,
+                              uint8_t *symk, void *workspace, size_t ws_bytes, uint32_t *status, cudaStream_t st) {
+    const LnpLayout L = lnp_carve(D, C, M, workspace);
+    if (L.bytes > ws_bytes) return cudaErrorInvalidValue;
+    const int64_t P = (int64_t)B * T;
+    if (P == 0) return cudaSuccess;
+    const int NE = lnp_ne(M), NT = ceil_div(2 * C, NE);
+    CUtensorMap tmH, tmW;
+    if (!make_tmap(&tmH, H, (uint64_t)P, (uint64_t)D, kLnpM) ||
+        !make_tmap(&tmW, L.wp, (uint64_t)NT * 2 * NE, (uint64_t)D, (uint32_t)(2 * NE)))
+        return cudaErrorInvalidValue;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int smem = (int)lnp_smem_bytes();
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        e = cudaFuncSetAttribute(lnp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+    }
+    lnp_prep_kernel<<<(unsigned)(NT * NE), 256, 0, st>>>(gamma, beta, Wq, Wk, D, C, NE, L.wp, L.cs, L.bv);
+    dim3 grid((unsigned)ceil_div64(P, kLnpM), (unsigned)NT);
+    lnp_kernel<<<grid, kLnpThreads, smem, st>>>(tmH, tmW, P, T, D, C, M, NE, eps, L.cs, L.bv, symq, symk, status);
+    return cudaGetLastError();
+}
+
+}  // namespace rosa

@@ -132,6 +132,30 @@ int rosa_match_device_status(const void *workspace, cudaStream_t stream, uint32_
     return ROSA_OK;
 }
 
+namespace {
+bool lnp_sizes_ok(int D, int C, int M) {
+    return D >= 8 && D % 8 == 0 && M >= 1 && M <= 8 && C >= M && C % M == 0 && C <= (1 << 16) && D <= (1 << 20);
+}
+}  // namespace
+
+size_t rosa_ln_project_workspace_size(int D, int C, int M) {
+    if (!lnp_sizes_ok(D, C, M)) return 0;
+    return rosa::ln_project_workspace_bytes(D, C, M);
+}
+
+int rosa_ln_project_discretize(const rosa_bf16 *H, const float *gamma, const float *beta, const rosa_bf16 *Wq,
+                               const rosa_bf16 *Wk, int B, int T, int D, int C, int M, float eps, uint8_t *symq,
+                               uint8_t *symk, void *workspace, size_t ws_bytes, uint32_t *dev_status,
+                               cudaStream_t stream) {
+    if (B < 0 || T < 0 || !lnp_sizes_ok(D, C, M) || !(eps >= 0.f)) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)B * T >= ((int64_t)1 << 31)) return ROSA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!H || !Wq || !Wk || !symq || !symk || !aligned(H, 16))) return ROSA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256)) return ROSA_ERR_WORKSPACE;
+    if (ws_bytes < rosa::ln_project_workspace_bytes(D, C, M)) return ROSA_ERR_WORKSPACE;
+    return cuda_status(rosa::launch_ln_project(H, gamma, beta, Wq, Wk, B, T, D, C, M, eps, symq, symk, workspace,
+                                               ws_bytes, dev_status, stream));
+}
+
 int rosa_inject(const int32_t *sym, const rosa_bf16 *e0, const rosa_bf16 *e1, const rosa_bf16 *W_out, int B, int R,
                 int M, int T, int D, rosa_bf16 *inj, uint32_t *dev_status, cudaStream_t stream) {
     if (B < 0 || T < 0 || R < 1 || M < 1 || M > 8 || D < 1) return ROSA_ERR_INVALID_ARG;
