@@ -14,6 +14,7 @@
 // fp32 accumulator in tensor memory.  The epilogue reads the accumulator
 // back with tcgen05.ld, rounds to bf16 and stores the rows.
 #include <cstdint>
+#include <cstring>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,6 +36,7 @@ struct InjSmem {
     alignas(1024) unsigned char a[kInjM * 128];        // y block, K-major SW128
     alignas(1024) unsigned char b[kInjMaxN * 128];     // W_out block, K-major SW128
     uint16_t e0[kInjK], e1[kInjK];
+    int32_t sym[kInjK][kInjM];                         // recalled symbols of the block's routes, per row
     uint64_t mbar;
     uint32_t tmem;
     int failed;
@@ -46,9 +48,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __global__ void __launch_bounds__(kInjThreads, 1)
-inject_kernel(const int32_t *__restrict__ sym, const uint16_t *__restrict__ e0, const uint16_t *__restrict__ e1,
-              const uint16_t *__restrict__ W, int R, int M, int T, int D, int BN, int64_t P, bool wvec,
-              uint16_t *__restrict__ out, uint32_t *__restrict__ status) {
+inject_kernel(const __grid_constant__ CUtensorMap tmOut, bool tma_out, const int32_t *__restrict__ sym,
+              const uint16_t *__restrict__ e0, const uint16_t *__restrict__ e1, const uint16_t *__restrict__ W, int R,
+              int M, int T, int D, int BN, int64_t P, bool wvec, uint16_t *__restrict__ out,
+              uint32_t *__restrict__ status) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     InjSmem &sm = *reinterpret_cast<InjSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -85,38 +88,38 @@ inject_kernel(const int32_t *__restrict__ sym, const uint16_t *__restrict__ e0, 
             sm.e0[tid] = c < C ? e0[c] : 0;
             sm.e1[tid] = c < C ? e1[c] : 0;
         }
+        // the symbols of this block's routes for this row: independent loads,
+        // coalesced across the warp (consecutive rows are consecutive t)
+        const int r0 = k0 / M, nr = min(C - 1, k0 + kInjK - 1) / M - r0 + 1;   // routes touched, <= 64
+#pragma unroll 8
+        for (int i = 0; i < kInjK; ++i)
+            if (i < nr) sm.sym[i][tid] = row_ok ? sym[sym_row + (int64_t)(r0 + i) * T] : -1;
         __syncthreads();
         // A: the embedding of this row's 64 channels, eight per 16-byte chunk
-        {
-            int r_prev = -1;
-            int32_t a = -1;
-#pragma unroll 1
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w[4];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    uint16_t v2[2];
+        for (int ch = 0; ch < 8; ++ch) {
+            uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int kk = ch * 8 + h * 2 + e;
-                        const int c = k0 + kk;
-                        uint16_t v = 0;
-                        if (row_ok && c < C) {
-                            const int r = c / M;
-                            if (r != r_prev) {
-                                a = sym[sym_row + (int64_t)r * T];
-                                r_prev = r;
-                            }
-                            if (a >= 0) v = ((a >> (c - r * M)) & 1) ? sm.e1[kk] : sm.e0[kk];
-                        }
-                        v2[e] = v;
+            for (int h = 0; h < 4; ++h) {
+                uint16_t v2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int kk = ch * 8 + h * 2 + e;
+                    const int c = k0 + kk;
+                    uint16_t v = 0;
+                    if (c < C) {
+                        const int r = c / M;
+                        const int32_t a = sm.sym[r - r0][tid];
+                        if (a >= 0) v = ((a >> (c - r * M)) & 1) ? sm.e1[kk] : sm.e0[kk];
                     }
-                    w[h] = (uint32_t)v2[0] | ((uint32_t)v2[1] << 16);
+                    v2[e] = v;
                 }
-                *reinterpret_cast<uint4 *>(sm.a + umma::sw128_offset(tid, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+                w[h] = (uint32_t)v2[0] | ((uint32_t)v2[1] << 16);
             }
+            *reinterpret_cast<uint4 *>(sm.a + umma::sw128_offset(tid, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         // B: rows n0 .. n0+BN-1 of W_out, channels k0 .. k0+63 (zeros outside)
+#pragma unroll 16
         for (int i = tid; i < BN * 8; i += kInjThreads) {
             const int nr = i >> 3, ch = i & 7;
             const int n = n0 + nr, c = k0 + ch * 8;
@@ -152,7 +155,38 @@ inject_kernel(const int32_t *__restrict__ sym, const uint16_t *__restrict__ e0, 
         if (sm.failed) break;
     }
     umma::tc_fence_after();
-    if (!sm.failed) {
+    if (!sm.failed && tma_out) {
+        // epilogue through shared memory: each 64-column box of the tile is
+        // written row by row (thread = row) in the 128-byte swizzle, so the
+        // eight 16-byte chunks of consecutive rows fall in distinct banks, and
+        // leaves in one TMA store (rows and columns past the output are clipped).
+        // The operand tiles are free now: three box buffers (A, then B twice).
+        unsigned char *bufs[3] = {sm.a, sm.b, sm.b + kInjM * 128};
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int c0 = 0, box = 0; c0 < BN && n0 + c0 < D; c0 += 64, ++box) {
+            unsigned char *buf = bufs[box % 3];
+            if (box >= 3) {   // the buffer's previous store must have read it
+                if (tid == 0) umma::tma_store_wait_read();
+                __syncthreads();
+            }
+            uint32_t r[32], w[32];
+            umma::tmem_ld_32cols(trow + (uint32_t)c0, r);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            umma::tmem_ld_32cols(trow + (uint32_t)(c0 + 32), r);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                w[16 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4 *>(buf + umma::sw128_offset(tid, ch * 8)) =
+                    make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+            umma::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) umma::tma_store_2d(&tmOut, n0 + c0, (int)p0, buf);
+        }
+        if (tid == 0) umma::tma_store_wait_read();
+    } else if (!sm.failed) {
         // epilogue: warp w owns rows 32w .. 32w+31 of the tile (TMEM lanes)
         const int64_t row = p0 + warp * 32 + lane;
         const bool vec = (D % 8) == 0;
@@ -216,8 +250,14 @@ cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t
     if (BN < 16) BN = 16;
     const int C = R * M;
     const bool wvec = (C % 8 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0);
+    // the output leaves by TMA stores when its rows are 16-byte aligned and BN
+    // is a whole number of 64-column boxes
+    CUtensorMap tmOut;
+    const bool tma_out = (BN % 64 == 0) && make_tmap_bf16_2d(&tmOut, out, (uint64_t)P, (uint64_t)D, kInjM, 64);
+    if (!tma_out) memset(&tmOut, 0, sizeof tmOut);
     dim3 grid((unsigned)ceil_div64(P, kInjM), (unsigned)ceil_div(D, BN));
-    inject_kernel<<<grid, kInjThreads, smem, st>>>(sym, e0, e1, W, R, M, T, D, BN, P, wvec, out, status);
+    inject_kernel<<<grid, kInjThreads, smem, st>>>(tmOut, tma_out, sym, e0, e1, W, R, M, T, D, BN, P, wvec, out,
+                                                   status);
     return cudaGetLastError();
 }
 

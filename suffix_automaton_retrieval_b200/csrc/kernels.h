@@ -2,9 +2,16 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace rosa {
+
+// Tensor map of a 2-D bf16 tensor [rows][cols] for TMA (tmap.cu): box of
+// box_cols (64: one 128-byte swizzle row) x box_rows; false if the encoder is
+// unavailable or the rows are not 16-byte aligned.
+bool make_tmap_bf16_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                       uint32_t box_cols);
 
 // Streaming multiprocessors of the current device (queried once per device);
 // grids of grid-stride kernels are sized in multiples of it.

@@ -21,7 +21,6 @@
 // Effective columns n < C are query channels, C <= n < 2C key channels; a
 // CTA covers NE of them (a multiple of both 8 and M, at most 128).
 #include <cstdint>
-#include <mutex>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,10 +33,11 @@
 namespace rosa {
 namespace {
 
-constexpr int kLnpM = 128;          // rows per tile
+constexpr int kLnpM = 256;          // rows per CTA: two M = 128 MMAs share each weight block
+constexpr int kLnpMmaM = 128;       // rows of one single-CTA MMA (M = 256 exists only for CTA pairs)
 constexpr int kLnpK = 64;           // K per block (one 128-byte swizzle row)
-constexpr int kLnpThreads = 128;
-constexpr int kLnpStages = 2;
+constexpr int kLnpThreads = 256;    // one row each for the statistics; warps 4-7 take the second half
+constexpr int kLnpStages = 3;
 constexpr uint32_t kLnpWaitPolls = 1u << 24;
 
 int gcd_int(int a, int b) { return b ? gcd_int(b, a % b) : a; }
@@ -49,7 +49,7 @@ int lnp_ne(int M) {
 }
 
 struct LnpSmem {
-    alignas(1024) unsigned char a[kLnpStages][kLnpM * 128];   // H block, K-major SW128
+    alignas(1024) unsigned char a[kLnpStages][kLnpM * 128];   // H block (256 rows), K-major SW128
     alignas(1024) unsigned char b[kLnpStages][256 * 128];     // hi / lo weight rows, K-major SW128
     uint64_t full[kLnpStages], done[kLnpStages];
     uint32_t tmem;
@@ -155,7 +155,7 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
         umma::fence_mbar_init();
         sm.failed = 0;
     }
-    if (warp == 0) umma::tmem_alloc(&sm.tmem, 256);
+    if (warp == 0) umma::tmem_alloc(&sm.tmem, 512);   // accumulators of the two row halves
     umma::tc_fence_before();
     __syncthreads();
     umma::tc_fence_after();
@@ -168,12 +168,11 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
             umma::tma_load_2d(sm.b[s], &tmW, s * kLnpK, tile * N, &sm.full[s]);
         }
     }
-    const uint32_t idesc = umma::make_idesc_bf16_f32(kLnpM, N);
+    const uint32_t idesc = umma::make_idesc_bf16_f32(kLnpMmaM, N);   // each MMA covers one 128-row half
     float s1 = 0.f, s2 = 0.f;   // this thread's row: sum of h and of h^2
     for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb & 1;
-        const uint32_t ph = (uint32_t)((kb >> 1) & 1);
-        if (!umma::mbar_wait_bounded(&sm.full[s], ph, kLnpWaitPolls)) sm.failed = 1;
+        const int s = kb % kLnpStages;
+        if (!umma::mbar_wait_bounded(&sm.full[s], (uint32_t)((kb / kLnpStages) & 1), kLnpWaitPolls)) sm.failed = 1;
         if (!sm.failed) {
             const unsigned char *row = sm.a[s] + tid * 128;
 #pragma unroll
@@ -192,42 +191,51 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
             umma::tc_fence_after();
             const uint32_t abase = umma::smem_u32(sm.a[s]), bbase = umma::smem_u32(sm.b[s]);
 #pragma unroll
-            for (int kk = 0; kk < kLnpK / 16; ++kk)
-                umma::mma_bf16(tmem, umma::make_kmajor_sw128_desc(abase + kk * 32),
-                               umma::make_kmajor_sw128_desc(bbase + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+                for (int kk = 0; kk < kLnpK / 16; ++kk)
+                    umma::mma_bf16(tmem + half * 256, umma::make_kmajor_sw128_desc(abase + half * kLnpMmaM * 128 + kk * 32),
+                                   umma::make_kmajor_sw128_desc(bbase + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             umma::mma_commit(&sm.done[s]);
         }
-        __syncthreads();   // every row's statistics read of stage s is done
+        __syncthreads();   // every row's statistics read of stages up to s is done
         if (sm.failed) break;
-        if (kb + kLnpStages < nkb && tid == 0) {
-            // refill stage s once its MMAs have read it
-            if (!umma::mbar_wait_bounded(&sm.done[s], ph, kLnpWaitPolls)) {
+        // Refill the previous block's stage with block kb - 1 + kLnpStages once its
+        // MMAs have read it: they were issued before this block's, so the tensor
+        // pipe keeps this block's MMAs queued while the issuing thread waits.
+        const int kp = kb - 1;
+        if (kp >= 0 && kp + kLnpStages < nkb && tid == 0) {
+            const int sp = kp % kLnpStages;
+            if (!umma::mbar_wait_bounded(&sm.done[sp], (uint32_t)((kp / kLnpStages) & 1), kLnpWaitPolls)) {
                 sm.failed = 1;
             } else {
-                umma::mbar_arrive_expect_tx(&sm.full[s], a_bytes + b_bytes);
-                umma::tma_load_2d(sm.a[s], &tmH, (kb + kLnpStages) * kLnpK, (int)p0, &sm.full[s]);
-                umma::tma_load_2d(sm.b[s], &tmW, (kb + kLnpStages) * kLnpK, tile * N, &sm.full[s]);
+                umma::mbar_arrive_expect_tx(&sm.full[sp], a_bytes + b_bytes);
+                umma::tma_load_2d(sm.a[sp], &tmH, (kp + kLnpStages) * kLnpK, (int)p0, &sm.full[sp]);
+                umma::tma_load_2d(sm.b[sp], &tmW, (kp + kLnpStages) * kLnpK, tile * N, &sm.full[sp]);
             }
         }
     }
     // the last commit covers every MMA of the tile
     if (!sm.failed && nkb > 0) {
         const int kl = nkb - 1;
-        if (!umma::mbar_wait_bounded(&sm.done[kl & 1], (uint32_t)((kl >> 1) & 1), kLnpWaitPolls)) sm.failed = 1;
+        if (!umma::mbar_wait_bounded(&sm.done[kl % kLnpStages], (uint32_t)((kl / kLnpStages) & 1), kLnpWaitPolls))
+            sm.failed = 1;
     }
     __syncthreads();
     umma::tc_fence_after();
     if (!sm.failed) {
-        // epilogue: thread = row (TMEM lane 32*warp + lane)
+        // epilogue: thread = row; warps 0-3 read the first half's accumulator
+        // (TMEM columns 0..255), warps 4-7 the second half's (256..511)
         const int64_t p = p0 + tid;
+        const uint32_t tacc = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * 256);
         const float mu = s1 / (float)D;
         const float var = fmaxf(s2 / (float)D - mu * mu, 0.f);
         const float rstd = rsqrtf(var + eps);
         uint32_t bits[4] = {0, 0, 0, 0};   // threshold bits of the NE effective columns
         for (int c0 = 0; c0 < NE; c0 += 32) {
             uint32_t h[32], l[32];
-            umma::tmem_ld_32cols(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, h);
-            umma::tmem_ld_32cols(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(NE + c0), l);
+            umma::tmem_ld_32cols(tacc + (uint32_t)c0, h);
+            umma::tmem_ld_32cols(tacc + (uint32_t)(NE + c0), l);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int cn = c0 + j;
@@ -257,39 +265,7 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
     }
     umma::tc_fence_before();
     __syncthreads();
-    if (warp == 0) umma::tmem_dealloc(tmem, 256);
-}
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver's tensor-map encoder, looked up once through the runtime.
-EncodeTiledFn encode_fn() {
-    static std::once_flag once;
-    static EncodeTiledFn fn = nullptr;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2-D bf16 tensor [rows][cols] (cols contiguous), box of 64 columns x box_rows
-// rows, 128-byte swizzle, zero fill outside.
-bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (warp == 0) umma::tmem_dealloc(tmem, 512);
 }
 
 size_t lnp_smem_bytes() { return sizeof(LnpSmem) + 1024; }
@@ -307,8 +283,8 @@ cudaError_t launch_ln_project(const uint16_t *H, const float *gamma, const float
     if (P == 0) return cudaSuccess;
     const int NE = lnp_ne(M), NT = ceil_div(2 * C, NE);
     CUtensorMap tmH, tmW;
-    if (!make_tmap(&tmH, H, (uint64_t)P, (uint64_t)D, kLnpM) ||
-        !make_tmap(&tmW, L.wp, (uint64_t)NT * 2 * NE, (uint64_t)D, (uint32_t)(2 * NE)))
+    if (!make_tmap_bf16_2d(&tmH, H, (uint64_t)P, (uint64_t)D, kLnpM, 64) ||
+        !make_tmap_bf16_2d(&tmW, L.wp, (uint64_t)NT * 2 * NE, (uint64_t)D, (uint32_t)(2 * NE), 64))
         return cudaErrorInvalidValue;
     static bool attr_done[64] = {};
     int dev = 0;

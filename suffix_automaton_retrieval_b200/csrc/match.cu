@@ -90,7 +90,7 @@ Geometry make_geometry(int S, int T, int K, int g, bool same, int mcf = 0) {
     // array, which the stable sort keeps among equal symbols.
     G.idbits = bits_for(G.n > 0 ? G.n - 1 : 0);
     if (G.idbits < 1) G.idbits = 1;
-    const int budget = min(40, 64 - G.idbits);
+    const int budget = min(G.bps <= 4 ? 32 : 40, 64 - G.idbits);   // small alphabets: fewer passes pay
     G.D0 = max(1, budget / G.bps);
     G.keybits = G.idbits + G.D0 * G.bps;
     G.ntps = ceil_div(G.n, kRadixTile);

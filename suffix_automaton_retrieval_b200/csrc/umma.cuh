@@ -163,3 +163,28 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, 
 
 }  // namespace umma
 }  // namespace rosa
+
+namespace rosa {
+namespace umma {
+
+// One thread: 2-D tiled store of the box at (x, y) from shared memory (the
+// tensor map clips what lies outside the tensor), as one bulk group.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, const void *src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// One thread: wait until the shared memory of every committed bulk store has
+// been read (it may then be overwritten).
+__device__ __forceinline__ void tma_store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// One thread: wait until every committed bulk store has completed.
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+}  // namespace umma
+}  // namespace rosa
