@@ -6,13 +6,17 @@
 // m = I[tau >= 0], the embedding y_c = m((1 - b^) e0_c + b^ e1_c), and the
 // injection inj = W_out y.
 //
-// One CTA computes a 128-row x BN-column tile of inj (rows are positions
-// b*T + t).  For every 64-channel block of K it builds the A tile (y, bf16)
-// directly in shared memory from the recalled symbols, so the embedding
-// never touches global memory, stages the matching W_out block, and one
-// thread issues four tcgen05 MMAs (M = 128, N = BN, K = 16 each) into an
-// fp32 accumulator in tensor memory.  The epilogue reads the accumulator
-// back with tcgen05.ld, rounds to bf16 and stores the rows.
+// Main kernel (C <= 512 channels): persistent CTAs, each owning 128-row
+// tiles of inj (rows are positions b*T + t).  For a row tile the CTA builds
+// the whole A operand (y, bf16, K-major with the 128-byte swizzle) in shared
+// memory from the recalled symbols once, so the embedding never touches
+// global memory, then walks the output in 128-column tiles: W_out blocks
+// arrive by TMA through a three-stage ring, one thread issues the tcgen05
+// MMAs into one of two fp32 accumulators in tensor memory, and while the
+// tensor cores work on column tile j the eight warps drain tile j-1 (two
+// warps per 32 accumulator lanes, one 64-column box each), round to bf16,
+// stage the box in the swizzled layout and send it out with a TMA store.
+// Wider embeddings (C > 512) use a one-tile-per-CTA kernel.
 #include <cstdint>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -47,8 +51,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// One CTA per 128-row x BN-column tile (any C): the A tile is built per
+// 64-channel K block, W_out staged by 16-byte loads, four MMAs per block.
 __global__ void __launch_bounds__(kInjThreads, 1)
-inject_kernel(const __grid_constant__ CUtensorMap tmOut, bool tma_out, const int32_t *__restrict__ sym,
+inject_tile_kernel(const __grid_constant__ CUtensorMap tmOut, bool tma_out, const int32_t *__restrict__ sym,
               const uint16_t *__restrict__ e0, const uint16_t *__restrict__ e1, const uint16_t *__restrict__ W, int R,
               int M, int T, int D, int BN, int64_t P, bool wvec, uint16_t *__restrict__ out,
               uint32_t *__restrict__ status) {
@@ -221,6 +227,303 @@ inject_kernel(const __grid_constant__ CUtensorMap tmOut, bool tma_out, const int
     if (warp == 0) umma::tmem_dealloc(tmem, ncols);
 }
 
+
+// ---- persistent kernel (C <= 512) -------------------------------------------
+
+constexpr int kIpN = 128;                       // columns per accumulator / column tile
+constexpr int kIpThreads = 256;                 // warps w and w + 4 share TMEM lanes 32*(w % 4)
+constexpr int kIpStages = 3;                    // W_out blocks in flight
+constexpr int kIpMaxKb = 8;                     // K blocks of a resident A tile (C <= 512)
+constexpr uint32_t kIpTile = kInjM * 128;       // 16 KB: 128 rows x 64 bf16, K-major SW128
+
+// Shared-memory carve of the persistent kernel, from a 1024-aligned base.
+struct IpCarve {
+    uint32_t a, w, ob, e0, e1, bars, slot, total;
+};
+
+__host__ __device__ inline IpCarve ip_carve(int nkb) {
+    IpCarve c{};
+    c.a = 0;
+    c.w = c.a + (uint32_t)nkb * kIpTile;
+    c.ob = c.w + kIpStages * kIpTile;                // two output boxes (one per warp group)
+    c.e0 = c.ob + 2 * kIpTile;
+    c.e1 = c.e0 + (uint32_t)nkb * 64 * 2;            // e0, e1 padded with zeros to nkb * 64 channels
+    c.bars = c.e1 + (uint32_t)nkb * 64 * 2;          // multiple of 128: 8-byte aligned
+    c.slot = c.bars + 8 * (2 * kIpStages + 2);
+    c.total = c.slot + 16;
+    return c;
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Two bf16 channels of a 32-bit word: e1 where the bit is set, else e0; zero where the mask is clear.
+__device__ __forceinline__ uint32_t select_pair(uint32_t z0, uint32_t z1, uint32_t bits, uint32_t mask, int k) {
+    const uint32_t bs = (((bits >> k) & 1u) ? 0x0000FFFFu : 0u) | (((bits >> (k + 1)) & 1u) ? 0xFFFF0000u : 0u);
+    const uint32_t ms = (((mask >> k) & 1u) ? 0x0000FFFFu : 0u) | (((mask >> (k + 1)) & 1u) ? 0xFFFF0000u : 0u);
+    return ((z1 & bs) | (z0 & ~bs)) & ms;
+}
+
+__global__ void __launch_bounds__(kIpThreads, 2)
+inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmOut, bool tma_w,
+                         bool tma_out, const int32_t *__restrict__ sym, const uint16_t *__restrict__ e0,
+                         const uint16_t *__restrict__ e1, const uint16_t *__restrict__ W, int R, int M, int T, int D,
+                         int64_t P, int nkb, uint16_t *__restrict__ out, uint32_t *__restrict__ status) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~(uintptr_t)1023);
+    const IpCarve cv = ip_carve(nkb);
+    unsigned char *sa = base + cv.a, *sw = base + cv.w, *sob = base + cv.ob;
+    uint16_t *se0 = reinterpret_cast<uint16_t *>(base + cv.e0), *se1 = reinterpret_cast<uint16_t *>(base + cv.e1);
+    uint64_t *wfull = reinterpret_cast<uint64_t *>(base + cv.bars);
+    uint64_t *wempty = wfull + kIpStages, *accfull = wfull + 2 * kIpStages;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(base + cv.slot);
+    volatile int *failed = reinterpret_cast<volatile int *>(tslot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int C = R * M;
+    const int nrt = (int)ceil_div64(P, kInjM), NJ = ceil_div(D, kIpN);
+    const int my_rt = (nrt - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int64_t total_wb = (int64_t)my_rt * NJ * nkb;   // W_out blocks this CTA consumes
+
+    if (tid == 0) {
+        for (int s = 0; s < kIpStages; ++s) {
+            umma::mbar_init(&wfull[s], 1);
+            umma::mbar_init(&wempty[s], 1);
+        }
+        umma::mbar_init(&accfull[0], 1);
+        umma::mbar_init(&accfull[1], 1);
+        umma::fence_mbar_init();
+        *failed = 0;
+    }
+    for (int c = tid; c < nkb * 64; c += kIpThreads) {
+        se0[c] = c < C ? e0[c] : 0;
+        se1[c] = c < C ? e1[c] : 0;
+    }
+    if (warp == 0) umma::tmem_alloc(tslot, 2 * kIpN);
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t idesc = umma::make_idesc_bf16_f32(kInjM, kIpN);
+
+    // W_out block x of this CTA's sequence: column tile (x / nkb) % NJ, K block x % nkb
+    int64_t w_issued = 0;
+    auto issue_w = [&](int64_t x) {
+        const int64_t u = x % ((int64_t)NJ * nkb);
+        const int jj = (int)(u / nkb), kk = (int)(u % nkb);
+        const int s = (int)(x % kIpStages);
+        umma::mbar_arrive_expect_tx(&wfull[s], kIpTile);
+        umma::tma_load_2d(sw + s * kIpTile, &tmW, kk * 64, jj * kIpN, &wfull[s]);
+    };
+    if (tma_w && tid == 0)
+        for (; w_issued < kIpStages && w_issued < total_wb; ++w_issued) issue_w(w_issued);
+
+    int64_t wb = 0;            // W_out blocks consumed
+    int q = 0;                 // column tiles issued
+    int pend_i = -1, pend_j = 0, pend_q = 0;
+    const int g = warp >> 2, lbase = (warp & 3) * 32;
+
+    // Epilogue of column tile qq (row tile ii, column tile jj): all threads.
+    auto epilogue = [&](int qq, int ii, int jj) {
+        const int col0 = jj * kIpN + g * 64;
+        const bool live = col0 < D;
+        bool ok = umma::mbar_wait_bounded(&accfull[qq & 1], (uint32_t)((qq >> 1) & 1), kWaitPolls);
+        ok = __all_sync(ROSA_FULL_MASK, ok);
+        if (!ok) *failed = 1;
+        umma::tc_fence_after();
+        const int row = lbase + lane;
+        const uint32_t ta = tmem + ((uint32_t)lbase << 16) + (uint32_t)((qq & 1) * kIpN + g * 64);
+        if (tma_out) {
+            unsigned char *buf = sob + g * kIpTile;
+            if ((tid & 127) == 0) umma::tma_store_wait_read();   // the box's previous store has read it
+            named_bar(1 + g, 128);
+            if (ok && live) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {   // 32 columns = four 16-byte chunks at a time
+                    uint32_t r[32];
+                    umma::tmem_ld_32cols(ta + 32 * h, r);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(r[8 * c4 + 0]), __uint_as_float(r[8 * c4 + 1]));
+                        v.y = pack_bf16x2(__uint_as_float(r[8 * c4 + 2]), __uint_as_float(r[8 * c4 + 3]));
+                        v.z = pack_bf16x2(__uint_as_float(r[8 * c4 + 4]), __uint_as_float(r[8 * c4 + 5]));
+                        v.w = pack_bf16x2(__uint_as_float(r[8 * c4 + 6]), __uint_as_float(r[8 * c4 + 7]));
+                        *reinterpret_cast<uint4 *>(buf + umma::sw128_offset(row, 32 * h + 8 * c4)) = v;
+                    }
+                }
+            }
+            umma::fence_async_smem();
+            named_bar(1 + g, 128);
+            if ((tid & 127) == 0 && ok && live) umma::tma_store_2d(&tmOut, col0, ii * kInjM, buf);
+        } else if (ok && live) {
+            const int64_t p = (int64_t)ii * kInjM + row;
+            uint16_t *dst = out + p * D + col0;
+            const int left = D - col0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t r[32];
+                umma::tmem_ld_32cols(ta + 32 * h, r);
+                if (p < P) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(r[j]));
+                        if (32 * h + j < left) dst[32 * h + j] = *reinterpret_cast<const uint16_t *>(&b);
+                    }
+                }
+            }
+        }
+    };
+
+    for (int i = blockIdx.x; i < nrt; i += gridDim.x) {
+        // the previous row tile's last column tile: its MMAs still read A
+        if (pend_i >= 0) {
+            epilogue(pend_q, pend_i, pend_j);
+            pend_i = -1;
+        }
+        // A: row = tid % 128, channels [64 kb + 32 half, +32) of every K block
+        {
+            const int row = tid & 127, half = tid >> 7;
+            const int64_t p = (int64_t)i * kInjM + row;
+            const bool valid = p < P;
+            const int32_t *srow = sym;
+            if (valid) {
+                const int64_t b = p / T;
+                srow = sym + b * (int64_t)R * T + (p - b * T);
+            }
+            const uint32_t lowm = (1u << M) - 1u;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int cbase = kb * 64 + half * 32;
+                uint32_t vb = 0, mm = 0;
+                if (cbase < C) {
+                    const int r0 = cbase / M, r1 = min(C - 1, cbase + 31) / M;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int r = r0 + u;
+                        if (r <= r1) {
+                            const int32_t av = valid ? __ldg(srow + (int64_t)r * T) : -1;
+                            const uint32_t bits = av >= 0 ? ((uint32_t)av & lowm) : 0u;
+                            const uint32_t mk = av >= 0 ? lowm : 0u;
+                            const int pos = r * M - cbase;
+                            if (pos >= 0) {
+                                vb |= bits << pos;
+                                mm |= mk << pos;
+                            } else {
+                                vb |= bits >> -pos;
+                                mm |= mk >> -pos;
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int k0 = ch * 8;
+                    const uint4 z0 = *reinterpret_cast<const uint4 *>(se0 + cbase + k0);
+                    const uint4 z1 = *reinterpret_cast<const uint4 *>(se1 + cbase + k0);
+                    uint4 v;
+                    v.x = select_pair(z0.x, z1.x, vb, mm, k0 + 0);
+                    v.y = select_pair(z0.y, z1.y, vb, mm, k0 + 2);
+                    v.z = select_pair(z0.z, z1.z, vb, mm, k0 + 4);
+                    v.w = select_pair(z0.w, z1.w, vb, mm, k0 + 6);
+                    *reinterpret_cast<uint4 *>(sa + kb * kIpTile + umma::sw128_offset(row, half * 32 + k0)) = v;
+                }
+            }
+            umma::fence_async_smem();
+        }
+        for (int j = 0; j < NJ; ++j) {
+            umma::tc_fence_before();
+            __syncthreads();   // A built; the previous epilogue's TMEM reads are done
+            if (*failed) break;
+            const uint32_t dacc = tmem + (uint32_t)((q & 1) * kIpN);
+            if (tma_w) {
+                if (tid == 0) {
+                    umma::tc_fence_after();
+                    for (int kb = 0; kb < nkb; ++kb, ++wb) {
+                        const int s = (int)(wb % kIpStages);
+                        if (!umma::mbar_wait_bounded(&wfull[s], (uint32_t)((wb / kIpStages) & 1), kWaitPolls)) {
+                            *failed = 1;
+                            break;
+                        }
+                        const uint32_t ab = umma::smem_u32(sa + kb * kIpTile), bb = umma::smem_u32(sw + s * kIpTile);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma::mma_bf16(dacc, umma::make_kmajor_sw128_desc(ab + kk * 32),
+                                           umma::make_kmajor_sw128_desc(bb + kk * 32), idesc,
+                                           (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma::mma_commit(&wempty[s]);
+                        // refill the previous block's stage once its MMAs have read it
+                        if (wb >= 1 && wb - 1 + kIpStages < total_wb && w_issued == wb - 1 + kIpStages) {
+                            const int sp = (int)((wb - 1) % kIpStages);
+                            if (!umma::mbar_wait_bounded(&wempty[sp], (uint32_t)(((wb - 1) / kIpStages) & 1),
+                                                         kWaitPolls)) {
+                                *failed = 1;
+                                break;
+                            }
+                            issue_w(w_issued++);
+                        }
+                    }
+                    umma::mma_commit(&accfull[q & 1]);
+                }
+            } else {
+                // W_out rows are not 16-byte aligned for TMA: every thread stages a share
+                for (int kb = 0; kb < nkb; ++kb, ++wb) {
+                    const int s = (int)(wb % kIpStages);
+                    if (wb >= kIpStages &&
+                        !umma::mbar_wait_bounded(&wempty[s], (uint32_t)(((wb - kIpStages) / kIpStages) & 1),
+                                                 kWaitPolls))
+                        *failed = 1;
+                    for (int e = tid; e < kIpN * 8; e += kIpThreads) {
+                        const int nr = e >> 3, ch = e & 7;
+                        const int n = j * kIpN + nr, c = kb * 64 + ch * 8;
+                        uint16_t t8[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) t8[x] = (n < D && c + x < C) ? W[(int64_t)n * C + c + x] : 0;
+                        *reinterpret_cast<uint4 *>(sw + s * kIpTile + umma::sw128_offset(nr, ch * 8)) =
+                            make_uint4(t8[0] | ((uint32_t)t8[1] << 16), t8[2] | ((uint32_t)t8[3] << 16),
+                                       t8[4] | ((uint32_t)t8[5] << 16), t8[6] | ((uint32_t)t8[7] << 16));
+                    }
+                    umma::fence_async_smem();
+                    __syncthreads();
+                    if (tid == 0 && !*failed) {
+                        umma::tc_fence_after();
+                        const uint32_t ab = umma::smem_u32(sa + kb * kIpTile), bb = umma::smem_u32(sw + s * kIpTile);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma::mma_bf16(dacc, umma::make_kmajor_sw128_desc(ab + kk * 32),
+                                           umma::make_kmajor_sw128_desc(bb + kk * 32), idesc,
+                                           (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma::mma_commit(&wempty[s]);
+                    }
+                }
+                if (tid == 0 && !*failed) umma::mma_commit(&accfull[q & 1]);
+            }
+            if (pend_i >= 0) epilogue(pend_q, pend_i, pend_j);
+            pend_i = i;
+            pend_j = j;
+            pend_q = q;
+            ++q;
+        }
+        __syncthreads();
+        if (*failed) break;
+    }
+    __syncthreads();
+    if (pend_i >= 0 && !*failed) epilogue(pend_q, pend_i, pend_j);
+    // nothing may be in flight at exit: loads not consumed, MMAs, stores
+    if (tid == 0 && tma_w)
+        for (int64_t x = wb; x < w_issued; ++x)
+            umma::mbar_wait_bounded(&wfull[x % kIpStages], (uint32_t)((x / kIpStages) & 1), kWaitPolls);
+    if (tid == 0 && *failed && q > 0) umma::mbar_wait_bounded(&accfull[(q - 1) & 1], (uint32_t)(((q - 1) >> 1) & 1), kWaitPolls);
+    if ((tid & 127) == 0 && tma_out) umma::tma_store_wait_all();
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, 2 * kIpN);
+    if (tid == 0 && *failed && status) atomicOr(status, ROSA_DEV_TIMEOUT);
+}
+
+size_t ip_smem_bytes(int nkb) { return ip_carve(nkb).total + 1024; }
+
 }  // namespace
 
 // Dynamic shared memory of one CTA: the tiles plus alignment slack, and at
@@ -235,20 +538,47 @@ cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t
                           int M, int T, int D, uint16_t *out, uint32_t *status, cudaStream_t st) {
     const int64_t P = (int64_t)B * T;
     if (P == 0 || D == 0) return cudaSuccess;
-    static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const int C = R * M;
+    const int nkb = ceil_div(C, kInjK);
+    if (nkb <= kIpMaxKb) {
+        static bool ip_attr[64] = {};
+        if (dev < 0 || dev >= 64 || !ip_attr[dev]) {
+            e = cudaFuncSetAttribute(inject_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)ip_smem_bytes(kIpMaxKb));
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) ip_attr[dev] = true;
+        }
+        const int smem = (int)ip_smem_bytes(nkb);
+        CUtensorMap tmW, tmOut;
+        const bool tma_w = C >= kInjK && make_tmap_bf16_2d(&tmW, W, (uint64_t)D, (uint64_t)C, kInjM, 64);
+        const bool tma_out = D >= 64 && make_tmap_bf16_2d(&tmOut, out, (uint64_t)P, (uint64_t)D, kInjM, 64);
+        if (!tma_w) memset(&tmW, 0, sizeof tmW);
+        if (!tma_out) memset(&tmOut, 0, sizeof tmOut);
+        // at most two CTAs per SM: each holds 256 of the SM's 512 tensor-memory columns
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, inject_persistent_kernel, kIpThreads, smem);
+        if (e != cudaSuccess) return e;
+        per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);
+        const int64_t nrt = ceil_div64(P, kInjM);
+        const int64_t slots = (int64_t)per_sm * device_sm_count();
+        const unsigned grid = (unsigned)(nrt < slots ? nrt : slots);
+        inject_persistent_kernel<<<grid, kIpThreads, smem, st>>>(tmW, tmOut, tma_w, tma_out, sym, e0, e1, W, R, M, T,
+                                                                  D, P, nkb, out, status);
+        return cudaGetLastError();
+    }
+    static bool attr_done[64] = {};
     const int smem = (int)inject_smem_bytes();
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(inject_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(inject_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     // N tile: all of D when it fits one MMA, else 256 (a multiple of 16 in [16, 256])
     int BN = D >= kInjMaxN ? kInjMaxN : ((D + 15) / 16) * 16;
     if (BN < 16) BN = 16;
-    const int C = R * M;
     const bool wvec = (C % 8 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0);
     // the output leaves by TMA stores when its rows are 16-byte aligned and BN
     // is a whole number of 64-column boxes
@@ -256,8 +586,8 @@ cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t
     const bool tma_out = (BN % 64 == 0) && make_tmap_bf16_2d(&tmOut, out, (uint64_t)P, (uint64_t)D, kInjM, 64);
     if (!tma_out) memset(&tmOut, 0, sizeof tmOut);
     dim3 grid((unsigned)ceil_div64(P, kInjM), (unsigned)ceil_div(D, BN));
-    inject_kernel<<<grid, kInjThreads, smem, st>>>(tmOut, tma_out, sym, e0, e1, W, R, M, T, D, BN, P, wvec, out,
-                                                   status);
+    inject_tile_kernel<<<grid, kInjThreads, smem, st>>>(tmOut, tma_out, sym, e0, e1, W, R, M, T, D, BN, P, wvec, out,
+                                                        status);
     return cudaGetLastError();
 }
 

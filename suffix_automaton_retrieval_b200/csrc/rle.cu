@@ -108,8 +108,11 @@ __device__ __forceinline__ unsigned tile_flags(const uint8_t *__restrict__ x, in
     return f;
 }
 
-// Slot s*T + j of a padded run stream: a symbol below K that no real run
-// depends on (hash of the slot).
+// Slot j of stream s's padded key (which = 0) or query (which = 1) run
+// stream: a symbol below K that no real run depends on, hashed from the slot
+// and the side.  The two sides draw independent symbols: identical padded
+// tails would share histories as long as the padding and make the suffix
+// sorting and the LCP work grow with it.
 __device__ __forceinline__ uint8_t pad_symbol(int64_t slot, int K) {
     uint32_t h = (uint32_t)slot * 0x9E3779B1u;
     h ^= h >> 15;
@@ -205,7 +208,7 @@ rle_write_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, i
     const int n = nrun[s * 2 + which];
     for (int j = p0 + threadIdx.x; j < min(p0 + kRleTile, T); j += kRleThreads) {
         if (j >= n) {
-            rs[j] = pad_symbol((int64_t)s * T + j, K);
+            rs[j] = pad_symbol((((int64_t)s * T + j) << 1) | which, K);
             rt[j] = T;
         }
     }

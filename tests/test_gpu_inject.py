@@ -68,7 +68,7 @@ def _check(got, sym, e0, e1, W, B, R, M, tag):
 
 @pytest.mark.parametrize("B,R,M,T,D", [(1, 64, 1, 300, 2048), (2, 16, 2, 200, 512), (1, 5, 3, 77, 40),
                                        (1, 256, 2, 130, 512), (1, 4, 8, 129, 300), (3, 7, 1, 33, 16),
-                                       (1, 96, 2, 257, 264)])
+                                       (1, 96, 2, 257, 264), (1, 160, 4, 100, 136), (2, 32, 2, 40000, 200)])
 def test_inject_parity(rosa, B, R, M, T, D):
     sym, e0, e1, W = _inputs(B, R, M, T, D, seed=B * 1000 + R * 10 + M + T + D)
     got = rosa.inject(sym.to(DEV), e0.to(DEV), e1.to(DEV), W.to(DEV), B, R, M)
@@ -106,3 +106,18 @@ def test_inject_full_qwen_proj_64_shape(rosa):
     got = rosa.inject(sym.to(DEV), e0.to(DEV), e1.to(DEV), W.to(DEV), B, R, M)
     torch.cuda.synchronize()
     _check(got, sym, e0, e1, W, B, R, M, "qwen-proj-64 shape")
+
+
+def test_inject_full_markov_4_train_shape(rosa):
+    """markov-4-train-shaped: 8 x 8192 positions, 256 routes of 2 bits (512
+    channels, eight K blocks), width 512; several row tiles per CTA.  Sampled
+    positions of every batch element are compared with the oracle."""
+    B, R, M, T, D = 8, 256, 2, 8192, 512
+    sym, e0, e1, W = _inputs(B, R, M, T, D, seed=256)
+    got = rosa.inject(sym.to(DEV), e0.to(DEV), e1.to(DEV), W.to(DEV), B, R, M)
+    torch.cuda.synchronize()
+    sel = np.unique(np.concatenate([np.arange(0, 300), np.arange(T - 300, T),
+                                    np.random.default_rng(5).choice(T, 400, replace=False)]))
+    sub = sym.reshape(B, R, T)[:, :, sel].reshape(B * R, len(sel)).contiguous()
+    got_sub = got.reshape(B, T, D)[:, sel, :].contiguous()
+    _check(got_sub, sub, e0, e1, W, B, R, M, "markov-4-train shape (sampled)")
