@@ -34,7 +34,7 @@ constexpr int kInjM = 128;          // rows per tile = UMMA M
 constexpr int kInjK = 64;           // channels per K block = one 128-byte swizzle row
 constexpr int kInjThreads = 128;    // four warps: one per 32 TMEM lanes in the epilogue
 constexpr int kInjMaxN = 256;       // UMMA N limit for M = 128
-constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr uint32_t kWaitPolls = umma::kWaitPolls;
 
 struct InjSmem {
     alignas(1024) unsigned char a[kInjM * 128];        // y block, K-major SW128
@@ -229,9 +229,20 @@ inject_tile_kernel(const __grid_constant__ CUtensorMap tmOut, bool tma_out, cons
 
 
 // ---- persistent kernel (C <= 512) -------------------------------------------
+//
+// Warp roles (320 threads):
+//   warps 0-7  build the A tile of each row tile, then drain the accumulators
+//              of its column tiles (warps w and w + 4 share TMEM lanes
+//              32*(w % 4) and take one 64-column box each);
+//   warp 8     lane 0 issues the MMAs;
+//   warp 9     produces the W_out blocks (lane 0 by TMA, or the whole warp by
+//              plain loads when W_out rows are not 16-byte aligned).
+// The roles meet only on mbarriers: W_out stage full / empty, accumulator
+// full / empty (two accumulators of 128 columns), A full / empty.
 
 constexpr int kIpN = 128;                       // columns per accumulator / column tile
-constexpr int kIpThreads = 256;                 // warps w and w + 4 share TMEM lanes 32*(w % 4)
+constexpr int kIpWorkers = 256;                 // warps 0-7
+constexpr int kIpThreads = kIpWorkers + 64;     // + MMA warp + W_out producer warp
 constexpr int kIpStages = 3;                    // W_out blocks in flight
 constexpr int kIpMaxKb = 8;                     // K blocks of a resident A tile (C <= 512)
 constexpr uint32_t kIpTile = kInjM * 128;       // 16 KB: 128 rows x 64 bf16, K-major SW128
@@ -241,21 +252,38 @@ struct IpCarve {
     uint32_t a, w, ob, e0, e1, bars, slot, total;
 };
 
+// barriers: wfull[S], wempty[S], accfull[2], accempty[2], afull, aempty, drain
+constexpr int kIpBars = 2 * kIpStages + 7;
+
 __host__ __device__ inline IpCarve ip_carve(int nkb) {
     IpCarve c{};
     c.a = 0;
     c.w = c.a + (uint32_t)nkb * kIpTile;
-    c.ob = c.w + kIpStages * kIpTile;                // two output boxes (one per warp group)
+    c.ob = c.w + kIpStages * kIpTile;                // two output boxes (one per worker group)
     c.e0 = c.ob + 2 * kIpTile;
     c.e1 = c.e0 + (uint32_t)nkb * 64 * 2;            // e0, e1 padded with zeros to nkb * 64 channels
     c.bars = c.e1 + (uint32_t)nkb * 64 * 2;          // multiple of 128: 8-byte aligned
-    c.slot = c.bars + 8 * (2 * kIpStages + 2);
+    c.slot = c.bars + 8 * kIpBars;
     c.total = c.slot + 16;
     return c;
 }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(umma::smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that also gives up once another role has flagged a failure.
+__device__ __forceinline__ bool ip_wait(uint64_t *bar, uint32_t parity, volatile int *failed) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (umma::mbar_try_wait(bar, parity)) return true;
+        if (*failed) return false;
+    }
+    *failed = 1;
+    return false;
 }
 
 // Two bf16 channels of a 32-bit word: e1 where the bit is set, else e0; zero where the mask is clear.
@@ -277,7 +305,8 @@ inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_c
     unsigned char *sa = base + cv.a, *sw = base + cv.w, *sob = base + cv.ob;
     uint16_t *se0 = reinterpret_cast<uint16_t *>(base + cv.e0), *se1 = reinterpret_cast<uint16_t *>(base + cv.e1);
     uint64_t *wfull = reinterpret_cast<uint64_t *>(base + cv.bars);
-    uint64_t *wempty = wfull + kIpStages, *accfull = wfull + 2 * kIpStages;
+    uint64_t *wempty = wfull + kIpStages, *accfull = wfull + 2 * kIpStages, *accempty = accfull + 2;
+    uint64_t *afull = accempty + 2, *aempty = afull + 1, *drain = aempty + 1;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(base + cv.slot);
     volatile int *failed = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -285,7 +314,12 @@ inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_c
     const int C = R * M;
     const int nrt = (int)ceil_div64(P, kInjM), NJ = ceil_div(D, kIpN);
     const int my_rt = (nrt - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int64_t total_wb = (int64_t)my_rt * NJ * nkb;   // W_out blocks this CTA consumes
+    const int64_t nq = (int64_t)my_rt * NJ;         // column tiles of this CTA
+    // CTAs start their column walk at different tiles, so that concurrent
+    // stores (and W_out reads) spread over the output's rows instead of all
+    // hitting the same offsets
+    const int crot = (int)(blockIdx.x % (unsigned)NJ);
+    const int64_t total_wb = nq * nkb;              // W_out blocks
 
     if (tid == 0) {
         for (int s = 0; s < kIpStages; ++s) {
@@ -294,6 +328,11 @@ inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_c
         }
         umma::mbar_init(&accfull[0], 1);
         umma::mbar_init(&accfull[1], 1);
+        umma::mbar_init(&accempty[0], kIpWorkers);
+        umma::mbar_init(&accempty[1], kIpWorkers);
+        umma::mbar_init(afull, kIpWorkers);
+        umma::mbar_init(aempty, 1);
+        umma::mbar_init(drain, 1);
         umma::fence_mbar_init();
         *failed = 0;
     }
@@ -306,104 +345,111 @@ inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_c
     __syncthreads();
     umma::tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t idesc = umma::make_idesc_bf16_f32(kInjM, kIpN);
 
-    // W_out block x of this CTA's sequence: column tile (x / nkb) % NJ, K block x % nkb
-    int64_t w_issued = 0;
-    auto issue_w = [&](int64_t x) {
-        const int64_t u = x % ((int64_t)NJ * nkb);
-        const int jj = (int)(u / nkb), kk = (int)(u % nkb);
-        const int s = (int)(x % kIpStages);
-        umma::mbar_arrive_expect_tx(&wfull[s], kIpTile);
-        umma::tma_load_2d(sw + s * kIpTile, &tmW, kk * 64, jj * kIpN, &wfull[s]);
-    };
-    if (tma_w && tid == 0)
-        for (; w_issued < kIpStages && w_issued < total_wb; ++w_issued) issue_w(w_issued);
-
-    int64_t wb = 0;            // W_out blocks consumed
-    int q = 0;                 // column tiles issued
-    int pend_i = -1, pend_j = 0, pend_q = 0;
-    const int g = warp >> 2, lbase = (warp & 3) * 32;
-
-    // Epilogue of column tile qq (row tile ii, column tile jj): all threads.
-    auto epilogue = [&](int qq, int ii, int jj) {
-        const int col0 = jj * kIpN + g * 64;
-        const bool live = col0 < D;
-        bool ok = umma::mbar_wait_bounded(&accfull[qq & 1], (uint32_t)((qq >> 1) & 1), kWaitPolls);
-        ok = __all_sync(ROSA_FULL_MASK, ok);
-        if (!ok) *failed = 1;
-        umma::tc_fence_after();
-        const int row = lbase + lane;
-        const uint32_t ta = tmem + ((uint32_t)lbase << 16) + (uint32_t)((qq & 1) * kIpN + g * 64);
-        if (tma_out) {
-            unsigned char *buf = sob + g * kIpTile;
-            if ((tid & 127) == 0) umma::tma_store_wait_read();   // the box's previous store has read it
-            named_bar(1 + g, 128);
-            if (ok && live) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {   // 32 columns = four 16-byte chunks at a time
-                    uint32_t r[32];
-                    umma::tmem_ld_32cols(ta + 32 * h, r);
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(r[8 * c4 + 0]), __uint_as_float(r[8 * c4 + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(r[8 * c4 + 2]), __uint_as_float(r[8 * c4 + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(r[8 * c4 + 4]), __uint_as_float(r[8 * c4 + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(r[8 * c4 + 6]), __uint_as_float(r[8 * c4 + 7]));
-                        *reinterpret_cast<uint4 *>(buf + umma::sw128_offset(row, 32 * h + 8 * c4)) = v;
-                    }
+    if (warp == 9) {
+        // ---- W_out producer: block x = column tile ((x / nkb) % NJ + crot) % NJ, K block x % nkb
+        int64_t issued = 0;
+        for (int64_t x = 0; x < total_wb; ++x) {
+            const int s = (int)(x % kIpStages);
+            if (x >= kIpStages && !ip_wait(&wempty[s], (uint32_t)(((x / kIpStages) + 1) & 1), failed)) break;
+            const int64_t u = x % ((int64_t)NJ * nkb);
+            const int jj = ((int)(u / nkb) + crot) % NJ, kk = (int)(u % nkb);
+            unsigned char *dst = sw + s * kIpTile;
+            if (tma_w) {
+                if (lane == 0) {
+                    umma::mbar_arrive_expect_tx(&wfull[s], kIpTile);
+                    umma::tma_load_2d(dst, &tmW, kk * 64, jj * kIpN, &wfull[s]);
                 }
-            }
-            umma::fence_async_smem();
-            named_bar(1 + g, 128);
-            if ((tid & 127) == 0 && ok && live) umma::tma_store_2d(&tmOut, col0, ii * kInjM, buf);
-        } else if (ok && live) {
-            const int64_t p = (int64_t)ii * kInjM + row;
-            uint16_t *dst = out + p * D + col0;
-            const int left = D - col0;
+            } else {
+                for (int e = lane; e < kIpN * 8; e += 32) {
+                    const int nr = e >> 3, ch = e & 7;
+                    const int n = jj * kIpN + nr, c = kk * 64 + ch * 8;
+                    uint16_t t8[8];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t r[32];
-                umma::tmem_ld_32cols(ta + 32 * h, r);
-                if (p < P) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(r[j]));
-                        if (32 * h + j < left) dst[32 * h + j] = *reinterpret_cast<const uint16_t *>(&b);
-                    }
+                    for (int z = 0; z < 8; ++z) t8[z] = (n < D && c + z < C) ? W[(int64_t)n * C + c + z] : 0;
+                    *reinterpret_cast<uint4 *>(dst + umma::sw128_offset(nr, ch * 8)) =
+                        make_uint4(t8[0] | ((uint32_t)t8[1] << 16), t8[2] | ((uint32_t)t8[3] << 16),
+                                   t8[4] | ((uint32_t)t8[5] << 16), t8[6] | ((uint32_t)t8[7] << 16));
                 }
+                umma::fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&wfull[s]);
             }
+            issued = x + 1;
         }
-    };
-
-    for (int i = blockIdx.x; i < nrt; i += gridDim.x) {
-        // the previous row tile's last column tile: its MMAs still read A
-        if (pend_i >= 0) {
-            epilogue(pend_q, pend_i, pend_j);
-            pend_i = -1;
-        }
-        // A: row = tid % 128, channels [64 kb + 32 half, +32) of every K block
-        {
-            const int row = tid & 127, half = tid >> 7;
-            const int64_t p = (int64_t)i * kInjM + row;
-            const bool valid = p < P;
-            const int32_t *srow = sym;
-            if (valid) {
-                const int64_t b = p / T;
-                srow = sym + b * (int64_t)R * T + (p - b * T);
-            }
-            const uint32_t lowm = (1u << M) - 1u;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int cbase = kb * 64 + half * 32;
-                uint32_t vb = 0, mm = 0;
-                if (cbase < C) {
-                    const int r0 = cbase / M, r1 = min(C - 1, cbase + 31) / M;
+        // no load may still be landing at exit: wait for the last one of each stage
+        if (tma_w && lane == 0)
+            for (int s = 0; s < kIpStages; ++s)
+                if (issued > s) {
+                    const int64_t last = s + ((issued - 1 - s) / kIpStages) * kIpStages;
+                    if (!umma::mbar_wait_bounded(&wfull[s], (uint32_t)((last / kIpStages) & 1), kWaitPolls)) *failed = 1;
+                }
+    } else if (warp == 8) {
+        // ---- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = umma::make_idesc_bf16_f32(kInjM, kIpN);
+            int64_t q = 0, x = 0;
+            bool ok = true;
+            for (int k = 0; k < my_rt && ok; ++k) {
+                ok = ip_wait(afull, (uint32_t)(k & 1), failed);
+                for (int j = 0; j < NJ && ok; ++j, ++q) {
+                    const int b = (int)(q & 1);
+                    if (q >= 2) ok = ip_wait(&accempty[b], (uint32_t)(((q >> 1) + 1) & 1), failed);
+                    umma::tc_fence_after();
+                    const uint32_t dacc = tmem + (uint32_t)(b * kIpN);
+                    for (int kb = 0; kb < nkb && ok; ++kb, ++x) {
+                        const int s = (int)(x % kIpStages);
+                        ok = ip_wait(&wfull[s], (uint32_t)((x / kIpStages) & 1), failed);
+                        if (!ok) break;
+                        umma::tc_fence_after();
+                        const uint32_t ab = umma::smem_u32(sa + kb * kIpTile), bb = umma::smem_u32(sw + s * kIpTile);
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int r = r0 + u;
-                        if (r <= r1) {
-                            const int32_t av = valid ? __ldg(srow + (int64_t)r * T) : -1;
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma::mma_bf16(dacc, umma::make_kmajor_sw128_desc(ab + kk * 32),
+                                           umma::make_kmajor_sw128_desc(bb + kk * 32), idesc,
+                                           (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma::mma_commit(&wempty[s]);
+                    }
+                    umma::mma_commit(&accfull[b]);
+                }
+                umma::mma_commit(aempty);
+            }
+            // every MMA issued has completed before the CTA leaves
+            umma::mma_commit(drain);
+            if (!umma::mbar_wait_bounded(drain, 0u, kWaitPolls)) *failed = 1;
+        }
+    } else {
+        // ---- workers: A tiles and epilogues
+        const int g = warp >> 2, lbase = (warp & 3) * 32;
+        const int row = tid & 127, half = tid >> 7;
+        const uint32_t lowm = (1u << M) - 1u;
+        int64_t q = 0;
+        bool ok = true;
+        for (int k = 0; k < my_rt && ok; ++k) {
+            const int i = (int)blockIdx.x + k * (int)gridDim.x;
+            if (k >= 1) ok = ip_wait(aempty, (uint32_t)((k - 1) & 1), failed);
+            if (!ok) break;
+            // A: row = tid % 128, channels [64 kb + 32 half, +32) of every K block
+            {
+                const int64_t p = (int64_t)i * kInjM + row;
+                const bool valid = p < P;
+                const int32_t *srow = sym;
+                if (valid) {
+                    const int64_t bb = p / T;
+                    srow = sym + bb * (int64_t)R * T + (p - bb * T);
+                }
+                // Symbols of one batch -> the bf16 embedding of 32 channels per K block.
+                // One-bit routes: a K block's 32 channels are 32 routes, one batch per
+                // block.  Routes of 2+ bits: 32 channels span at most 16 routes, so two
+                // K blocks share a batch.  Every load of a batch is issued before the
+                // first is used.
+                auto emit = [&](int kbd, int cbase, int rlo, int rhi, const int32_t *sv, int first) {
+                    uint32_t vb = 0, mm = 0;
+#pragma unroll
+                    for (int u = 0; u < 16 * (2 - first / 16) && u < 32; ++u) {
+                        const int r = rlo + u;
+                        if (r <= rhi) {
+                            const int32_t av = sv[first + u];
                             const uint32_t bits = av >= 0 ? ((uint32_t)av & lowm) : 0u;
                             const uint32_t mk = av >= 0 ? lowm : 0u;
                             const int pos = r * M - cbase;
@@ -416,106 +462,108 @@ inject_persistent_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_c
                             }
                         }
                     }
-                }
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int k0 = ch * 8;
-                    const uint4 z0 = *reinterpret_cast<const uint4 *>(se0 + cbase + k0);
-                    const uint4 z1 = *reinterpret_cast<const uint4 *>(se1 + cbase + k0);
-                    uint4 v;
-                    v.x = select_pair(z0.x, z1.x, vb, mm, k0 + 0);
-                    v.y = select_pair(z0.y, z1.y, vb, mm, k0 + 2);
-                    v.z = select_pair(z0.z, z1.z, vb, mm, k0 + 4);
-                    v.w = select_pair(z0.w, z1.w, vb, mm, k0 + 6);
-                    *reinterpret_cast<uint4 *>(sa + kb * kIpTile + umma::sw128_offset(row, half * 32 + k0)) = v;
-                }
-            }
-            umma::fence_async_smem();
-        }
-        for (int j = 0; j < NJ; ++j) {
-            umma::tc_fence_before();
-            __syncthreads();   // A built; the previous epilogue's TMEM reads are done
-            if (*failed) break;
-            const uint32_t dacc = tmem + (uint32_t)((q & 1) * kIpN);
-            if (tma_w) {
-                if (tid == 0) {
-                    umma::tc_fence_after();
-                    for (int kb = 0; kb < nkb; ++kb, ++wb) {
-                        const int s = (int)(wb % kIpStages);
-                        if (!umma::mbar_wait_bounded(&wfull[s], (uint32_t)((wb / kIpStages) & 1), kWaitPolls)) {
-                            *failed = 1;
-                            break;
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int k0 = ch * 8;
+                        const uint4 z0 = *reinterpret_cast<const uint4 *>(se0 + cbase + k0);
+                        const uint4 z1 = *reinterpret_cast<const uint4 *>(se1 + cbase + k0);
+                        uint4 v;
+                        v.x = select_pair(z0.x, z1.x, vb, mm, k0 + 0);
+                        v.y = select_pair(z0.y, z1.y, vb, mm, k0 + 2);
+                        v.z = select_pair(z0.z, z1.z, vb, mm, k0 + 4);
+                        v.w = select_pair(z0.w, z1.w, vb, mm, k0 + 6);
+                        *reinterpret_cast<uint4 *>(sa + kbd * kIpTile + umma::sw128_offset(row, half * 32 + k0)) = v;
+                    }
+                };
+                if (M == 1) {
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const int cbase = kb * 64 + half * 32;
+                        const int r0 = cbase, r1 = cbase < C ? min(C - 1, cbase + 31) : cbase - 1;
+                        int32_t sv[32];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            sv[u] = (valid && r0 + u <= r1) ? __ldg(srow + (int64_t)(r0 + u) * T) : -1;
+                        emit(kb, cbase, r0, r1, sv, 0);
+                    }
+                } else {
+                    for (int kb = 0; kb < nkb; kb += 2) {
+                        const int ca = kb * 64 + half * 32, cb = ca + 64;
+                        const int ra0 = ca / M, ra1 = ca < C ? min(C - 1, ca + 31) / M : ra0 - 1;
+                        const int rb0 = cb / M, rb1 = (kb + 1 < nkb && cb < C) ? min(C - 1, cb + 31) / M : rb0 - 1;
+                        int32_t sv[32];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            sv[u] = (valid && ra0 + u <= ra1) ? __ldg(srow + (int64_t)(ra0 + u) * T) : -1;
+                            sv[16 + u] = (valid && rb0 + u <= rb1) ? __ldg(srow + (int64_t)(rb0 + u) * T) : -1;
                         }
-                        const uint32_t ab = umma::smem_u32(sa + kb * kIpTile), bb = umma::smem_u32(sw + s * kIpTile);
+                        emit(kb, ca, ra0, ra1, sv, 0);
+                        if (kb + 1 < nkb) emit(kb + 1, cb, rb0, rb1, sv, 16);
+                    }
+                }
+                umma::fence_async_smem();
+                mbar_arrive(afull);
+            }
+            // epilogues of this row tile's column tiles
+            for (int j = 0; j < NJ; ++j, ++q) {
+                const int b = (int)(q & 1);
+                const int col0 = ((j + crot) % NJ) * kIpN + g * 64;
+                const bool live = col0 < D;
+                ok = ip_wait(&accfull[b], (uint32_t)((q >> 1) & 1), failed);
+                ok = __all_sync(ROSA_FULL_MASK, ok);
+                umma::tc_fence_after();
+                const uint32_t ta = tmem + ((uint32_t)lbase << 16) + (uint32_t)(b * kIpN + g * 64);
+                const int orow = lbase + lane;
+                if (tma_out) {
+                    unsigned char *buf = sob + g * kIpTile;
+                    if ((tid & 127) == 0) umma::tma_store_wait_read();   // the box's previous store has read it
+                    named_bar(1 + g, 128);
+                    if (ok && live) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma::mma_bf16(dacc, umma::make_kmajor_sw128_desc(ab + kk * 32),
-                                           umma::make_kmajor_sw128_desc(bb + kk * 32), idesc,
-                                           (kb > 0 || kk > 0) ? 1u : 0u);
-                        umma::mma_commit(&wempty[s]);
-                        // refill the previous block's stage once its MMAs have read it
-                        if (wb >= 1 && wb - 1 + kIpStages < total_wb && w_issued == wb - 1 + kIpStages) {
-                            const int sp = (int)((wb - 1) % kIpStages);
-                            if (!umma::mbar_wait_bounded(&wempty[sp], (uint32_t)(((wb - 1) / kIpStages) & 1),
-                                                         kWaitPolls)) {
-                                *failed = 1;
-                                break;
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t r[32];
+                            umma::tmem_ld_32cols(ta + 32 * h, r);
+#pragma unroll
+                            for (int c4 = 0; c4 < 4; ++c4) {
+                                uint4 v;
+                                v.x = pack_bf16x2(__uint_as_float(r[8 * c4 + 0]), __uint_as_float(r[8 * c4 + 1]));
+                                v.y = pack_bf16x2(__uint_as_float(r[8 * c4 + 2]), __uint_as_float(r[8 * c4 + 3]));
+                                v.z = pack_bf16x2(__uint_as_float(r[8 * c4 + 4]), __uint_as_float(r[8 * c4 + 5]));
+                                v.w = pack_bf16x2(__uint_as_float(r[8 * c4 + 6]), __uint_as_float(r[8 * c4 + 7]));
+                                *reinterpret_cast<uint4 *>(buf + umma::sw128_offset(orow, 32 * h + 8 * c4)) = v;
                             }
-                            issue_w(w_issued++);
                         }
                     }
-                    umma::mma_commit(&accfull[q & 1]);
-                }
-            } else {
-                // W_out rows are not 16-byte aligned for TMA: every thread stages a share
-                for (int kb = 0; kb < nkb; ++kb, ++wb) {
-                    const int s = (int)(wb % kIpStages);
-                    if (wb >= kIpStages &&
-                        !umma::mbar_wait_bounded(&wempty[s], (uint32_t)(((wb - kIpStages) / kIpStages) & 1),
-                                                 kWaitPolls))
-                        *failed = 1;
-                    for (int e = tid; e < kIpN * 8; e += kIpThreads) {
-                        const int nr = e >> 3, ch = e & 7;
-                        const int n = j * kIpN + nr, c = kb * 64 + ch * 8;
-                        uint16_t t8[8];
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) t8[x] = (n < D && c + x < C) ? W[(int64_t)n * C + c + x] : 0;
-                        *reinterpret_cast<uint4 *>(sw + s * kIpTile + umma::sw128_offset(nr, ch * 8)) =
-                            make_uint4(t8[0] | ((uint32_t)t8[1] << 16), t8[2] | ((uint32_t)t8[3] << 16),
-                                       t8[4] | ((uint32_t)t8[5] << 16), t8[6] | ((uint32_t)t8[7] << 16));
-                    }
+                    umma::tc_fence_before();
+                    mbar_arrive(&accempty[b]);           // the accumulator may be overwritten
                     umma::fence_async_smem();
-                    __syncthreads();
-                    if (tid == 0 && !*failed) {
-                        umma::tc_fence_after();
-                        const uint32_t ab = umma::smem_u32(sa + kb * kIpTile), bb = umma::smem_u32(sw + s * kIpTile);
+                    named_bar(1 + g, 128);
+                    if ((tid & 127) == 0 && ok && live) umma::tma_store_2d(&tmOut, col0, i * kInjM, buf);
+                } else {
+                    if (ok && live) {
+                        const int64_t p = (int64_t)i * kInjM + orow;
+                        uint16_t *dst = out + p * D + col0;
+                        const int left = D - col0;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma::mma_bf16(dacc, umma::make_kmajor_sw128_desc(ab + kk * 32),
-                                           umma::make_kmajor_sw128_desc(bb + kk * 32), idesc,
-                                           (kb > 0 || kk > 0) ? 1u : 0u);
-                        umma::mma_commit(&wempty[s]);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t r[32];
+                            umma::tmem_ld_32cols(ta + 32 * h, r);
+                            if (p < P) {
+#pragma unroll
+                                for (int z = 0; z < 32; ++z) {
+                                    const __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(r[z]));
+                                    if (32 * h + z < left) dst[32 * h + z] = *reinterpret_cast<const uint16_t *>(&hv);
+                                }
+                            }
+                        }
                     }
+                    umma::tc_fence_before();
+                    mbar_arrive(&accempty[b]);
                 }
-                if (tid == 0 && !*failed) umma::mma_commit(&accfull[q & 1]);
+                if (!ok) break;
             }
-            if (pend_i >= 0) epilogue(pend_q, pend_i, pend_j);
-            pend_i = i;
-            pend_j = j;
-            pend_q = q;
-            ++q;
         }
-        __syncthreads();
-        if (*failed) break;
+        if ((tid & 127) == 0 && tma_out) umma::tma_store_wait_all();
     }
-    __syncthreads();
-    if (pend_i >= 0 && !*failed) epilogue(pend_q, pend_i, pend_j);
-    // nothing may be in flight at exit: loads not consumed, MMAs, stores
-    if (tid == 0 && tma_w)
-        for (int64_t x = wb; x < w_issued; ++x)
-            umma::mbar_wait_bounded(&wfull[x % kIpStages], (uint32_t)((x / kIpStages) & 1), kWaitPolls);
-    if (tid == 0 && *failed && q > 0) umma::mbar_wait_bounded(&accfull[(q - 1) & 1], (uint32_t)(((q - 1) >> 1) & 1), kWaitPolls);
-    if ((tid & 127) == 0 && tma_out) umma::tma_store_wait_all();
     umma::tc_fence_before();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(tmem, 2 * kIpN);
@@ -558,6 +606,14 @@ cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t
         if (!tma_w) memset(&tmW, 0, sizeof tmW);
         if (!tma_out) memset(&tmOut, 0, sizeof tmOut);
         // at most two CTAs per SM: each holds 256 of the SM's 512 tensor-memory columns
+        static bool ip_carve_set[64] = {};
+        if (dev >= 0 && dev < 64 && !ip_carve_set[dev]) {
+            // the whole unified L1 / shared array as shared memory, so that two CTAs fit where they can
+            e = cudaFuncSetAttribute(inject_persistent_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+            ip_carve_set[dev] = true;
+        }
         int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, inject_persistent_kernel, kIpThreads, smem);
         if (e != cudaSuccess) return e;

@@ -38,7 +38,7 @@ constexpr int kLnpMmaM = 128;       // rows of one single-CTA MMA (M = 256 exist
 constexpr int kLnpK = 64;           // K per block (one 128-byte swizzle row)
 constexpr int kLnpThreads = 256;    // one row each for the statistics; warps 4-7 take the second half
 constexpr int kLnpStages = 3;
-constexpr uint32_t kLnpWaitPolls = 1u << 24;
+constexpr uint32_t kLnpWaitPolls = umma::kWaitPolls;
 
 int gcd_int(int a, int b) { return b ? gcd_int(b, a % b) : a; }
 
@@ -51,15 +51,19 @@ int lnp_ne(int M) {
 struct LnpSmem {
     alignas(1024) unsigned char a[kLnpStages][kLnpM * 128];   // H block (256 rows), K-major SW128
     alignas(1024) unsigned char b[kLnpStages][256 * 128];     // hi / lo weight rows, K-major SW128
+    float cs[128], bv[128];                                    // this tile's column constants
     uint64_t full[kLnpStages], done[kLnpStages];
     uint32_t tmem;
     int failed;
 };
 
+constexpr int kPrepCols = 32;    // effective columns per prep CTA
+constexpr int kPrepK = 128;      // rows of W per prep CTA
+
 struct LnpLayout {
     uint16_t *wp;     // [NT * 2NE rows][D]: per tile NE high rows then NE low rows
-    float *cs;        // [NT * NE]: column sums of hi + lo
-    float *bv;        // [NT * NE]: beta . W
+    float *cs;        // [ceil(D / kPrepK)][NT * NE]: partial column sums of hi + lo
+    float *bv;        // [ceil(D / kPrepK)][NT * NE]: partial beta . W
     size_t bytes;
 };
 
@@ -75,9 +79,10 @@ LnpLayout lnp_carve(int D, int C, int M, void *base) {
         off += align256(n);
         return p;
     };
+    const int nkc = ceil_div(D, kPrepK);
     L.wp = (uint16_t *)take((size_t)NT * 2 * NE * D * 2);
-    L.cs = (float *)take((size_t)NT * NE * 4);
-    L.bv = (float *)take((size_t)NT * NE * 4);
+    L.cs = (float *)take((size_t)nkc * NT * NE * 4);
+    L.bv = (float *)take((size_t)nkc * NT * NE * 4);
     L.bytes = off;
     return L;
 }
@@ -89,20 +94,27 @@ __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-// One CTA per effective column (padding columns of the last tile write zeros).
+// One CTA per 32 effective columns x 128 rows of W (padding columns of the
+// last tile write zeros): a warp reads 32 consecutive columns of one row, the
+// high and low parts are transposed in shared memory and leave as 256-byte
+// row pieces; each CTA writes its partial column sums (the main kernel adds
+// the 128-row partials in a fixed order).
 __global__ void __launch_bounds__(256)
 lnp_prep_kernel(const float *__restrict__ gamma, const float *__restrict__ beta, const uint16_t *__restrict__ Wq,
-                const uint16_t *__restrict__ Wk, int D, int C, int NE, uint16_t *__restrict__ wp, float *__restrict__ cs,
-                float *__restrict__ bv) {
-    __shared__ float red[2][8];
-    const int n = blockIdx.x;
-    const int tile = n / NE, cn = n - tile * NE;
-    uint16_t *hi = wp + ((int64_t)tile * 2 * NE + cn) * D;
-    uint16_t *lo = wp + ((int64_t)tile * 2 * NE + NE + cn) * D;
+                const uint16_t *__restrict__ Wk, int D, int C, int NE, int NTNE, uint16_t *__restrict__ wp,
+                float *__restrict__ cs, float *__restrict__ bv) {
+    __shared__ __align__(16) uint16_t th[kPrepCols][kPrepK + 8], tl[kPrepCols][kPrepK + 8];
+    __shared__ float red[2][8][kPrepCols];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n0 = blockIdx.x * kPrepCols, k0 = blockIdx.y * kPrepK;
+    const int n = n0 + lane;
+    const bool valid = n < 2 * C;
     float s_cs = 0.f, s_bv = 0.f;
-    for (int k = threadIdx.x; k < D; k += 256) {
+#pragma unroll
+    for (int i = warp; i < kPrepK; i += 8) {   // all loads of a thread issued together
+        const int k = k0 + i;
         uint16_t h = 0, l = 0;
-        if (n < 2 * C) {
+        if (valid && k < D) {
             const float w = bf16_bits_to_float(n < C ? Wq[(int64_t)k * C + n] : Wk[(int64_t)k * C + n - C]);
             const float ws = (gamma ? gamma[k] : 1.f) * w;
             h = bf16_bits_rn(ws);
@@ -110,27 +122,33 @@ lnp_prep_kernel(const float *__restrict__ gamma, const float *__restrict__ beta,
             s_cs += bf16_bits_to_float(h) + bf16_bits_to_float(l);
             s_bv += (beta ? beta[k] : 0.f) * w;
         }
-        hi[k] = h;
-        lo[k] = l;
+        th[lane][i] = h;
+        tl[lane][i] = l;
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        s_cs += __shfl_xor_sync(ROSA_FULL_MASK, s_cs, o);
-        s_bv += __shfl_xor_sync(ROSA_FULL_MASK, s_bv, o);
-    }
-    if ((threadIdx.x & 31) == 0) {
-        red[0][threadIdx.x >> 5] = s_cs;
-        red[1][threadIdx.x >> 5] = s_bv;
-    }
+    red[0][warp][lane] = s_cs;
+    red[1][warp][lane] = s_bv;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    // rows n0 .. n0+31 of the high and low planes, columns k0 .. k0+255
+    const int kn = min(kPrepK, D - k0);
+    for (int r = warp; r < kPrepCols; r += 8) {
+        const int nn = n0 + r;
+        if (nn >= NTNE) break;
+        const int tile = nn / NE, cn = nn - tile * NE;
+        uint16_t *hi = wp + ((int64_t)tile * 2 * NE + cn) * D + k0;
+        uint16_t *lo = wp + ((int64_t)tile * 2 * NE + NE + cn) * D + k0;
+        for (int c = lane * 8; c < kn; c += 32 * 8) {   // D % 8 == 0: whole 16-byte pieces
+            *reinterpret_cast<uint4 *>(hi + c) = *reinterpret_cast<const uint4 *>(&th[r][c]);
+            *reinterpret_cast<uint4 *>(lo + c) = *reinterpret_cast<const uint4 *>(&tl[r][c]);
+        }
+    }
+    if (warp == 0 && n < NTNE) {
         float a = 0.f, c = 0.f;
         for (int w = 0; w < 8; ++w) {
-            a += red[0][w];
-            c += red[1][w];
+            a += red[0][w][lane];
+            c += red[1][w][lane];
         }
-        cs[n] = a;
-        bv[n] = c;
+        cs[(int64_t)blockIdx.y * NTNE + n] = a;
+        bv[(int64_t)blockIdx.y * NTNE + n] = c;
     }
 }
 
@@ -154,6 +172,17 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
         }
         umma::fence_mbar_init();
         sm.failed = 0;
+    }
+    // the epilogue's per-column constants, read once per CTA
+    if (tid < NE) {
+        const int nkc = ceil_div(D, kPrepK), NTNE = gridDim.y * NE;
+        float a = 0.f, c = 0.f;
+        for (int kc = 0; kc < nkc; ++kc) {
+            a += cs[(int64_t)kc * NTNE + tile * NE + tid];
+            c += bv[(int64_t)kc * NTNE + tile * NE + tid];
+        }
+        sm.cs[tid] = a;
+        sm.bv[tid] = c;
     }
     if (warp == 0) umma::tmem_alloc(&sm.tmem, 512);   // accumulators of the two row halves
     umma::tc_fence_before();
@@ -231,32 +260,44 @@ lnp_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUte
         const float mu = s1 / (float)D;
         const float var = fmaxf(s2 / (float)D - mu * mu, 0.f);
         const float rstd = rsqrtf(var + eps);
-        uint32_t bits[4] = {0, 0, 0, 0};   // threshold bits of the NE effective columns
-        for (int c0 = 0; c0 < NE; c0 += 32) {
-            uint32_t h[32], l[32];
-            umma::tmem_ld_32cols(tacc + (uint32_t)c0, h);
-            umma::tmem_ld_32cols(tacc + (uint32_t)(NE + c0), l);
+        // threshold bits of the NE effective columns, kept in registers: every
+        // index into them is a compile-time constant or an explicit select
+        uint32_t bits[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int cn = c0 + j;
-                if (cn < NE) {
-                    const int n = tile * NE + cn;
-                    const float acc = __uint_as_float(h[j]) + __uint_as_float(l[j]);
-                    const float x = rstd * (acc - mu * cs[n]) + bv[n];
-                    if (x > 0.f) bits[cn >> 5] |= 1u << (cn & 31);
+        for (int w = 0; w < 4; ++w) {
+            const int c0 = 32 * w;
+            if (c0 < NE) {
+                uint32_t h[32], l[32];
+                umma::tmem_ld_32cols(tacc + (uint32_t)c0, h);
+                umma::tmem_ld_32cols(tacc + (uint32_t)(NE + c0), l);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int cn = c0 + j;
+                    if (cn < NE) {
+                        const float acc = __uint_as_float(h[j]) + __uint_as_float(l[j]);
+                        const float x = rstd * (acc - mu * sm.cs[cn]) + sm.bv[cn];
+                        if (x > 0.f) bits[w] |= 1u << j;
+                    }
                 }
             }
         }
         if (p < P) {
             const int64_t b = p / T, t = p - b * T;
             const int R = C / M;
-            for (int cn = 0; cn < NE; cn += M) {
+            const uint32_t lowm = (1u << M) - 1u;
+            // effective column n = tile*NE + cn is bit 0 of route n / M of the query
+            // channels (n < C) or route n / M - R of the key channels; M divides NE and C
+            int ra = tile * NE / M;
+            for (int cn = 0; cn < NE; cn += M, ++ra) {
                 const int n = tile * NE + cn;
                 if (n >= 2 * C) break;
-                unsigned a = 0;
-                for (int j = 0; j < M; ++j) a |= ((bits[(cn + j) >> 5] >> ((cn + j) & 31)) & 1u) << j;
-                const bool isq = n < C;
-                const int r = (isq ? n : n - C) / M;
+                // M bits from column cn on (M divides NE, so they may straddle two words)
+                const int wd = cn >> 5, o = cn & 31;
+                const uint32_t lo = wd == 0 ? bits[0] : wd == 1 ? bits[1] : wd == 2 ? bits[2] : bits[3];
+                const uint32_t hi = wd == 0 ? bits[1] : wd == 1 ? bits[2] : wd == 2 ? bits[3] : 0u;
+                const uint32_t a = ((lo >> o) | (o ? hi << (32 - o) : 0u)) & lowm;
+                const bool isq = ra < R;
+                const int r = isq ? ra : ra - R;
                 (isq ? symq : symk)[(b * R + r) * (int64_t)T + t] = (uint8_t)a;
             }
         }
@@ -296,7 +337,8 @@ cudaError_t launch_ln_project(const uint16_t *H, const float *gamma, const float
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
-    lnp_prep_kernel<<<(unsigned)(NT * NE), 256, 0, st>>>(gamma, beta, Wq, Wk, D, C, NE, L.wp, L.cs, L.bv);
+    lnp_prep_kernel<<<dim3((unsigned)ceil_div(NT * NE, kPrepCols), (unsigned)ceil_div(D, kPrepK)), 256, 0, st>>>(
+        gamma, beta, Wq, Wk, D, C, NE, NT * NE, L.wp, L.cs, L.bv);
     dim3 grid((unsigned)ceil_div64(P, kLnpM), (unsigned)NT);
     lnp_kernel<<<grid, kLnpThreads, smem, st>>>(tmH, tmW, P, T, D, C, M, NE, eps, L.cs, L.bv, symq, symk, status);
     return cudaGetLastError();

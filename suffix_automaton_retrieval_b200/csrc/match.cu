@@ -1175,11 +1175,14 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, const uint32_t *leaf
         }
         if (l >= r) { alive = false; break; }
     }
-    if (alive) {   // values with X's top nlev bits
+    if (alive) {   // values with X's top nlev bits, eight independent loads at a time
         int best = -1;
-        for (int i = l; i < r; ++i) {
-            const int v = (int)leaf[i];
-            if (v <= X && v > best) best = v;
+        for (int i0 = l; i0 < r; i0 += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int v = i0 + u < r ? (int)__ldg(leaf + i0 + u) : -1;
+                if (v <= X && v > best) best = v;
+            }
         }
         if (best >= 0) return best;
     }
@@ -1200,7 +1203,10 @@ __device__ int wavelet_max_le(const WWord *W, const int *Z, const uint32_t *leaf
         }
     }
     int best = -1;
-    for (int i = l; i < r; ++i) best = max(best, (int)leaf[i]);
+    for (int i0 = l; i0 < r; i0 += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) best = max(best, i0 + u < r ? (int)__ldg(leaf + i0 + u) : -1);
+    }
     return best;
 }
 
@@ -1924,7 +1930,8 @@ __global__ void bound_finish_kernel(Geometry G, ResolveArgs A, Outs O,
 }
 
 // Largest admissible key position inside each parked query's key range.
-__global__ void wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, Outs O,
+__global__ void __launch_bounds__(256, 8)
+wavelet_query_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym, Outs O,
                                      const int32_t *__restrict__ wq, const int *__restrict__ wq_count) {
     const int nq = *wq_count;
     const int nw = (G.T >> 6) + 1;

@@ -54,22 +54,29 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// A waiting thread is suspended until the phase completes or this many
+// nanoseconds pass, instead of re-polling the barrier word: the barrier stays
+// free for the TMA engine's and the tensor cores' arrivals.
+constexpr uint32_t kSuspendNs = 1000000;
+// Polls of a bounded wait: about two seconds.
+constexpr uint32_t kWaitPolls = 2000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
 
 // Waits for the phase with the given parity to complete, at most `limit`
-// polls (each poll may itself wait a bounded time in hardware).  Returns
-// false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit) {
+// polls (each suspends the thread for up to kSuspendNs).  Returns false when
+// the limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
