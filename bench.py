@@ -457,19 +457,21 @@ def reduce_over_ranks(local_ms: float, local_units: float, device=None):
 # call's launches), keyed by workload, with the digest of the CUDA sources
 # the capture was taken on.  The figure is reported only while the sources
 # are unchanged; otherwise the line carries null.
-PROFILED_DRAM_BYTES = {}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu pass per
+# launch) of one full-size match call, with the digest of the sources the
+# match kernels are built from; reported as `traffic` only while they match.
+PROFILED_DRAM_BYTES = {"zipf-256-131k": (9894443776, "8ccd53b42ca4bb41")}
+MATCH_SOURCES = ("match.cu", "common.cuh")
 
 
-def cuda_source_digest() -> str:
-    """sha256 over the CUDA sources of the library (file names and bytes)."""
-    import glob
+def cuda_source_digest(files=MATCH_SOURCES) -> str:
+    """sha256 over the named CUDA sources of the library (file names and bytes)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "suffix_automaton_retrieval_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
-                    glob.glob(os.path.join(csrc, "*.h"))):
-        h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+    for name in sorted(files):
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
 

@@ -227,9 +227,12 @@ keys0_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geome
     const uint8_t *a = (kind == 0 ? k : q) + (int64_t)s * G.T;
     const int p0 = tile * kKeysTile;
     const int lim = min(kKeysTile, G.T - p0);
-    for (int i = threadIdx.x; i < kMaxD0 + kKeysTile; i += kKeysThreads) {
+#pragma unroll
+    for (int u = 0; u < (kMaxD0 + kKeysTile + kKeysThreads - 1) / kKeysThreads; ++u) {   // all loads in flight
+        const int i = u * kKeysThreads + threadIdx.x;
         const int p = p0 - kMaxD0 + i;
-        sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;   // zeros before the start pad short strings
+        if (i < kMaxD0 + kKeysTile)
+            sb[i] = (p >= 0 && p < G.T) ? a[p] : 0;   // zeros before the start pad short strings
     }
     __syncthreads();
     const uint32_t symmask = (1u << G.bps) - 1u;
@@ -960,52 +963,69 @@ key_tile_count_kernel(Geometry G, const uint32_t *__restrict__ sa, int *__restri
 }
 
 // Level-0 sequence (key positions in rank order), the exclusive key count
-// before every rank (q != k), and the level-0 ones per wavelet tile.
+// before every rank (q != k), and the level-0 ones per wavelet tile.  The
+// tile's sa loads and the key count of the tiles before it are in flight
+// together (a warp sums the per-tile counts), and one scan over the 8 x 8
+// (round, warp) key counts gives every thread its offsets.
 __global__ void __launch_bounds__(256)
 wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, const int *__restrict__ ktile,
                        int32_t *__restrict__ kcount, uint32_t *__restrict__ a0, int *__restrict__ wcnt0) {
-    __shared__ int wk[8];
+    __shared__ int wk[kRadixIPT * 8];     // keys per (round, warp), then exclusive offsets
     __shared__ int pre_s;
+    __shared__ int ones[2];
     const int s = blockIdx.x / G.ntps, tt = blockIdx.x - s * G.ntps;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t base = (int64_t)s * G.n + (int64_t)tt * kRadixTile;
     const int lim = min(kRadixTile, G.n - tt * kRadixTile);
     const int ntw = ceil_div(G.T, kWTile);
-    if (threadIdx.x == 0) {
-        int p = 0;
-        if (G.allkeys) p = tt * kRadixTile;
-        else for (int i = 0; i < tt; ++i) p += ktile[(int64_t)s * G.ntps + i];
-        pre_s = p;
-    }
-    // this tile's keys take consecutive key indices, so they touch at most two wavelet tiles
-    __shared__ int ones[2];
-    if (threadIdx.x < 2) ones[threadIdx.x] = 0;
-    __syncthreads();
-    int run = pre_s;
-    const int t0 = run / kWTile;
-    int c0 = 0, c1 = 0;   // level-0 ones landing in wavelet tiles t0 and t0 + 1
     uint32_t xs[kRadixIPT];
-#pragma unroll
-    for (int u = 0; u < kRadixIPT; ++u) {   // loads first: the loop below has barriers
-        const int i = u * 256 + threadIdx.x;
-        xs[u] = i < lim ? sa[base + i] : 0u;
-    }
 #pragma unroll
     for (int u = 0; u < kRadixIPT; ++u) {
         const int i = u * 256 + threadIdx.x;
-        const bool ok = i < lim;
-        const uint32_t x = xs[u];
-        const bool key = ok && (int)x < G.T;
-        const unsigned bal = __ballot_sync(ROSA_FULL_MASK, key);
-        if (lane == 0) wk[warp] = __popc(bal);
-        __syncthreads();
-        int wpre = 0, rtot = 0;
-        for (int w = 0; w < 8; ++w) {
-            if (w < warp) wpre += wk[w];
-            rtot += wk[w];
+        xs[u] = i < lim ? sa[base + i] : 0u;
+    }
+    if (warp == 0) {
+        int p = 0;
+        if (G.allkeys) {
+            p = tt * kRadixTile;
+        } else {
+            for (int i = lane; i < tt; i += 32) p += ktile[(int64_t)s * G.ntps + i];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) p += __shfl_xor_sync(ROSA_FULL_MASK, p, o);
         }
-        const int kidx = run + wpre + __popc(bal & lanemask_lt());
-        if (ok && !G.allkeys) kcount[base + i] = kidx;
+        if (lane == 0) pre_s = p;
+    }
+    if (threadIdx.x < 2) ones[threadIdx.x] = 0;
+    unsigned bal[kRadixIPT];
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {
+        const int i = u * 256 + threadIdx.x;
+        bal[u] = __ballot_sync(ROSA_FULL_MASK, i < lim && (int)xs[u] < G.T);
+        if (lane == 0) wk[u * 8 + warp] = __popc(bal[u]);
+    }
+    __syncthreads();
+    if (warp == 0) {   // exclusive scan of the 64 counts, round-major
+        const int c0v = wk[lane], c1v = wk[32 + lane];
+        int i0 = c0v, i1 = c1v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(ROSA_FULL_MASK, i0, o), y1 = __shfl_up_sync(ROSA_FULL_MASK, i1, o);
+            if (lane >= o) { i0 += y0; i1 += y1; }
+        }
+        const int first = __shfl_sync(ROSA_FULL_MASK, i0, 31);
+        wk[lane] = pre_s + i0 - c0v;
+        wk[32 + lane] = pre_s + first + i1 - c1v;
+    }
+    __syncthreads();
+    const int t0 = pre_s / kWTile;
+    int c0 = 0, c1 = 0;   // level-0 ones landing in wavelet tiles t0 and t0 + 1
+#pragma unroll
+    for (int u = 0; u < kRadixIPT; ++u) {
+        const int i = u * 256 + threadIdx.x;
+        const uint32_t x = xs[u];
+        const bool key = (bal[u] >> lane) & 1u;
+        const int kidx = wk[u * 8 + warp] + __popc(bal[u] & lanemask_lt());
+        if (i < lim && !G.allkeys) kcount[base + i] = kidx;
         if (key) {
             a0[(int64_t)s * G.T + kidx] = x;
             if ((x >> (nbits - 1)) & 1u) {
@@ -1013,8 +1033,6 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
                 else ++c1;
             }
         }
-        run += rtot;
-        __syncthreads();
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -1043,6 +1061,14 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = nbits - 1 - lv;
     const int *cnt = wcnt + ((int64_t)lv * G.S + s) * ntw;
+    const int lim = min(kWTile, G.T - tt * kWTile);
+    const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
+    uint32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {   // the tile's values and the tile counts are loaded together
+        const int i = warp * 256 + u * 32 + lane;
+        v[u] = i < lim ? src[i] : 0u;
+    }
     int a = 0, tot = 0;
     for (int i = threadIdx.x; i < ntw; i += 256) {
         const int c = cnt[i];
@@ -1054,17 +1080,12 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         a += __shfl_xor_sync(ROSA_FULL_MASK, a, o);
         tot += __shfl_xor_sync(ROSA_FULL_MASK, tot, o);
     }
-    const int lim = min(kWTile, G.T - tt * kWTile);
-    const uint32_t *src = in + (int64_t)s * G.T + (int64_t)tt * kWTile;
-    uint32_t v[8];
     unsigned bal[8];
     int mine = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const int i = warp * 256 + u * 32 + lane;
-        const bool ok = i < lim;
-        v[u] = ok ? src[i] : 0u;
-        bal[u] = __ballot_sync(ROSA_FULL_MASK, ok && ((v[u] >> b) & 1u));
+        bal[u] = __ballot_sync(ROSA_FULL_MASK, i < lim && ((v[u] >> b) & 1u));
         mine += __popc(bal[u]);
     }
     if (lane == 0) {
