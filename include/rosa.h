@@ -172,6 +172,10 @@ ROSA_API int rosa_match_cf_launch_count(int S, int T, int M, int q_is_k);
  *   len[s, t]     = L              (counted in runs)
  *   sym[s, t]     = v[s, s_{l*+1}]  (-1 if L = 0)
  * Without adjacent repeats every run is one symbol and this is rosa_match.
+ * With K = 2 folded streams alternate, so the answer for query run m is the
+ * last admissible key run with d_m's symbol, L = min(l*, m) + 1; the call
+ * computes that directly instead of sorting (same results; symbols >= 2 are
+ * flagged, and for such streams the outputs of this path are unspecified).
  * Shapes, ownership and errors as for rosa_match; the workspace is at least
  * rosa_match_rle_workspace_size(S, T, K) bytes (256-byte aligned) and its
  * status word is read with rosa_match_device_status.

@@ -231,6 +231,42 @@ __global__ void rle_bound_kernel(int S, int T, int g, const int32_t *__restrict_
     }
 }
 
+// Binary alphabet (K = 2): consecutive runs differ, so a folded stream
+// alternates and its whole run history is fixed by its last symbol.  The
+// run-level suffix of query run m then matches key run l over min(m, l) + 1
+// runs when the two symbols agree and not at all otherwise, so the longest
+// admissible match ends at the last admissible key run with query run m's
+// symbol: X_m or X_m - 1.  Every real run's symbol is also checked against
+// the alphabet (the status word of the workspace).
+__global__ void rle_binary_kernel(int S, int T, const int32_t *__restrict__ nrun, const uint8_t *__restrict__ qr,
+                                  const uint8_t *__restrict__ kr, const int32_t *__restrict__ xb,
+                                  int32_t *__restrict__ rend, int32_t *__restrict__ rlen, uint32_t *__restrict__ status) {
+    const int64_t total = (int64_t)S * T;
+    bool bad = false;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int s = (int)(i / T), m = (int)(i - (int64_t)s * T);
+        const int nk = nrun[s * 2], nq = nrun[s * 2 + 1];
+        if (m < nk) bad |= kr[i] >= 2;
+        int e = -1, L = 0;
+        if (m < nq) {
+            const uint8_t d = qr[i];
+            bad |= d >= 2;
+            const int X = xb[i];
+            if (X >= 0) {
+                const int l = kr[(int64_t)s * T + X] == d ? X : X - 1;
+                if (l >= 0) {
+                    e = l;
+                    L = min(l, m) + 1;
+                }
+            }
+        }
+        rend[i] = e;
+        rlen[i] = L;
+    }
+    if (bad) atomicOr(status, ROSA_DEV_SYMBOL_RANGE);
+}
+
 // Every position reads its query run's answer and maps it to the time axis.
 __global__ void __launch_bounds__(kRleThreads)
 rle_map_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ vs, int T, int ntile, int qwhich,
@@ -289,7 +325,7 @@ size_t match_rle_workspace_bytes(int S, int T, int K, bool same) {
 
 int match_rle_launch_count(int S, int T, int K, bool same) {
     if (S == 0 || T == 0) return 0;
-    return 4 + match_launch_count(S, T, K, same) + 1;
+    return 4 + (K == 2 ? 1 : match_launch_count(S, T, K, same)) + 1;
 }
 
 cudaError_t launch_match_rle(const uint8_t *q, const uint8_t *k, const uint8_t *v, int S, int T, int K, int g,
@@ -310,9 +346,16 @@ cudaError_t launch_match_rle(const uint8_t *q, const uint8_t *k, const uint8_t *
     rle_write_kernel<<<tiles, kRleThreads, 0, st>>>(q, k, T, K, ntile, nwhich, L.tcnt, L.nrun, L.kr, L.qr, L.kstart,
                                                     L.qstart, L.krun);
     rle_bound_kernel<<<(unsigned)(device_sm_count() * 8), 256, 0, st>>>(S, T, g, L.nrun, L.qstart, L.krun, L.xb);
-    cudaError_t e = launch_match(L.qr, L.kr, nullptr, S, T, K, g, L.rend, L.rlen, L.rsym, workspace, L.match_bytes,
-                                 st, L.xb);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (K == 2) {
+        uint32_t *status = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + kStatusOffset);
+        if ((e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+        rle_binary_kernel<<<(unsigned)(device_sm_count() * 8), 256, 0, st>>>(S, T, L.nrun, L.qr, L.kr, L.xb, L.rend,
+                                                                             L.rlen, status);
+    } else {
+        e = launch_match(L.qr, L.kr, nullptr, S, T, K, g, L.rend, L.rlen, L.rsym, workspace, L.match_bytes, st, L.xb);
+        if (e != cudaSuccess) return e;
+    }
     rle_map_kernel<<<(unsigned)((int64_t)S * ntile), kRleThreads, 0, st>>>(q, v ? v : k, T, ntile, same ? 0 : 1,
                                                                            L.tcnt, L.kstart, L.rend, L.rlen, end_idx,
                                                                            len, sym);
