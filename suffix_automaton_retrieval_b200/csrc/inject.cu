@@ -614,9 +614,23 @@ cudaError_t launch_inject(const int32_t *sym, const uint16_t *e0, const uint16_t
             if (e != cudaSuccess) return e;
             ip_carve_set[dev] = true;
         }
-        int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, inject_persistent_kernel, kIpThreads, smem);
-        if (e != cudaSuccess) return e;
+        // CTAs per SM from the SM's shared memory and registers (at most two:
+        // each CTA holds 256 of the SM's 512 tensor-memory columns)
+        static int ip_regs[64] = {};
+        if (dev >= 0 && dev < 64 && ip_regs[dev] == 0) {
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, inject_persistent_kernel)) != cudaSuccess) return e;
+            ip_regs[dev] = fa.numRegs;
+        }
+        int smem_sm = 0, smem_rsv = 0, regs_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess)
+            return e;
+        const int regs = (dev >= 0 && dev < 64) ? ip_regs[dev] : 96;
+        const int regs_cta = ((regs * 32 + 255) / 256) * 256 * (kIpThreads / 32);   // per-warp allocation units
+        int per_sm = smem_sm / (smem + smem_rsv);
+        if (regs_cta > 0) per_sm = min(per_sm, regs_sm / regs_cta);
         per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);
         const int64_t nrt = ceil_div64(P, kInjM);
         const int64_t slots = (int64_t)per_sm * device_sm_count();

@@ -1388,7 +1388,12 @@ __device__ __forceinline__ void defer_wavelet(const Outs &O, int64_t o, int L, i
 // whole blocks per step from their summaries (smallest key position, LCP
 // minimum) and scans only the first block that holds an admissible key.
 __device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int lim, int lane) {
+    // The running LCP first drops to <= lim at the first lane whose own edge
+    // is <= lim (the carry from earlier steps is > lim, or the scan would have
+    // ended), so a ballot finds the stop and one warp min-reduction over the
+    // lanes before a hit gives the running LCP there.
     constexpr int kNB = kRWin / 32;
+    const unsigned lt = lanemask_lt();
     int blk, cnt0, r;
     if (dir < 0) {
         const int rtop = jl - 1;
@@ -1403,14 +1408,16 @@ __device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int l
     }
     int e = lane < cnt0 ? (dir < 0 ? w.lc[r + 1] : w.lc[r]) : INT_MAX;
     const bool valid = lane < cnt0 && w.kp[r] <= X;
-    int pm = warp_prefix_min(e, lane);
-    unsigned sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
-    const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid && pm > lim);
+    unsigned sm = __ballot_sync(ROSA_FULL_MASK, e <= lim);
     int fs = sm ? __ffs(sm) - 1 : 32;
-    const int fv = vm ? __ffs(vm) - 1 : 32;
-    if (fv < fs) return __shfl_sync(ROSA_FULL_MASK, pm, fv);
+    const unsigned before_fs = fs < 32 ? ((1u << fs) - 1u) : ROSA_FULL_MASK;
+    const unsigned vm = __ballot_sync(ROSA_FULL_MASK, valid) & before_fs;
+    if (vm) {
+        const int fv = __ffs(vm) - 1;
+        return __reduce_min_sync(ROSA_FULL_MASK, lane <= fv ? e : INT_MAX);
+    }
     if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
-    int carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
+    int carry = __reduce_min_sync(ROSA_FULL_MASK, e);
     for (int B0 = blk + dir;; B0 += 32 * dir) {   // ends at the window edge at the latest
         const int B = B0 + dir * lane;
         bool has = false;
@@ -1423,26 +1430,25 @@ __device__ int warp_nearest_smem(const WinSmem &w, int jl, int X, int dir, int l
         } else {
             e = kNeedHard;
         }
-        pm = min(carry, warp_prefix_min(e, lane));
-        sm = __ballot_sync(ROSA_FULL_MASK, pm <= lim);
+        sm = __ballot_sync(ROSA_FULL_MASK, e <= lim);
         const unsigned hm = __ballot_sync(ROSA_FULL_MASK, has);
         fs = sm ? __ffs(sm) - 1 : 32;
         const int fh = hm ? __ffs(hm) - 1 : 32;
         if (fh < 32 && fh <= fs) {   // the first block with an admissible key, entered above lim
-            const int before = __shfl_up_sync(ROSA_FULL_MASK, pm, 1);
-            int cin = __shfl_sync(ROSA_FULL_MASK, before, fh);
-            if (fh == 0) cin = carry;
+            const int cin = min(carry, __reduce_min_sync(ROSA_FULL_MASK, lane < fh ? e : INT_MAX));
             const int Bh = B0 + dir * fh;
             const int rr = dir < 0 ? 32 * Bh + 31 - lane : 32 * Bh + lane;
             const int e2 = dir < 0 ? w.lc[rr + 1] : w.lc[rr];
-            const int pm2 = min(cin, warp_prefix_min(e2, lane));
-            const unsigned sm2 = __ballot_sync(ROSA_FULL_MASK, pm2 <= lim);
-            const unsigned vm2 = __ballot_sync(ROSA_FULL_MASK, w.kp[rr] <= X && pm2 > lim);
-            const int fs2 = sm2 ? __ffs(sm2) - 1 : 32, fv2 = vm2 ? __ffs(vm2) - 1 : 32;
-            return fv2 < fs2 ? __shfl_sync(ROSA_FULL_MASK, pm2, fv2) : 0;
+            const unsigned sm2 = __ballot_sync(ROSA_FULL_MASK, e2 <= lim);
+            const int fs2 = sm2 ? __ffs(sm2) - 1 : 32;
+            const unsigned vm2 = __ballot_sync(ROSA_FULL_MASK, w.kp[rr] <= X) &
+                                 (fs2 < 32 ? ((1u << fs2) - 1u) : ROSA_FULL_MASK);
+            if (!vm2) return 0;
+            const int fv2 = __ffs(vm2) - 1;
+            return min(cin, __reduce_min_sync(ROSA_FULL_MASK, lane <= fv2 ? e2 : INT_MAX));
         }
         if (fs < 32) return __shfl_sync(ROSA_FULL_MASK, e, fs) == kNeedHard ? kNeedHard : 0;
-        carry = __shfl_sync(ROSA_FULL_MASK, pm, 31);
+        carry = min(carry, __reduce_min_sync(ROSA_FULL_MASK, e));
     }
 }
 
