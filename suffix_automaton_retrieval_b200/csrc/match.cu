@@ -1329,15 +1329,6 @@ __device__ __forceinline__ void write_result(const uint8_t *vsym, const Outs &O,
     }
 }
 
-__device__ __forceinline__ int warp_prefix_min(int x, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(ROSA_FULL_MASK, x, o);
-        if (lane >= o) x = min(x, y);
-    }
-    return x;
-}
-
 // Staged window of one resolve tile (local ranks 0..kRWin-1):
 //   kp[i]  key position of local rank i, INT_MAX for query items and ranks
 //          outside the stream;
@@ -1739,6 +1730,10 @@ enum ScanMode { NEAREST = 0, BOUND = 1 };
 template <int MODE>
 __device__ bool warp_fine(const StreamView &v, int first, int cnt, int dir, int X, int lim, int lane, int &carry,
                           int &result) {
+    // carry (the running LCP before this step) is above lim (NEAREST) or at
+    // least lim (BOUND), or the scan would have ended: the stop is the first
+    // lane whose own edge crosses lim, and a warp min-reduction over the
+    // lanes up to a hit gives the running LCP there
     const int r = first + dir * lane;
     const bool act = lane < cnt && r >= 0 && r < v.n;
     int e = INT_MAX;
@@ -1749,14 +1744,13 @@ __device__ bool warp_fine(const StreamView &v, int first, int cnt, int dir, int 
     } else if (lane < cnt) {
         e = -1;   // ran off the stream: ends every scan
     }
-    const int m = min(carry, warp_prefix_min(e, lane));
     if (MODE == NEAREST) {
-        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && m <= lim);
-        const unsigned valm = __ballot_sync(ROSA_FULL_MASK, valid && m > lim);
+        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && e <= lim);
         const int fs = stopm ? __ffs(stopm) - 1 : 32;
-        const int fv = valm ? __ffs(valm) - 1 : 32;
-        if (fv < fs) {
-            result = __shfl_sync(ROSA_FULL_MASK, m, fv);
+        const unsigned valm = __ballot_sync(ROSA_FULL_MASK, valid) & (fs < 32 ? ((1u << fs) - 1u) : ROSA_FULL_MASK);
+        if (valm) {
+            const int fv = __ffs(valm) - 1;
+            result = min(carry, __reduce_min_sync(ROSA_FULL_MASK, lane <= fv ? e : INT_MAX));
             return true;
         }
         if (fs < 32) {
@@ -1764,7 +1758,7 @@ __device__ bool warp_fine(const StreamView &v, int first, int cnt, int dir, int 
             return true;
         }
     } else {
-        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && m < lim);
+        const unsigned stopm = __ballot_sync(ROSA_FULL_MASK, lane < cnt && e < lim);
         if (stopm) {
             const int fs = __ffs(stopm) - 1;
             result = first + dir * (fs - 1);
@@ -1772,7 +1766,7 @@ __device__ bool warp_fine(const StreamView &v, int first, int cnt, int dir, int 
         }
         result = first + dir * (cnt - 1);
     }
-    carry = __shfl_sync(ROSA_FULL_MASK, m, 31);
+    carry = min(carry, __reduce_min_sync(ROSA_FULL_MASK, e));
     return false;
 }
 
@@ -1799,12 +1793,13 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
                 bm2 = min(edge, v.em2[b2]);
                 hv2 = v.mp2[b2] <= X;
             }
-            const int M2 = min(carry, warp_prefix_min(bm2, lane));
-            const bool st2 = MODE == NEAREST ? (!in2 || hv2 || M2 <= lim) : (!in2 || M2 < lim);
+            // the first stop: the first block that leaves the stream, holds an
+            // admissible key, or whose own LCP minimum crosses lim (carry does not)
+            const bool st2 = MODE == NEAREST ? (!in2 || hv2 || bm2 <= lim) : (!in2 || bm2 < lim);
             const unsigned sm2 = __ballot_sync(ROSA_FULL_MASK, st2);
             const int f2 = sm2 ? __ffs(sm2) - 1 : 32;
             if (f2 > 0) {
-                carry = min(carry, __shfl_sync(ROSA_FULL_MASK, M2, f2 - 1));
+                carry = min(carry, __reduce_min_sync(ROSA_FULL_MASK, lane < f2 ? bm2 : INT_MAX));
                 if (MODE == BOUND) {
                     const int bl = nb2 + dir * (f2 - 1);
                     result = dir < 0 ? bl * kL2 : bl * kL2 + kL2 - 1;
@@ -1824,12 +1819,11 @@ __device__ int warp_scan(const StreamView &v, int j, int dir, int X, int lim, in
             bm = min(edge, v.em1[b]);
             has_valid = v.mp1[b] <= X;
         }
-        const int M = min(carry, warp_prefix_min(bm, lane));
-        const bool stop_here = MODE == NEAREST ? (!inside || has_valid || M <= lim) : (!inside || M < lim);
+        const bool stop_here = MODE == NEAREST ? (!inside || has_valid || bm <= lim) : (!inside || bm < lim);
         const unsigned sm = __ballot_sync(ROSA_FULL_MASK, stop_here);
         const int f = sm ? __ffs(sm) - 1 : 32;
         if (f > 0) {
-            carry = min(carry, __shfl_sync(ROSA_FULL_MASK, M, f - 1));
+            carry = min(carry, __reduce_min_sync(ROSA_FULL_MASK, lane < f ? bm : INT_MAX));
             if (MODE == BOUND) {
                 const int bl = nb + dir * (f - 1);
                 result = dir < 0 ? bl * kL1 : bl * kL1 + kL1 - 1;
