@@ -892,12 +892,8 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int first = __shfl_sync(ROSA_FULL_MASK, l[u], 0);
-        int mp = pos[u], me = lane == 0 ? INT_MAX : l[u];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            mp = min(mp, __shfl_xor_sync(ROSA_FULL_MASK, mp, o));
-            me = min(me, __shfl_xor_sync(ROSA_FULL_MASK, me, o));
-        }
+        const int mp = __reduce_min_sync(ROSA_FULL_MASK, pos[u]);
+        const int me = __reduce_min_sync(ROSA_FULL_MASK, lane == 0 ? INT_MAX : l[u]);
         const int blk = u * 8 + warp;   // 32-rank block within the 1024
         const int b1 = B2 * (kL2 / kL1) + blk;
         if (lane == 0) {
@@ -914,12 +910,8 @@ summary_kernel(Geometry G, const uint32_t *__restrict__ sa, const int32_t *__res
     if (threadIdx.x == 0) edge_in = l[0];
     __syncthreads();
     if (warp == 0) {
-        int p2 = wpos[lane], e2 = min(wemin[lane], wfirst[lane]);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            p2 = min(p2, __shfl_xor_sync(ROSA_FULL_MASK, p2, o));
-            e2 = min(e2, __shfl_xor_sync(ROSA_FULL_MASK, e2, o));
-        }
+        const int p2 = __reduce_min_sync(ROSA_FULL_MASK, wpos[lane]);
+        const int e2 = __reduce_min_sync(ROSA_FULL_MASK, min(wemin[lane], wfirst[lane]));
         if (lane == 0) {
             minpos2[(int64_t)s * G.nb2 + B2] = p2;
             emin2[(int64_t)s * G.nb2 + B2] = e2;
@@ -951,8 +943,7 @@ key_tile_count_kernel(Geometry G, const uint32_t *__restrict__ sa, int *__restri
     const int lim = min(kRadixTile, G.n - tt * kRadixTile);
     int c = 0;
     for (int i = threadIdx.x; i < lim; i += 256) c += (int)sa[base + i] < G.T ? 1 : 0;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(ROSA_FULL_MASK, c, o);
+    c = __reduce_add_sync(ROSA_FULL_MASK, c);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -990,8 +981,7 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
             p = tt * kRadixTile;
         } else {
             for (int i = lane; i < tt; i += 32) p += ktile[(int64_t)s * G.ntps + i];
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) p += __shfl_xor_sync(ROSA_FULL_MASK, p, o);
+            p = __reduce_add_sync(ROSA_FULL_MASK, p);
         }
         if (lane == 0) pre_s = p;
     }
@@ -1034,11 +1024,8 @@ wavelet_compact_kernel(Geometry G, int nbits, const uint32_t *__restrict__ sa, c
             }
         }
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        c0 += __shfl_xor_sync(ROSA_FULL_MASK, c0, o);
-        c1 += __shfl_xor_sync(ROSA_FULL_MASK, c1, o);
-    }
+    c0 = __reduce_add_sync(ROSA_FULL_MASK, c0);
+    c1 = __reduce_add_sync(ROSA_FULL_MASK, c1);
     if (lane == 0) {
         if (c0) atomicAdd(&ones[0], c0);
         if (c1) atomicAdd(&ones[1], c1);
@@ -1075,11 +1062,8 @@ wavelet_level_kernel(Geometry G, int nbits, int lv, const uint32_t *__restrict__
         tot += c;
         if (i < tt) a += c;
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        a += __shfl_xor_sync(ROSA_FULL_MASK, a, o);
-        tot += __shfl_xor_sync(ROSA_FULL_MASK, tot, o);
-    }
+    a = __reduce_add_sync(ROSA_FULL_MASK, a);
+    tot = __reduce_add_sync(ROSA_FULL_MASK, tot);
     unsigned bal[8];
     int mine = 0;
 #pragma unroll
@@ -1523,13 +1507,9 @@ resolve_tile_kernel(Geometry G, ResolveArgs A, const uint8_t *__restrict__ vsym,
     __syncthreads();
     for (int B = warp; B < kRWin / 32; B += kRThreads / 32) {
         const int r = 32 * B + lane;
-        int kmin = w.kp[r], el = w.lc[r + 1], er = w.lc[r];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            kmin = min(kmin, __shfl_xor_sync(ROSA_FULL_MASK, kmin, o));
-            el = min(el, __shfl_xor_sync(ROSA_FULL_MASK, el, o));
-            er = min(er, __shfl_xor_sync(ROSA_FULL_MASK, er, o));
-        }
+        const int kmin = __reduce_min_sync(ROSA_FULL_MASK, w.kp[r]);
+        const int el = __reduce_min_sync(ROSA_FULL_MASK, w.lc[r + 1]);
+        const int er = __reduce_min_sync(ROSA_FULL_MASK, w.lc[r]);
         if (lane == 0) { w.bkp[B] = kmin; w.beL[B] = el; w.beR[B] = er; }
     }
     // sparse table levels, four byte entries per step with byte-wise SIMD minima
