@@ -37,7 +37,9 @@ __device__ __forceinline__ uint8_t positive_bit(uint16_t h) {
 __global__ void __launch_bounds__(kDiscThreads)
 discretize_kernel(const uint16_t *__restrict__ x0, const uint16_t *__restrict__ x1, int B, int T, int C, int M,
                   int CC, bool vec, uint8_t *__restrict__ sym0, uint8_t *__restrict__ sym1) {
-    __shared__ uint8_t bits[kDiscTT][kDiscCC];
+    // rows padded by one word: the packing phase reads a column (32 positions of
+    // one channel), which would otherwise hit a single bank 32 times
+    __shared__ uint8_t bits[kDiscTT][kDiscCC + 4];
     const int which = blockIdx.z >= (unsigned)B;
     const int b = blockIdx.z - which * B;
     const uint16_t *__restrict__ x = which ? x1 : x0;
