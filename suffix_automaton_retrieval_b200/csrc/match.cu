@@ -428,7 +428,7 @@ __device__ __forceinline__ uint64_t g0_key(uint64_t full, const Geometry &G) {
     return ((full >> G.idbits) << kAvailBits) | (uint64_t)min(p + 1, G.D0 + 1);
 }
 
-__global__ void __launch_bounds__(256, 6)
+__global__ void __launch_bounds__(256)
 groups0_kernel(const uint64_t *__restrict__ keys, uint32_t *__restrict__ sa, Geometry G, int32_t *__restrict__ rank,
                int32_t *__restrict__ lcp, int2 *small, int2 *large, int *counts_next, int32_t *__restrict__ ties,
                int *tie_count) {
@@ -776,20 +776,6 @@ __global__ void dbl_regroup_kernel(const int2 *__restrict__ small, const int2 *_
 // ---------------------------------------------------------------------------
 constexpr int kLcpSerial = 24;         // symbols past D0 one thread compares before handing off
 
-// Four symbols of a stream ending at byte address `e` (the symbol at e in the
-// top byte, e-3 in the low byte), from aligned words that lie inside
-// [lo, hi); returns false (nothing read) where they would not.
-__device__ __forceinline__ bool load4_back(const uint8_t *e, const uint8_t *lo, const uint8_t *hi, uint32_t &v) {
-    const uintptr_t a = (uintptr_t)(e - 3);
-    const uintptr_t w = a & ~(uintptr_t)3;
-    const int sh = (int)(a & 3);
-    if (w < (uintptr_t)lo || w + (sh ? 8 : 4) > (uintptr_t)hi) return false;
-    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(w);
-    const uint32_t w1 = sh ? *reinterpret_cast<const uint32_t *>(w + 4) : 0u;
-    v = __funnelshift_r(w0, w1, 8 * sh);
-    return true;
-}
-
 // Positions listed by groups0 (inside unresolved round-0 groups): their
 // neighbours share the first D0 symbols; compare onward in the final order.
 __global__ void lcp_ties_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ k, Geometry G,
@@ -807,23 +793,24 @@ __global__ void lcp_ties_kernel(const uint8_t *__restrict__ q, const uint8_t *__
         int m = G.D0;
         const int lim = min(p1, p2) + 1;
         const int stop = min(lim, G.D0 + kLcpSerial);
-        // four symbols per word while all four lie before `stop`, then symbol by symbol
-        const uint8_t *b1 = (int)x1 < G.T ? k : q, *b2 = (int)x2 < G.T ? k : q;
-        const uint8_t *e1 = b1 + (int64_t)G.S * G.T, *e2 = b2 + (int64_t)G.S * G.T;
-        for (;;) {
-            uint32_t v1, v2;
-            if (m + 3 >= stop || !load4_back(s1 + p1 - m, b1, e1, v1) || !load4_back(s2 + p2 - m, b2, e2, v2)) break;
-            const uint32_t x = v1 ^ v2;
-            if (x) {
-                m += __clz(x) >> 3;
-                break;
-            }
-            m += 4;
-        }
         while (m < stop && s1[p1 - m] == s2[p2 - m]) ++m;
         lcp[gi] = m;
         if (m == stop && m < lim) long_list[atomicAdd(long_count, 1)] = (int32_t)gi;   // still equal: a warp finishes it
     }
+}
+
+// Four symbols of a stream ending at byte address `e` (the symbol at e in the
+// top byte, e-3 in the low byte), from aligned words that lie inside
+// [lo, hi); returns false (nothing read) where they would not.
+__device__ __forceinline__ bool load4_back(const uint8_t *e, const uint8_t *lo, const uint8_t *hi, uint32_t &v) {
+    const uintptr_t a = (uintptr_t)(e - 3);
+    const uintptr_t w = a & ~(uintptr_t)3;
+    const int sh = (int)(a & 3);
+    if (w < (uintptr_t)lo || w + (sh ? 8 : 4) > (uintptr_t)hi) return false;
+    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(w);
+    const uint32_t w1 = sh ? *reinterpret_cast<const uint32_t *>(w + 4) : 0u;
+    v = __funnelshift_r(w0, w1, 8 * sh);
+    return true;
 }
 
 // Long common prefixes (repeats): one warp per pair, 4 symbols per lane and
