@@ -140,3 +140,51 @@ def test_rle_pins_catch_mutants():
         with pytest.raises(AssertionError):
             check_rle_stream(q, k, k, g, e, l, s, full=True)
             raise RuntimeError(f"mutant {name} passed the run-level checker")
+
+
+def _binary_rle_closed_form(q, k, v, g):
+    """Run-level retrieval on a binary alphabet written out from the fact the
+    GPU's binary path rests on: folded binary streams alternate, so query run m
+    shares min(m, l) + 1 runs with key run l when their symbols agree and none
+    otherwise; the answer is the last admissible key run with query run m's
+    symbol.  Independent of the oracle's code (numpy on one stream)."""
+    T = len(q)
+    def runs(a):
+        starts = [0] + [t for t in range(1, T) if a[t] != a[t - 1]]
+        run_of = np.zeros(T, np.int64)
+        for i, s in enumerate(starts):
+            run_of[s:] = i
+        return np.array(starts), run_of
+    ks, krun = runs(k)
+    qs, qrun = runs(q)
+    end = np.full(T, -1, np.int64); ln = np.zeros(T, np.int64); sym = np.full(T, -1, np.int64)
+    for t in range(T):
+        m = qrun[t]
+        p = qs[m] - g + 1                 # the next key run must start by here
+        if p < 0:
+            continue
+        X = krun[p] - 1                   # last admissible key run
+        if X < 0:
+            continue
+        l = X if k[ks[X]] == q[qs[m]] else X - 1
+        if l < 0:
+            continue
+        end[t] = ks[l + 1] - 1
+        ln[t] = min(l, m) + 1
+        sym[t] = v[ks[l + 1]]
+    return end, ln, sym
+
+
+def test_rle_binary_closed_form_matches_the_definition():
+    rng = np.random.default_rng(2024)
+    for trial in range(300):
+        T = int(rng.integers(1, 160))
+        r = int(rng.choice([1, 2, 4]))
+        q = np.repeat(rng.integers(0, 2, T), rng.integers(1, r + 1, T))[:T].astype(np.uint8)
+        k = q if rng.random() < 0.3 else np.repeat(rng.integers(0, 2, T), rng.integers(1, r + 1, T))[:T].astype(np.uint8)
+        v = k if rng.random() < 0.5 else rng.integers(0, 256, T).astype(np.uint8)
+        g = int(rng.integers(1, 4))
+        want = oracle.match_rle_brute(q[None], k[None], v[None], g=g)
+        got = _binary_rle_closed_form(q, k, v, g)
+        for name, a, b in zip(("end", "len", "sym"), got, want):
+            assert np.array_equal(a, b[0]), (trial, name, T, g, q.tolist(), k.tolist())
