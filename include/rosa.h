@@ -277,8 +277,13 @@ ROSA_API int rosa_ln_project_discretize(const rosa_bf16 *H, const float *gamma, 
  *     inj[b, t, d] = bf16(sum_c W_out[d, c] * y[b, t, c])  (fp32 accumulation)
  * dev_status: optional device word; ROSA_DEV_TIMEOUT is or-ed into it if a
  * kernel's bounded wait ran out (the affected tiles are not written).
- * Requires B, T >= 0, 1 <= M <= 8, R >= 1, D >= 1; any alignment (rows of
- * W_out that are 16-byte aligned take the vector path).
+ * Requires B, T >= 0, 1 <= M <= 8, R >= 1, D >= 1; any alignment.  W_out
+ * arrives by TMA when C >= 64, C % 8 == 0 and W_out is 16-byte aligned, and
+ * inj leaves by TMA stores when D >= 64, D % 8 == 0 and inj is 16-byte
+ * aligned; other shapes take plain loads and stores.  With C <= 512 the call
+ * runs persistent CTAs that each hold 256 of an SM's 512 tensor-memory
+ * columns until they finish (a kernel that holds tensor memory on the same
+ * SMs delays them).
  */
 ROSA_API int rosa_inject(const int32_t *sym, const rosa_bf16 *e0, const rosa_bf16 *e1, const rosa_bf16 *W_out,
                          int B, int R, int M, int T, int D, rosa_bf16 *inj, uint32_t *dev_status,
