@@ -228,3 +228,34 @@ def test_workload_streams_of_a_shard():
     assert bench.workload_streams({"S": 512, "R": 256, "shard": {"batches": [2, 4], "of": 8}}) == 2048
     assert bench.workload_streams({"S": 32, "R": 32, "shard": {"routes": [32, 64], "of": 64}}) == 64
     assert bench.workload_streams({"S": 64, "R": 64}) == 64
+
+
+def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
+    """`traffic` comes from a DRAM capture of the match call; it is reported only
+    while the matcher's sources still have the digest the capture was taken on."""
+    nbytes, digest = bench.PROFILED_DRAM_BYTES["zipf-256-131k"]
+    assert nbytes > 234881024                       # more than the call's algorithmic bytes
+    monkeypatch.setattr(bench, "cuda_source_digest", lambda files=bench.MATCH_SOURCES: digest)
+    assert bench.profiled_traffic("zipf-256-131k", "match") == nbytes
+    assert bench.profiled_traffic("zipf-256-131k", "gather") is None
+    assert bench.profiled_traffic("markov-4-train", "match") is None
+    monkeypatch.setattr(bench, "cuda_source_digest", lambda files=bench.MATCH_SOURCES: "0" * 16)
+    assert bench.profiled_traffic("zipf-256-131k", "match") is None
+
+
+def test_match_source_digest_tracks_the_matcher_only(tmp_path, monkeypatch):
+    """The digest covers the matcher's sources, so edits elsewhere (the dense
+    kernels) keep the match traffic valid while edits to the matcher void it."""
+    import shutil
+    csrc = os.path.join(ROOT, "suffix_automaton_retrieval_b200", "csrc")
+    fake = tmp_path / "suffix_automaton_retrieval_b200" / "csrc"
+    fake.mkdir(parents=True)
+    for name in os.listdir(csrc):
+        if name.endswith((".cu", ".cuh", ".h")):
+            shutil.copy(os.path.join(csrc, name), fake / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d0 = bench.cuda_source_digest()
+    (fake / "inject.cu").write_text((fake / "inject.cu").read_text() + "\n// edit\n")
+    assert bench.cuda_source_digest() == d0
+    (fake / "match.cu").write_text((fake / "match.cu").read_text() + "\n// edit\n")
+    assert bench.cuda_source_digest() != d0
